@@ -1,0 +1,116 @@
+// Shared device helpers of libcsa: element conversion, the per-device status
+// word, and the mapping from a query row to its visible compressed entries.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace csa {
+
+// ---------------------------------------------------------------- status word
+// Error bits recorded by kernels instead of faulting; read (and cleared) by
+// csa_get_device_status().
+enum : unsigned {
+  kStatusTimeout = 1u,   // a bounded wait gave up
+  kStatusBadIndex = 2u,  // an out-of-range block index was skipped
+  kStatusMetadata = 4u,  // cu_seqlens / cu_blocks / cache_len inconsistent
+};
+
+__device__ unsigned g_status;
+
+__device__ __forceinline__ void flag_status(unsigned bits) { atomicOr(&g_status, bits); }
+
+// ---------------------------------------------------------------- conversions
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// 16-byte vector of V elements of T (V = 4 for fp32, 8 for bf16).
+template <typename T> struct Vec16 {
+  static constexpr int V = 16 / sizeof(T);
+  union {
+    uint4 u;
+    T e[V];
+  };
+};
+
+template <typename T>
+__device__ __forceinline__ void load_vec_f32(const T* p, float* out) {
+  Vec16<T> v;
+  v.u = *reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < Vec16<T>::V; ++i) out[i] = to_f32(v.e[i]);
+}
+
+template <typename T>
+__device__ __forceinline__ void store_vec_f32(T* p, const float* in) {
+  Vec16<T> v;
+#pragma unroll
+  for (int i = 0; i < Vec16<T>::V; ++i) v.e[i] = from_f32<T>(in[i]);
+  *reinterpret_cast<uint4*>(p) = v.u;
+}
+
+// Map an fp32 score to an unsigned key whose unsigned order is the float
+// order (-0 is folded onto +0 first so that equal scores get equal keys).
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  f = f + 0.0f;
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------- rows
+// Where the compressed entries visible to one query row live.  Prefill rows
+// are packed sequences (cu_seqlens / cu_blocks); decode rows are one token of
+// sequence b over that sequence's cache of capacity `cap`.
+struct RowMap {
+  const int* cu_seqlens;  // prefill: [nseq+1]
+  const int* cu_blocks;   // prefill: [nseq+1]
+  int nseq;
+  int total_blocks;
+  const int* pos;         // decode: [B] token index of the new token
+  int cap;                // decode: cache capacity per sequence (0 = prefill)
+  int m;
+};
+
+// Visible entries of `row`: global entry index of block 0 and the count
+// floor(t/m).  Inconsistent metadata is flagged and clamped so that no access
+// leaves [0, total entries).
+__device__ __forceinline__ void row_entries(const RowMap& rm, int row, long long& base, int& avail) {
+  if (rm.cap > 0) {
+    int t = rm.pos[row];
+    int a = t >= 0 ? t / rm.m : 0;
+    if (a > rm.cap) {
+      flag_status(kStatusMetadata);
+      a = rm.cap;
+    }
+    base = (long long)row * rm.cap;
+    avail = a;
+    return;
+  }
+  int lo = 0, hi = rm.nseq;  // find the sequence: cu_seqlens[lo] <= row < cu_seqlens[lo+1]
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (rm.cu_seqlens[mid] <= row) lo = mid; else hi = mid;
+  }
+  int t = row - rm.cu_seqlens[lo];
+  int a = t / rm.m;
+  int b0 = rm.cu_blocks[lo], b1 = rm.cu_blocks[lo + 1];
+  if (b0 < 0 || b0 + a > b1 || b1 > rm.total_blocks) {
+    flag_status(kStatusMetadata);
+    b0 = max(0, min(b0, rm.total_blocks));
+    a = max(0, min(a, rm.total_blocks - b0));
+  }
+  base = b0;
+  avail = a;
+}
+
+}  // namespace csa

@@ -1,0 +1,595 @@
+// libcsa: the C ABI of include/csa.h.  Host code here validates arguments,
+// carves the caller's workspace and enqueues the kernels of the other files
+// of this directory on the caller's stream; every step of the path is one of
+// those kernels.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "../../include/csa.h"
+#include "common.cuh"
+#include "compress.cuh"
+#include "gemm_simt.cuh"
+#include "indexer_simt.cuh"
+#include "mqa_simt.cuh"
+#include "pack.cuh"
+
+using namespace csa;
+using bf16 = __nv_bfloat16;
+
+namespace {
+
+constexpr size_t kAlign = 1024;     // internal sub-buffer alignment
+constexpr size_t kPtrAlign = 256;   // required alignment of caller buffers
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+inline int round_up_int(int x, int a) { return (x + a - 1) / a * a; }
+
+std::atomic<uint64_t> g_launches{0};
+
+// Follows every kernel launch: counts it and maps a launch error.
+#define CSA_CHECK_LAUNCH()                                      \
+  do {                                                          \
+    g_launches.fetch_add(1, std::memory_order_relaxed);         \
+    if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA; \
+  } while (0)
+
+size_t elem_size(const csa_dims* d) { return d->dtype == CSA_BF16 ? 2 : 4; }
+
+// Host-side shape checks shared by every entry point.
+csa_status check_dims(const csa_dims* d) {
+  if (!d) return CSA_ERR_INVALID_ARG;
+  if (d->d <= 0 || d->c <= 0 || d->m <= 0 || d->cI <= 0 || d->nhI <= 0 || d->nh <= 0 ||
+      d->dc <= 0 || d->topk <= 0)
+    return CSA_ERR_INVALID_ARG;
+  if (d->dtype != CSA_F32 && d->dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  if (d->m != 1 && d->m != 2 && d->m != 4 && d->m != 8) return CSA_ERR_UNSUPPORTED;
+  if (d->c != 64 && d->c != 128 && d->c != 256 && d->c != 512 && d->c != 1024) return CSA_ERR_UNSUPPORTED;
+  if (d->cI != 32 && d->cI != 64 && d->cI != 128) return CSA_ERR_UNSUPPORTED;
+  const int v = d->dtype == CSA_BF16 ? 8 : 4;  // elements per 16-byte vector
+  if (d->dc % v || d->d % v) return CSA_ERR_UNSUPPORTED;
+  if (d->topk > 8192) return CSA_ERR_UNSUPPORTED;
+  if ((size_t)d->nhI * d->cI > 16384) return CSA_ERR_UNSUPPORTED;
+  return CSA_OK;
+}
+
+// ------------------------------------------------------------------ layouts
+struct PackLayout {
+  int N1b;    // bf16/f32 block of the H-side output: C^a C^b Z^a Z^b C^aI C^bI Z^aI Z^bI c^Q
+  int N1;     // N1b + nhI (w^I columns)
+  int N1p;    // N1 padded to the tile
+  int N2;     // nhI*cI + nh*c
+  int N2p;
+  size_t w1, w2, ba, bb, baI, bbI, total;
+};
+
+PackLayout pack_layout(const csa_dims* d) {
+  PackLayout L;
+  const size_t es = elem_size(d);
+  L.N1b = 4 * d->c + 4 * d->cI + d->dc;
+  L.N1 = L.N1b + d->nhI;
+  L.N1p = round_up_int(L.N1, 256);
+  L.N2 = d->nhI * d->cI + d->nh * d->c;
+  L.N2p = round_up_int(L.N2, 256);
+  size_t off = 0;
+  L.w1 = off; off = align_up(off + (size_t)L.N1p * d->d * es);
+  L.w2 = off; off = align_up(off + (size_t)L.N2p * d->dc * es);
+  L.ba = off; off = align_up(off + (size_t)d->m * d->c * 4);
+  L.bb = off; off = align_up(off + (size_t)d->m * d->c * 4);
+  L.baI = off; off = align_up(off + (size_t)d->m * d->cI * 4);
+  L.bbI = off; off = align_up(off + (size_t)d->m * d->cI * 4);
+  L.total = off;
+  return L;
+}
+
+struct FwdLayout {
+  size_t y1, wI, y2, ccomp, kicomp, idx, total;
+};
+
+FwdLayout fwd_layout(const csa_dims* d, int T) {
+  const PackLayout P = pack_layout(d);
+  const size_t es = elem_size(d);
+  const size_t nbmax = (size_t)(T / d->m);
+  FwdLayout L;
+  size_t off = 0;
+  L.y1 = off; off = align_up(off + (size_t)T * P.N1b * es);
+  L.wI = off; off = align_up(off + (size_t)T * d->nhI * 4);
+  L.y2 = off; off = align_up(off + (size_t)T * P.N2 * es);
+  L.ccomp = off; off = align_up(off + nbmax * d->c * es);
+  L.kicomp = off; off = align_up(off + nbmax * d->cI * es);
+  L.idx = off; off = align_up(off + (size_t)T * d->topk * 4);
+  L.total = off;
+  return L;
+}
+
+inline char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
+
+// ------------------------------------------------------------------ launchers
+csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const void* B, long long ldb,
+                       int M, int N, int K, const GemmOut& out, cudaStream_t st) {
+  if (M == 0) return CSA_OK;
+  SimtGemmArgs g{A, lda, B, ldb, M, N, K, out};
+  dim3 grid((N + 127) / 128, (M + 127) / 128);
+  if (d->dtype == CSA_BF16) gemm_simt_kernel<bf16><<<grid, 256, 0, st>>>(g);
+  else gemm_simt_kernel<float><<<grid, 256, 0, st>>>(g);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+template <typename T, int M>
+void compress_launch(const CompressArgs& a, long long items, cudaStream_t st) {
+  long long blocks = (items + 255) / 256;
+  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  if (blocks < 1) blocks = 1;
+  compress_kernel<T, M><<<(unsigned)blocks, 256, 0, st>>>(a);
+}
+
+csa_status launch_compress(const csa_dims* d, const CompressArgs& a, cudaStream_t st) {
+  const long long items = (long long)a.total_blocks * a.vecs_total;
+  if (items == 0) return CSA_OK;
+#define CSA_COMPRESS_CASE(MM)                                              \
+  case MM:                                                                 \
+    if (d->dtype == CSA_BF16) compress_launch<bf16, MM>(a, items, st);     \
+    else compress_launch<float, MM>(a, items, st);                         \
+    break;
+  switch (d->m) {
+    CSA_COMPRESS_CASE(1)
+    CSA_COMPRESS_CASE(2)
+    CSA_COMPRESS_CASE(4)
+    CSA_COMPRESS_CASE(8)
+    default: return CSA_ERR_UNSUPPORTED;
+  }
+#undef CSA_COMPRESS_CASE
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+size_t indexer_smem(const csa_dims* d, int sc_cap) {
+  return (size_t)(d->nhI * d->cI + d->nhI) * 4 + 256 * 4 + 40 * 4 + (size_t)sc_cap * 4;
+}
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+template <typename T, int CI>
+csa_status indexer_launch(const IndexerArgs& a, int rows, size_t smem, cudaStream_t st) {
+  auto k = indexer_topk_simt_kernel<T, CI>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return CSA_ERR_CUDA;
+  k<<<rows, 256, smem, st>>>(a);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+csa_status launch_indexer(const csa_dims* d, const IndexerArgs& a, int rows, cudaStream_t st) {
+  if (rows == 0) return CSA_OK;
+  const size_t smem = indexer_smem(d, a.sc_cap);
+  if (smem > kMaxSmem) return CSA_ERR_UNSUPPORTED;
+  const bool b = d->dtype == CSA_BF16;
+  switch (d->cI) {
+    case 32: return b ? indexer_launch<bf16, 32>(a, rows, smem, st) : indexer_launch<float, 32>(a, rows, smem, st);
+    case 64: return b ? indexer_launch<bf16, 64>(a, rows, smem, st) : indexer_launch<float, 64>(a, rows, smem, st);
+    case 128: return b ? indexer_launch<bf16, 128>(a, rows, smem, st) : indexer_launch<float, 128>(a, rows, smem, st);
+  }
+  return CSA_ERR_UNSUPPORTED;
+}
+
+template <typename T, int VEC>
+csa_status mqa_launch(const MqaArgs& a, int rows, cudaStream_t st) {
+  const size_t smem = (size_t)a.topk * 4;
+  auto k = mqa_simt_kernel<T, VEC>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return CSA_ERR_CUDA;
+  k<<<rows, 256, smem, st>>>(a);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+csa_status launch_mqa(const csa_dims* d, const MqaArgs& a, int rows, cudaStream_t st) {
+  if (rows == 0) return CSA_OK;
+  const bool b = d->dtype == CSA_BF16;
+  switch (d->c / 32) {
+    case 2: return b ? mqa_launch<bf16, 2>(a, rows, st) : mqa_launch<float, 2>(a, rows, st);
+    case 4: return b ? mqa_launch<bf16, 4>(a, rows, st) : mqa_launch<float, 4>(a, rows, st);
+    case 8: return b ? mqa_launch<bf16, 8>(a, rows, st) : mqa_launch<float, 8>(a, rows, st);
+    case 16: return b ? mqa_launch<bf16, 16>(a, rows, st) : mqa_launch<float, 16>(a, rows, st);
+    case 32: return b ? mqa_launch<bf16, 32>(a, rows, st) : mqa_launch<float, 32>(a, rows, st);
+  }
+  return CSA_ERR_UNSUPPORTED;
+}
+
+// A1: eqs. (1), (2), (5), (7) and the indexer-key projections, one GEMM
+csa_status project_hidden(const csa_dims* d, const void* packed, const void* H, int T, void* Y1, float* wI,
+                          cudaStream_t st) {
+  const PackLayout P = pack_layout(d);
+  GemmOut o;
+  memset(&o, 0, sizeof(o));
+  o.seg[0] = {0, P.N1b, Y1, P.N1b, 0};
+  o.seg[1] = {P.N1b, d->nhI, wI, d->nhI, 1};
+  o.nseg = 2;
+  return launch_gemm(d, H, d->d, at((void*)packed, P.w1), d->d, T, P.N1, d->d, o, st);
+}
+
+// A2: eqs. (6), (10) from the shared c^Q
+csa_status project_query(const csa_dims* d, const void* packed, const void* cQ, long long ld_cQ, int T,
+                         void* Y2, cudaStream_t st) {
+  const PackLayout P = pack_layout(d);
+  GemmOut o;
+  memset(&o, 0, sizeof(o));
+  o.seg[0] = {0, P.N2, Y2, P.N2, 0};
+  o.nseg = 1;
+  return launch_gemm(d, cQ, ld_cQ, at((void*)packed, P.w2), d->dc, T, P.N2, d->dc, o, st);
+}
+
+CompressArgs make_compress_args(const csa_dims* d, const int* cu_seqlens, const int* cu_blocks,
+                                int nseq, int T, int NB) {
+  CompressArgs a;
+  memset(&a, 0, sizeof(a));
+  a.cu_seqlens = cu_seqlens;
+  a.cu_blocks = cu_blocks;
+  a.nseq = nseq;
+  a.total_tokens = T;
+  a.total_blocks = NB;
+  return a;
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+extern "C" {
+
+const char* csa_status_string(csa_status s) {
+  switch (s) {
+    case CSA_OK: return "ok";
+    case CSA_ERR_INVALID_ARG: return "invalid argument";
+    case CSA_ERR_UNSUPPORTED: return "unsupported shape or configuration";
+    case CSA_ERR_CUDA: return "CUDA runtime error";
+    case CSA_ERR_DEVICE_TIMEOUT: return "a bounded device wait ran out";
+    case CSA_ERR_BAD_INDEX: return "out-of-range block index seen on the device";
+    case CSA_ERR_BAD_METADATA: return "inconsistent cu_seqlens / cu_blocks / cache metadata";
+    case CSA_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+csa_status csa_get_device_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return CSA_ERR_CUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return CSA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return CSA_ERR_CUDA;
+  if (v & kStatusTimeout) return CSA_ERR_DEVICE_TIMEOUT;
+  if (v & kStatusBadIndex) return CSA_ERR_BAD_INDEX;
+  if (v & kStatusMetadata) return CSA_ERR_BAD_METADATA;
+  return CSA_OK;
+}
+
+uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int csa_hidden_row_elems(const csa_dims* d) {
+  if (check_dims(d) != CSA_OK) return 0;
+  return pack_layout(d).N1b;
+}
+
+int csa_query_row_elems(const csa_dims* d) {
+  if (check_dims(d) != CSA_OK) return 0;
+  return pack_layout(d).N2;
+}
+
+csa_status csa_project_hidden(const csa_dims* d, const void* packed, const void* H, int T, void* Y1, float* wI,
+                              void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!packed || !H || !Y1 || !wI || T < 0) return CSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(packed) % kPtrAlign) return CSA_ERR_INVALID_ARG;
+  return project_hidden(d, packed, H, T, Y1, wI, (cudaStream_t)stream);
+}
+
+csa_status csa_project_query(const csa_dims* d, const void* packed, const void* cQ, int ld_cQ, int T, void* Y2,
+                             void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!packed || !cQ || !Y2 || T < 0 || ld_cQ < d->dc) return CSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(packed) % kPtrAlign) return CSA_ERR_INVALID_ARG;
+  return project_query(d, packed, cQ, ld_cQ, T, Y2, (cudaStream_t)stream);
+}
+
+size_t csa_packed_weights_bytes(const csa_dims* d) {
+  if (check_dims(d) != CSA_OK) return 0;
+  return pack_layout(d).total;
+}
+
+csa_status csa_pack_weights(const csa_dims* d, const csa_weights* w, void* packed, size_t packed_bytes,
+                            void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!w || !packed) return CSA_ERR_INVALID_ARG;
+  const void* all[] = {w->W_aKV, w->W_bKV, w->W_aZ, w->W_bZ, w->B_a, w->B_b, w->W_aKV_I, w->W_bKV_I,
+                       w->W_aZ_I, w->W_bZ_I, w->B_a_I, w->B_b_I, w->W_DQ, w->W_IUQ, w->W_UQ, w->W_w};
+  for (const void* p : all)
+    if (!p) return CSA_ERR_INVALID_ARG;
+  const PackLayout P = pack_layout(d);
+  if (packed_bytes < P.total) return CSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(packed) % kPtrAlign) return CSA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemsetAsync(packed, 0, P.total, st) != cudaSuccess) return CSA_ERR_CUDA;
+  const size_t es = elem_size(d);
+  // H-side: rows of W1t in the order of the GEMM's output columns
+  struct Part { const void* W; int in, out; char* dst; long long ld; };
+  char* w1 = at(packed, P.w1);
+  char* w2 = at(packed, P.w2);
+  const int c = d->c, cI = d->cI;
+  long long r1 = 0;
+  auto row1 = [&](int n) { char* p = w1 + r1 * d->d * es; r1 += n; return p; };
+  Part parts[16];
+  int np = 0;
+  parts[np++] = {w->W_aKV, d->d, c, row1(c), d->d};
+  parts[np++] = {w->W_bKV, d->d, c, row1(c), d->d};
+  parts[np++] = {w->W_aZ, d->d, c, row1(c), d->d};
+  parts[np++] = {w->W_bZ, d->d, c, row1(c), d->d};
+  parts[np++] = {w->W_aKV_I, d->d, cI, row1(cI), d->d};
+  parts[np++] = {w->W_bKV_I, d->d, cI, row1(cI), d->d};
+  parts[np++] = {w->W_aZ_I, d->d, cI, row1(cI), d->d};
+  parts[np++] = {w->W_bZ_I, d->d, cI, row1(cI), d->d};
+  parts[np++] = {w->W_DQ, d->d, d->dc, row1(d->dc), d->d};
+  parts[np++] = {w->W_w, d->d, d->nhI, row1(d->nhI), d->d};
+  parts[np++] = {w->W_IUQ, d->dc, d->nhI * cI, w2, d->dc};
+  parts[np++] = {w->W_UQ, d->dc, d->nh * c, w2 + (size_t)d->nhI * cI * d->dc * es, d->dc};
+  for (int i = 0; i < np; ++i) {
+    const Part& p = parts[i];
+    dim3 grid((p.out + 31) / 32, (p.in + 31) / 32), block(32, 8);
+    if (d->dtype == CSA_BF16)
+      transpose_kernel<bf16><<<grid, block, 0, st>>>(static_cast<const bf16*>(p.W), p.in, p.out,
+                                                     reinterpret_cast<bf16*>(p.dst), p.ld);
+    else
+      transpose_kernel<float><<<grid, block, 0, st>>>(static_cast<const float*>(p.W), p.in, p.out,
+                                                      reinterpret_cast<float*>(p.dst), p.ld);
+    CSA_CHECK_LAUNCH();
+  }
+  struct Bias { const void* src; size_t off; long long n; };
+  const Bias biases[4] = {{w->B_a, P.ba, (long long)d->m * c}, {w->B_b, P.bb, (long long)d->m * c},
+                          {w->B_a_I, P.baI, (long long)d->m * cI}, {w->B_b_I, P.bbI, (long long)d->m * cI}};
+  for (const Bias& b : biases) {
+    float* dst = reinterpret_cast<float*>(at(packed, b.off));
+    if (d->dtype == CSA_BF16) widen_kernel<bf16><<<64, 256, 0, st>>>(static_cast<const bf16*>(b.src), dst, b.n);
+    else widen_kernel<float><<<64, 256, 0, st>>>(static_cast<const float*>(b.src), dst, b.n);
+    CSA_CHECK_LAUNCH();
+  }
+  return CSA_OK;
+}
+
+csa_status csa_compress(const csa_dims* d, const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                        int ld, const float* Ba, const float* Bb, int width, const int* cu_seqlens,
+                        const int* cu_blocks, int nseq, int total_tokens, int total_blocks, void* out,
+                        void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!Ca || !Cb || !Za || !Zb || !Ba || !Bb || !cu_seqlens || !cu_blocks || !out) return CSA_ERR_INVALID_ARG;
+  if (nseq <= 0 || total_tokens < 0 || total_blocks < 0 || width <= 0 || ld < width) return CSA_ERR_INVALID_ARG;
+  if (total_blocks > total_tokens / d->m) return CSA_ERR_INVALID_ARG;
+  const int v = 16 / (int)elem_size(d);
+  if (width % v || ld % v) return CSA_ERR_UNSUPPORTED;
+  for (const void* p : {Ca, Cb, Za, Zb, (const void*)Ba, (const void*)Bb, (const void*)out})
+    if (reinterpret_cast<uintptr_t>(p) % 16) return CSA_ERR_UNSUPPORTED;
+  CompressArgs a = make_compress_args(d, cu_seqlens, cu_blocks, nseq, total_tokens, total_blocks);
+  a.seg[0] = {Ca, Cb, Za, Zb, ld, Ba, Bb, width, out};
+  a.nseg = 1;
+  a.vecs0 = width / v;
+  a.vecs_total = a.vecs0;
+  return launch_compress(d, a, (cudaStream_t)stream);
+}
+
+csa_status csa_indexer_topk(const csa_dims* d, const void* qI, int ld_qI, const float* wI, int ld_wI,
+                            const void* KI, const int* cu_seqlens, const int* cu_blocks, int nseq,
+                            int total_tokens, int total_blocks, int max_seqlen, int* idx, void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!qI || !wI || !KI || !cu_seqlens || !cu_blocks || !idx) return CSA_ERR_INVALID_ARG;
+  if (nseq <= 0 || total_tokens < 0 || total_blocks < 0 || max_seqlen < 0) return CSA_ERR_INVALID_ARG;
+  if (ld_qI < d->nhI * d->cI || ld_wI < d->nhI) return CSA_ERR_INVALID_ARG;
+  const int v = 16 / (int)elem_size(d);
+  if (ld_qI % v || reinterpret_cast<uintptr_t>(KI) % 16) return CSA_ERR_UNSUPPORTED;
+  IndexerArgs a;
+  a.qI = qI; a.ld_qI = ld_qI; a.wI = wI; a.ld_wI = ld_wI; a.KI = KI; a.idx = idx;
+  a.topk = d->topk; a.nhI = d->nhI;
+  a.sc_cap = max_seqlen / d->m;
+  a.rm = RowMap{cu_seqlens, cu_blocks, nseq, total_blocks, nullptr, 0, d->m};
+  return launch_indexer(d, a, total_tokens, (cudaStream_t)stream);
+}
+
+csa_status csa_sparse_mqa(const csa_dims* d, const void* q, int ld_q, const void* Ccomp, const int* idx,
+                          const int* cu_seqlens, const int* cu_blocks, int nseq, int total_tokens,
+                          int total_blocks, void* O, void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!q || !Ccomp || !idx || !cu_seqlens || !cu_blocks || !O) return CSA_ERR_INVALID_ARG;
+  if (nseq <= 0 || total_tokens < 0 || total_blocks < 0 || ld_q < d->nh * d->c) return CSA_ERR_INVALID_ARG;
+  const int v = 16 / (int)elem_size(d);
+  if (ld_q % v) return CSA_ERR_UNSUPPORTED;
+  MqaArgs a;
+  a.q = q; a.ld_q = ld_q; a.C = Ccomp; a.idx = idx; a.O = O; a.ld_O = (long long)d->nh * d->c;
+  a.topk = d->topk; a.nh = d->nh;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d->c));
+  a.rm = RowMap{cu_seqlens, cu_blocks, nseq, total_blocks, nullptr, 0, d->m};
+  return launch_mqa(d, a, total_tokens, (cudaStream_t)stream);
+}
+
+size_t csa_forward_workspace_bytes(const csa_dims* d, int total_tokens, int nseq) {
+  if (check_dims(d) != CSA_OK || total_tokens < 0 || nseq <= 0) return 0;
+  return fwd_layout(d, total_tokens).total;
+}
+
+csa_status csa_forward(const csa_dims* d, const void* packed, const void* H, const int* cu_seqlens,
+                       const int* cu_blocks, int nseq, int total_tokens, int total_blocks, int max_seqlen,
+                       void* O, void* Ccomp_out, void* KI_out, int* idx_out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!packed || !H || !cu_seqlens || !cu_blocks || !O || !ws) return CSA_ERR_INVALID_ARG;
+  if (nseq <= 0 || total_tokens < 0 || total_blocks < 0 || max_seqlen < 0) return CSA_ERR_INVALID_ARG;
+  if (total_blocks > total_tokens / d->m) return CSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % kPtrAlign || reinterpret_cast<uintptr_t>(packed) % kPtrAlign)
+    return CSA_ERR_INVALID_ARG;
+  for (const void* p : {H, (const void*)O, (const void*)Ccomp_out, (const void*)KI_out})
+    if (reinterpret_cast<uintptr_t>(p) % 16) return CSA_ERR_INVALID_ARG;
+  const int T = total_tokens, NB = total_blocks;
+  const FwdLayout L = fwd_layout(d, T);
+  if (ws_bytes < L.total) return CSA_ERR_WORKSPACE;
+  if (T == 0) return CSA_OK;
+  const PackLayout P = pack_layout(d);
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t es = elem_size(d);
+  const int c = d->c, cI = d->cI;
+  char* y1 = at(ws, L.y1);
+  float* wI = reinterpret_cast<float*>(at(ws, L.wI));
+  char* y2 = at(ws, L.y2);
+  void* Cc = Ccomp_out ? Ccomp_out : at(ws, L.ccomp);
+  void* KIc = KI_out ? KI_out : at(ws, L.kicomp);
+  int* idx = idx_out ? idx_out : reinterpret_cast<int*>(at(ws, L.idx));
+
+  s = project_hidden(d, packed, H, T, y1, wI, st);
+  if (s != CSA_OK) return s;
+  s = project_query(d, packed, y1 + (size_t)(4 * c + 4 * cI) * es, P.N1b, T, y2, st);
+  if (s != CSA_OK) return s;
+  // A3: eqs. (3), (4) for C^Comp and K^IComp in one launch
+  CompressArgs ca = make_compress_args(d, cu_seqlens, cu_blocks, nseq, T, NB);
+  ca.seg[0] = {y1, y1 + (size_t)c * es, y1 + (size_t)2 * c * es, y1 + (size_t)3 * c * es, P.N1b,
+               reinterpret_cast<const float*>(at((void*)packed, P.ba)),
+               reinterpret_cast<const float*>(at((void*)packed, P.bb)), c, Cc};
+  char* yI = y1 + (size_t)4 * c * es;
+  ca.seg[1] = {yI, yI + (size_t)cI * es, yI + (size_t)2 * cI * es, yI + (size_t)3 * cI * es, P.N1b,
+               reinterpret_cast<const float*>(at((void*)packed, P.baI)),
+               reinterpret_cast<const float*>(at((void*)packed, P.bbI)), cI, KIc};
+  ca.nseg = 2;
+  const int v = 16 / (int)es;
+  ca.vecs0 = c / v;
+  ca.vecs_total = (c + cI) / v;
+  s = launch_compress(d, ca, st);
+  if (s != CSA_OK) return s;
+  // A4: eqs. (8), (9)
+  IndexerArgs ia;
+  ia.qI = y2; ia.ld_qI = P.N2; ia.wI = wI; ia.ld_wI = d->nhI; ia.KI = KIc; ia.idx = idx;
+  ia.topk = d->topk; ia.nhI = d->nhI; ia.sc_cap = max_seqlen / d->m;
+  ia.rm = RowMap{cu_seqlens, cu_blocks, nseq, NB, nullptr, 0, d->m};
+  s = launch_indexer(d, ia, T, st);
+  if (s != CSA_OK) return s;
+  // A5: eq. (11)
+  MqaArgs ma;
+  ma.q = y2 + (size_t)d->nhI * cI * es; ma.ld_q = P.N2; ma.C = Cc; ma.idx = idx;
+  ma.O = O; ma.ld_O = (long long)d->nh * c; ma.topk = d->topk; ma.nh = d->nh;
+  ma.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c));
+  ma.rm = RowMap{cu_seqlens, cu_blocks, nseq, NB, nullptr, 0, d->m};
+  return launch_mqa(d, ma, T, st);
+}
+
+// ------------------------------------------------------------------ decode
+int csa_ring_row_elems(const csa_dims* d) {
+  if (check_dims(d) != CSA_OK) return 0;
+  return 4 * d->c + 4 * d->cI;
+}
+
+namespace {
+csa_status launch_append(const csa_dims* d, const void* packed, const void* rows, long long ld_rows,
+                         const int* pos, void* ring, void* Ccache, void* KIcache, int* cache_len, int cap,
+                         int B, cudaStream_t st) {
+  if (B == 0) return CSA_OK;
+  const PackLayout P = pack_layout(d);
+  AppendArgs a;
+  a.rows = rows; a.ld_rows = ld_rows; a.pos = pos; a.ring = ring; a.Ccache = Ccache; a.KIcache = KIcache;
+  a.cache_len = cache_len;
+  a.Ba = reinterpret_cast<const float*>(at((void*)packed, P.ba));
+  a.Bb = reinterpret_cast<const float*>(at((void*)packed, P.bb));
+  a.BaI = reinterpret_cast<const float*>(at((void*)packed, P.baI));
+  a.BbI = reinterpret_cast<const float*>(at((void*)packed, P.bbI));
+  a.c = d->c; a.cI = d->cI; a.cap = cap; a.ring_w = 4 * d->c + 4 * d->cI;
+#define CSA_APPEND_CASE(MM)                                                     \
+  case MM:                                                                      \
+    if (d->dtype == CSA_BF16) cache_append_kernel<bf16, MM><<<B, 256, 0, st>>>(a); \
+    else cache_append_kernel<float, MM><<<B, 256, 0, st>>>(a);                  \
+    break;
+  switch (d->m) {
+    CSA_APPEND_CASE(1)
+    CSA_APPEND_CASE(2)
+    CSA_APPEND_CASE(4)
+    CSA_APPEND_CASE(8)
+    default: return CSA_ERR_UNSUPPORTED;
+  }
+#undef CSA_APPEND_CASE
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+struct DecLayout {
+  size_t y1, wI, y2, idx, total;
+};
+DecLayout dec_layout(const csa_dims* d, int B) {
+  const PackLayout P = pack_layout(d);
+  const size_t es = elem_size(d);
+  DecLayout L;
+  size_t off = 0;
+  L.y1 = off; off = align_up(off + (size_t)B * P.N1b * es);
+  L.wI = off; off = align_up(off + (size_t)B * d->nhI * 4);
+  L.y2 = off; off = align_up(off + (size_t)B * P.N2 * es);
+  L.idx = off; off = align_up(off + (size_t)B * d->topk * 4);
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+csa_status csa_cache_append(const csa_dims* d, const void* packed, const void* rows, const int* pos,
+                            void* ring, void* Ccache, void* KIcache, int* cache_len, int cap, int B,
+                            void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!packed || !rows || !pos || !ring || !Ccache || !KIcache || !cache_len) return CSA_ERR_INVALID_ARG;
+  if (cap <= 0 || B < 0) return CSA_ERR_INVALID_ARG;
+  return launch_append(d, packed, rows, 4 * d->c + 4 * d->cI, pos, ring, Ccache, KIcache, cache_len, cap, B,
+                       (cudaStream_t)stream);
+}
+
+size_t csa_decode_workspace_bytes(const csa_dims* d, int B) {
+  if (check_dims(d) != CSA_OK || B < 0) return 0;
+  return dec_layout(d, B).total;
+}
+
+csa_status csa_decode(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
+                      void* Ccache, void* KIcache, int* cache_len, int cap, int B, void* O, int* idx_out,
+                      void* ws, size_t ws_bytes, void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!packed || !h || !pos || !ring || !Ccache || !KIcache || !cache_len || !O || !ws) return CSA_ERR_INVALID_ARG;
+  if (cap <= 0 || B < 0) return CSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % kPtrAlign || reinterpret_cast<uintptr_t>(packed) % kPtrAlign)
+    return CSA_ERR_INVALID_ARG;
+  const DecLayout L = dec_layout(d, B);
+  if (ws_bytes < L.total) return CSA_ERR_WORKSPACE;
+  if (B == 0) return CSA_OK;
+  const PackLayout P = pack_layout(d);
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t es = elem_size(d);
+  const int c = d->c, cI = d->cI;
+  char* y1 = at(ws, L.y1);
+  float* wI = reinterpret_cast<float*>(at(ws, L.wI));
+  char* y2 = at(ws, L.y2);
+  int* idx = idx_out ? idx_out : reinterpret_cast<int*>(at(ws, L.idx));
+  s = project_hidden(d, packed, h, B, y1, wI, st);
+  if (s != CSA_OK) return s;
+  s = launch_append(d, packed, y1, P.N1b, pos, ring, Ccache, KIcache, cache_len, cap, B, st);
+  if (s != CSA_OK) return s;
+  s = project_query(d, packed, y1 + (size_t)(4 * c + 4 * cI) * es, P.N1b, B, y2, st);
+  if (s != CSA_OK) return s;
+  IndexerArgs ia;
+  ia.qI = y2; ia.ld_qI = P.N2; ia.wI = wI; ia.ld_wI = d->nhI; ia.KI = KIcache; ia.idx = idx;
+  ia.topk = d->topk; ia.nhI = d->nhI; ia.sc_cap = cap;
+  ia.rm = RowMap{nullptr, nullptr, 0, 0, pos, cap, d->m};
+  s = launch_indexer(d, ia, B, st);
+  if (s != CSA_OK) return s;
+  MqaArgs ma;
+  ma.q = y2 + (size_t)d->nhI * cI * es; ma.ld_q = P.N2; ma.C = Ccache; ma.idx = idx;
+  ma.O = O; ma.ld_O = (long long)d->nh * c; ma.topk = d->topk; ma.nh = d->nh;
+  ma.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c));
+  ma.rm = RowMap{nullptr, nullptr, 0, 0, pos, cap, d->m};
+  return launch_mqa(d, ma, B, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,254 @@
+/*
+ * csa.h -- C ABI of libcsa.so, the B200 (sm_100a) forward path of
+ * Compressed Sparse Attention (CSA).
+ *
+ * Every formula is the one of the page "Compressed Sparse Attention
+ * (压缩稀疏注意力)" (cnblogs), equations (1)-(11); each entry point below names
+ * the equations it evaluates.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers marked [dev] are device pointers on the current CUDA device;
+ *    [host] pointers are host memory.  The caller owns every buffer, the
+ *    workspace included.  The library never allocates device memory, never
+ *    frees caller memory and never synchronises, except in
+ *    csa_get_device_status().
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  All work is enqueued asynchronously on it, in order.
+ *  - Matrices are dense row-major.  "ld" arguments are row strides in
+ *    ELEMENTS.  Element type = csa_dims.dtype for activations and weights
+ *    (fp32 or bf16); the indexer head weights w^I are always fp32 and block
+ *    indices always int32.
+ *  - Token indices t are 0-based and local to their sequence.  Packed
+ *    sequences are described by cu_seqlens[nseq+1] (token offsets, [dev]
+ *    int32, cu_seqlens[0] = 0) and cu_blocks[nseq+1] (offsets of each
+ *    sequence's compressed entries, [dev] int32, cu_blocks[b+1] - cu_blocks[b]
+ *    = floor(L_b / m)).  A sequence of L tokens has floor(L/m) compressed
+ *    entries; the L mod m tail tokens are not compressed.  Compression
+ *    blocks never cross a sequence boundary.
+ *  - Errors: arguments and shapes are checked on the host before anything is
+ *    launched (CSA_ERR_INVALID_ARG / CSA_ERR_UNSUPPORTED, nothing enqueued).
+ *    A failed launch returns CSA_ERR_CUDA.  Conditions found on the device
+ *    (an out-of-range block index given to csa_sparse_mqa, inconsistent
+ *    cu_seqlens/cu_blocks, a bounded wait that ran out) never fault: the
+ *    kernel skips the access, records a bit in a per-device status word and
+ *    returns; csa_get_device_status() reports and clears it.
+ *  - Nothing is thrown across this ABI.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,    /* NULL pointer, negative size, bad dims   */
+  CSA_ERR_UNSUPPORTED = 2,    /* valid but outside the kernels' limits   */
+  CSA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed     */
+  CSA_ERR_DEVICE_TIMEOUT = 4, /* a bounded device wait ran out           */
+  CSA_ERR_BAD_INDEX = 5,      /* out-of-range block index seen on device */
+  CSA_ERR_BAD_METADATA = 6,   /* cu_seqlens / cu_blocks inconsistent     */
+  CSA_ERR_WORKSPACE = 7       /* workspace smaller than required         */
+} csa_status;
+
+typedef enum { CSA_F32 = 0, CSA_BF16 = 1 } csa_dtype;
+
+/* Problem dimensions, named as on the page:
+ *   d    hidden size (H in R^{n x d})
+ *   c    head dimension of the KV entries (C^a, C^b, Z^a, Z^b in R^{n x c})
+ *   m    tokens per compressed entry
+ *   cI   indexer head dimension (K^IComp in R^{n/m x cI})
+ *   nhI  number of indexer query heads
+ *   nh   number of attention query heads
+ *   dc   query compression dimension (c^Q_t in R^{dc})
+ *   topk number of compressed entries kept per query (eq. 9)
+ *   dtype csa_dtype of activations and weights.  CSA_BF16 computes with
+ *        fp32 accumulation and stores intermediates in bf16 (w^I in fp32);
+ *        CSA_F32 computes and stores in fp32. */
+typedef struct {
+  int d, c, m, cI, nhI, nh, dc, topk;
+  int dtype;
+} csa_dims;
+
+/* The trainable parameters, each [in, out] row-major as in "X . W" on the
+ * page, all [dev] and of csa_dims.dtype.
+ *   W_aKV, W_bKV, W_aZ, W_bZ      [d, c]   eqs. (1), (2)
+ *   B_a, B_b                      [m, c]   position biases, eq. (3)
+ *   W_aKV_I .. W_bZ_I             [d, cI]  the indexer keys' own compression
+ *   B_a_I, B_b_I                  [m, cI]  parameters (same operation, width cI)
+ *   W_DQ                          [d, dc]  eq. (5)
+ *   W_IUQ                         [dc, nhI*cI]  eq. (6), heads concatenated
+ *   W_UQ                          [dc, nh*c]    eq. (10), heads concatenated
+ *   W_w                           [d, nhI]      eq. (7)                      */
+typedef struct {
+  const void *W_aKV, *W_bKV, *W_aZ, *W_bZ;
+  const void *B_a, *B_b;
+  const void *W_aKV_I, *W_bKV_I, *W_aZ_I, *W_bZ_I;
+  const void *B_a_I, *B_b_I;
+  const void *W_DQ, *W_IUQ, *W_UQ, *W_w;
+} csa_weights;
+
+/* ---------------------------------------------------------------------- */
+/* Weights                                                                 */
+/* ---------------------------------------------------------------------- */
+
+/* Bytes of the packed-weight buffer for these dims (0 if dims are invalid). */
+size_t csa_packed_weights_bytes(const csa_dims* dims);
+
+/* Re-lays the parameters of eqs. (1)-(7), (10) out for the projection
+ * kernels: the H-side matrices are concatenated along their output columns
+ * and transposed (one [N1, d] K-major matrix), the c^Q-side ones likewise
+ * ([N2, dc]); the biases are widened to fp32.  `packed` [dev] must hold
+ * csa_packed_weights_bytes(dims) bytes and be 256-byte aligned.  Run once
+ * per set of weights; every forward/decode call reads only `packed`. */
+csa_status csa_pack_weights(const csa_dims* dims, const csa_weights* w, void* packed,
+                            size_t packed_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Stages                                                                  */
+/* ---------------------------------------------------------------------- */
+
+/* Row width (elements) of the H-side projection output: the concatenation
+ * [C^a | C^b | Z^a | Z^b | C^aI | C^bI | Z^aI | Z^bI | c^Q] of one token,
+ * 4c + 4cI + dc elements of dtype. */
+int csa_hidden_row_elems(const csa_dims* dims);
+
+/* Row width (elements) of the c^Q-side projection output [q^I | q] of one
+ * token, nhI*cI + nh*c elements of dtype (heads concatenated, eqs. 6, 10). */
+int csa_query_row_elems(const csa_dims* dims);
+
+/* H-side projections, eqs. (1), (2), (5), (7) and the indexer-key
+ * projections, as one GEMM over the packed weights.
+ * H [dev]  : [T, d].   Y1 [dev] : [T, csa_hidden_row_elems] (row stride =
+ * that width).   wI [dev] : [T, nhI] fp32, the indexer head weights. */
+csa_status csa_project_hidden(const csa_dims* dims, const void* packed, const void* H, int T, void* Y1,
+                              float* wI, void* stream);
+
+/* c^Q-side projections, eqs. (6) and (10), from the shared latent query.
+ * cQ [dev] : [T, dc] with row stride ld_cQ (the c^Q columns of Y1 qualify).
+ * Y2 [dev] : [T, csa_query_row_elems] (row stride = that width). */
+csa_status csa_project_query(const csa_dims* dims, const void* packed, const void* cQ, int ld_cQ, int T,
+                             void* Y2, void* stream);
+
+/* Overlapping softmax compression, eqs. (3)-(4), for packed sequences.
+ * Ca, Cb, Za, Zb [dev] : [total_tokens, width] with row stride ld.
+ * Ba, Bb [dev]         : [m, width] position biases, fp32.
+ * out [dev]            : [total_blocks, width], row stride width.
+ * Entry i of a sequence uses the C^a/Z^a rows of its block i and the
+ * C^b/Z^b rows of block i-1; at i = 0 the Z^b logits are -inf and the C^b
+ * rows 0.  The softmax runs over the 2m logits of each channel. */
+csa_status csa_compress(const csa_dims* dims, const void* Ca, const void* Cb, const void* Za,
+                        const void* Zb, int ld, const float* Ba, const float* Bb, int width,
+                        const int* cu_seqlens, const int* cu_blocks, int nseq, int total_tokens,
+                        int total_blocks, void* out, void* stream);
+
+/* Lightning indexer (eq. 8) and top-k selector (eq. 9), prefill.
+ * qI [dev]  : [total_tokens, nhI*cI] (row stride ld_qI), heads concatenated.
+ * wI [dev]  : [total_tokens, nhI] fp32 (row stride ld_wI).
+ * KI [dev]  : [total_blocks, cI] compressed indexer keys.
+ * idx [dev] : [total_tokens, topk] int32 output.  Row t lists the chosen
+ *             local block indices s < floor(t/m) in ascending order, then -1.
+ *             k is clamped to floor(t/m); ties are broken by the lower s.
+ * max_seqlen [host] : an upper bound of every sequence length (it sizes the
+ *             per-query candidate storage; a longer sequence is clamped and
+ *             flags CSA_ERR_BAD_METADATA).
+ * The score matrix is never written to memory. */
+csa_status csa_indexer_topk(const csa_dims* dims, const void* qI, int ld_qI, const float* wI,
+                            int ld_wI, const void* KI, const int* cu_seqlens, const int* cu_blocks,
+                            int nseq, int total_tokens, int total_blocks, int max_seqlen, int* idx,
+                            void* stream);
+
+/* Shared-KV MQA over the selected entries, eqs. (10)-(11).
+ * q [dev]     : [total_tokens, nh*c] (row stride ld_q), heads concatenated.
+ * Ccomp [dev] : [total_blocks, c] compressed entries (keys AND values).
+ * idx [dev]   : [total_tokens, topk] int32 as produced by csa_indexer_topk;
+ *               -1 entries are skipped; an index outside [0, floor(t/m)) is
+ *               skipped and flags CSA_ERR_BAD_INDEX in the status word.
+ * O [dev]     : [total_tokens, nh*c] output, o_{t,h} = softmax(q K^T/sqrt(c)) V.
+ *               Rows with no selected entry are 0. */
+csa_status csa_sparse_mqa(const csa_dims* dims, const void* q, int ld_q, const void* Ccomp,
+                          const int* idx, const int* cu_seqlens, const int* cu_blocks, int nseq,
+                          int total_tokens, int total_blocks, void* O, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Whole forward pass (prefill)                                            */
+/* ---------------------------------------------------------------------- */
+
+/* Workspace bytes csa_forward needs for total_tokens tokens in nseq packed
+ * sequences (0 if the dims are invalid). */
+size_t csa_forward_workspace_bytes(const csa_dims* dims, int total_tokens, int nseq);
+
+/* CSA forward pass, eqs. (1)-(11).
+ * packed [dev]     : output of csa_pack_weights.
+ * H [dev]          : [total_tokens, d] hidden states.
+ * max_seqlen [host]: upper bound of every sequence length (as for
+ *                    csa_indexer_topk).
+ * O [dev]          : [total_tokens, nh*c] attention outputs o_{t,i}.
+ * Ccomp_out, KI_out, idx_out [dev, optional, may be NULL]: copies of
+ *                    C^Comp [total_blocks, c], K^IComp [total_blocks, cI]
+ *                    and the top-k indices [total_tokens, topk].
+ * ws [dev]         : workspace of ws_bytes >= csa_forward_workspace_bytes(),
+ *                    256-byte aligned; its contents need no initialisation. */
+csa_status csa_forward(const csa_dims* dims, const void* packed, const void* H,
+                       const int* cu_seqlens, const int* cu_blocks, int nseq, int total_tokens,
+                       int total_blocks, int max_seqlen, void* O, void* Ccomp_out, void* KI_out, int* idx_out,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Decode over a compressed cache                                          */
+/* ---------------------------------------------------------------------- */
+
+/* Row width of the per-sequence ring: 4c + 4cI elements of dtype, the raw
+ * rows [C^a | C^b | Z^a | Z^b | C^aI | C^bI | Z^aI | Z^bI] of one token. */
+int csa_ring_row_elems(const csa_dims* dims);
+
+/* Appends one token per sequence to the compressed cache.
+ * rows [dev]      : [B, csa_ring_row_elems] the new tokens' rows (eqs. 1-2).
+ * pos [dev]       : [B] int32, the new token's index t in its sequence.
+ * ring [dev]      : [B, 2m, csa_ring_row_elems], slot t mod 2m holds token t.
+ * Ccache [dev]    : [B, cap, c];  KIcache [dev] : [B, cap, cI].
+ * cache_len [dev] : [B] int32, must equal floor(t/m) on entry.
+ * The row is stored in slot t mod 2m; when (t+1) is a multiple of m, block
+ * i = (t+1)/m - 1 is compressed with eqs. (3)-(4) (C^a rows of block i, C^b
+ * rows of block i-1, or the i = 0 padding) into entry i of both caches and
+ * cache_len becomes i+1.  i >= cap flags CSA_ERR_BAD_INDEX and skips. */
+csa_status csa_cache_append(const csa_dims* dims, const void* packed, const void* rows,
+                            const int* pos, void* ring, void* Ccache, void* KIcache,
+                            int* cache_len, int cap, int B, void* stream);
+
+/* Workspace bytes csa_decode needs for B sequences. */
+size_t csa_decode_workspace_bytes(const csa_dims* dims, int B);
+
+/* One decode step: each of B independent sequences gets one new token h_b
+ * at position pos[b] and attends over its cached entries s < floor(t/m).
+ * h [dev] : [B, d].  O [dev] : [B, nh*c].  idx_out [dev, optional] : [B, topk].
+ * The caches, cache_len and ring are updated as by csa_cache_append. */
+csa_status csa_decode(const csa_dims* dims, const void* packed, const void* h, const int* pos,
+                      void* ring, void* Ccache, void* KIcache, int* cache_len, int cap, int B,
+                      void* O, int* idx_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Status                                                                  */
+/* ---------------------------------------------------------------------- */
+
+/* Synchronises `stream`, reads and clears the current device's status word
+ * and returns the most severe condition recorded since the last call
+ * (CSA_OK if none).  The only call that synchronises. */
+csa_status csa_get_device_status(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* csa_status_string(csa_status s);
+
+/* Number of kernels this library has enqueued in this process so far (all
+ * devices, all streams).  A monotone counter for accounting; never reset. */
+uint64_t csa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H_ */

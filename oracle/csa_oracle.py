@@ -300,7 +300,7 @@ def csa_forward(H, W, dims, seqlens, store="exact", rows=None, keep_scores=False
 # One decode step over a compressed cache
 # --------------------------------------------------------------------------
 
-def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="exact"):
+def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="exact", detail=None):
     """One new token per sequence attending over a compressed cache.
 
     The same equations as ``csa_forward`` for a single query token t = pos[b]
@@ -318,7 +318,8 @@ def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="e
     C_cache [B, cap, c], K_cache [B, cap, c^I], cache_len [B] and ring
     [B, 2m, 4c + 4c^I] are updated IN PLACE (copies are the caller's choice).
     cache_len[b] must equal floor(t/m) on entry.
-    Returns (O [B, n_h, c], idx [B, topk]).
+    Returns (O [B, n_h, c], idx [B, topk]).  If ``detail`` is a dict it
+    receives per sequence the scores I_t and the attention queries q_t.
     """
     m, k = dims["m"], dims["topk"]
     nh, nhI, c, cI = dims["nh"], dims["nhI"], dims["c"], dims["cI"]
@@ -371,4 +372,7 @@ def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="e
         sel = topk_select(I_t, k)
         idx[b] = sel
         O[b] = core_attn(q, C_cache[b, sel[sel >= 0]])
+        if detail is not None:
+            detail.setdefault("scores", []).append(I_t)
+            detail.setdefault("q", []).append(q)
     return O, idx

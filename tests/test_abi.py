@@ -1,0 +1,87 @@
+"""CPU-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import compressed_sparse_attention_09_b200 as csa
+from compressed_sparse_attention_09_b200 import capi
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "csa.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(csa_[a-z_]+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_binding_names():
+    assert declared_functions() == sorted(capi.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = csa.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_no_python_fallback_when_library_missing(monkeypatch, tmp_path):
+    monkeypatch.setattr(capi, "_lib", None)
+    monkeypatch.setattr(capi, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        capi.lib()
+
+
+TINY = csa.Dims(d=256, c=64, m=4, cI=32, nhI=4, nh=8, dc=128, topk=16, dtype=csa.CSA_F32)
+
+
+def test_sizes_and_strings():
+    assert csa.csa_packed_weights_bytes(TINY) > 0
+    assert csa.csa_forward_workspace_bytes(TINY, 256, 1) > 0
+    assert csa.csa_ring_row_elems(TINY) == 4 * 64 + 4 * 32
+    assert csa.csa_decode_workspace_bytes(TINY, 3) > 0
+    assert csa.status_string(0) == "ok"
+    bad = csa.Dims(d=256, c=63, m=4, cI=32, nhI=4, nh=8, dc=128, topk=16, dtype=csa.CSA_F32)
+    assert csa.csa_packed_weights_bytes(bad) == 0
+    assert csa.csa_forward_workspace_bytes(csa.Dims(0, 64, 4, 32, 4, 8, 128, 16, 0), 256, 1) == 0
+
+
+@pytest.mark.parametrize("dims,status", [
+    (csa.Dims(d=256, c=64, m=3, cI=32, nhI=4, nh=8, dc=128, topk=16, dtype=0), 2),    # m outside {1,2,4,8}
+    (csa.Dims(d=256, c=96, m=4, cI=32, nhI=4, nh=8, dc=128, topk=16, dtype=0), 2),    # c not a power of 2
+    (csa.Dims(d=256, c=64, m=4, cI=32, nhI=4, nh=8, dc=128, topk=0, dtype=0), 1),     # k = 0
+    (csa.Dims(d=256, c=64, m=4, cI=32, nhI=4, nh=8, dc=128, topk=16, dtype=7), 1),    # bad dtype
+])
+def test_host_validation_before_any_launch(dims, status):
+    L = csa.lib()
+    dummy = ctypes.c_void_p(1 << 20)
+    rc = L.csa_forward(ctypes.byref(dims.c_struct()), dummy, dummy, dummy, dummy, 1, 256, 64, 256, dummy,
+                       None, None, None, dummy, 1 << 30, None)
+    assert rc == status
+
+
+def test_null_pointers_rejected():
+    L = csa.lib()
+    d = ctypes.byref(TINY.c_struct())
+    assert L.csa_forward(d, None, None, None, None, 1, 256, 64, 256, None, None, None, None, None, 0, None) == 1
+    assert L.csa_compress(d, None, None, None, None, 64, None, None, 64, None, None, 1, 256, 64, None, None) == 1
+    assert L.csa_decode(d, None, None, None, None, None, None, None, 10, 1, None, None, None, 0, None) == 1
+
+
+def test_workspace_too_small_rejected():
+    L = csa.lib()
+    d = ctypes.byref(TINY.c_struct())
+    p = ctypes.c_void_p(1 << 20)   # 1024-aligned fake address; nothing is launched
+    need = csa.csa_forward_workspace_bytes(TINY, 256, 1)
+    assert L.csa_forward(d, p, p, p, p, 1, 256, 64, 256, p, None, None, None, p, need - 1, None) == 7
+
+
+def test_misaligned_workspace_rejected():
+    L = csa.lib()
+    d = ctypes.byref(TINY.c_struct())
+    p = ctypes.c_void_p(1 << 20)
+    q = ctypes.c_void_p((1 << 20) + 128)
+    assert L.csa_forward(d, p, p, p, p, 1, 256, 64, 256, p, None, None, None, q, 1 << 30, None) == 1

@@ -1,0 +1,263 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the fp64 oracle
+on the same seeded inputs (protocol and tolerances in tests/parity.py)."""
+import numpy as np
+import pytest
+import torch
+
+import compressed_sparse_attention_09_b200 as csa
+from compressed_sparse_attention_09_b200 import synth
+from oracle import csa_oracle as orc
+from parity import (check_topk_row, compare_dense, f64, gpu_forward, gpu_pack, store_mode,
+                    weights_f64)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def odims(dims):
+    return dict(m=dims.m, topk=dims.topk, nh=dims.nh, nhI=dims.nhI, c=dims.c, cI=dims.cI)
+
+
+def e2e(dims, seqlens, seed, rows=None):
+    """csa_forward vs the oracle: compressed entries, top-k sets, outputs."""
+    W = synth.make_weights(dims, seed)
+    H = synth.make_hidden(sum(seqlens), dims, seed)
+    g = gpu_forward(dims, W, H, seqlens)
+    o = orc.csa_forward(f64(H), weights_f64(W), odims(dims), list(seqlens), store=store_mode(dims),
+                        rows=rows, keep_scores=True)
+    compare_dense(f64(g["C_comp"]), o["C_comp"], dims.dtype, "C_comp")
+    compare_dense(f64(g["K_icomp"]), o["K_icomp"], dims.dtype, "K_icomp")
+    cu = np.concatenate([[0], np.cumsum(seqlens)])
+    kinds = {"exact": 0, "valid": 0}
+    want = np.zeros((len(o["rows"]), dims.nh, dims.c))
+    for r, t in enumerate(o["rows"]):
+        kinds[check_topk_row(g["idx"][t].numpy(), o["scores"][r], dims.topk)] += 1
+        b = int(np.searchsorted(cu, t, side="right") - 1)
+        sel = g["idx"][t].numpy()
+        sel = sel[sel >= 0]
+        want[r] = orc.core_attn(o["q"][r], o["C_comp"][o["cu_blocks"][b] + sel])
+    compare_dense(f64(g["O"][torch.as_tensor(o["rows"])]), want, dims.dtype, "O")
+    return kinds
+
+
+def test_tiny_fp32_full():
+    """The tiny fp32 workload end to end, every row (fp32 SIMT path, 1e-5)."""
+    w = synth.workloads()["tiny"]
+    kinds = e2e(w.dims, w.seqlens, w.seed)
+    assert kinds["exact"] > 0.9 * sum(kinds.values())
+
+
+SMALL_BF16 = csa.Dims(d=512, c=128, m=4, cI=64, nhI=16, nh=8, dc=256, topk=24, dtype=csa.CSA_BF16)
+
+
+def test_small_bf16_ragged():
+    """Ragged packed bf16: tails not divisible by m, a sequence shorter than m,
+    queries with fewer visible blocks than k."""
+    kinds = e2e(SMALL_BF16, (517, 3, 130, 1031), seed=21)
+    assert kinds["exact"] > 0.8 * sum(kinds.values())
+
+
+def test_small_bf16_m2_fp32():
+    e2e(csa.Dims(d=256, c=64, m=2, cI=32, nhI=8, nh=4, dc=128, topk=8, dtype=csa.CSA_F32), (77, 200), 22)
+    e2e(csa.Dims(d=256, c=64, m=2, cI=32, nhI=8, nh=4, dc=128, topk=8, dtype=csa.CSA_BF16), (77, 200), 23)
+
+
+def test_prefill_full_size_sampled_rows():
+    """The n = 8192 prefill workload at full size; outputs checked on sampled
+    rows (the first 2m rows, the last row and seeded random rows)."""
+    w = synth.workloads()["prefill"]
+    T = sum(w.seqlens)
+    rng = np.random.default_rng(5)
+    rows = sorted(set(range(2 * w.dims.m)) | {T - 1} | set(rng.integers(0, T, 24).tolist()))
+    kinds = e2e(w.dims, w.seqlens, w.seed, rows=rows)
+    assert kinds["exact"] >= 0.5 * len(rows)
+
+
+# ---------------------------------------------------------------- stages
+
+@pytest.mark.parametrize("dtype", [csa.CSA_F32, csa.CSA_BF16])
+@pytest.mark.parametrize("m", [1, 2, 4, 8])
+def test_stage_compress(dtype, m):
+    dims = csa.Dims(d=64, c=64, m=m, cI=32, nhI=4, nh=2, dc=64, topk=4, dtype=dtype)
+    lens = [m * 7 + 3, 1, m, 5 * m]
+    lens = [L for L in lens if L > 0]
+    T = sum(lens)
+    width, ld = 96, 4 * 96 + 8
+    Y = synth.make_normal((T, ld), dims, 31)
+    Ba = synth.make_normal((m, width), dims, 32, std=0.3).float()
+    Bb = synth.make_normal((m, width), dims, 33, std=0.3).float()
+    cu, cb = csa.cu_from_lengths(lens, m)
+    NB = int(cb[-1])
+    Yd = Y.to(DEV)
+    out = torch.empty(NB, width, dtype=Y.dtype, device=DEV)
+    csa.csa_compress(dims, Yd[:, 0:], Yd[:, width:], Yd[:, 2 * width:], Yd[:, 3 * width:], ld, Ba.to(DEV),
+                     Bb.to(DEV), width, cu.to(DEV), cb.to(DEV), len(lens), T, NB, out)
+    assert csa.csa_get_device_status() == 0
+    Y64 = f64(Y)
+    want = []
+    for b, L in enumerate(lens):
+        s = slice(int(cu[b]), int(cu[b + 1]))
+        want.append(orc.compress(Y64[s, 0:width], Y64[s, width:2 * width], Y64[s, 2 * width:3 * width],
+                                 Y64[s, 3 * width:4 * width], f64(Ba), f64(Bb), m))
+    want = orc.storage_round(np.concatenate(want), store_mode(dims))
+    compare_dense(f64(out.cpu()), want, dtype, "compress")
+
+
+def _indexer_case(dims, lens, seed, zero_w=False):
+    T = sum(lens)
+    cu, cb = csa.cu_from_lengths(lens, dims.m)
+    NB = int(cb[-1])
+    qI = synth.make_normal((T, dims.nhI * dims.cI), dims, seed)
+    wI = synth.make_normal((T, dims.nhI), dims, seed + 1).float()
+    if zero_w:
+        wI.zero_()
+    KI = synth.make_normal((NB, dims.cI), dims, seed + 2, std=0.5)
+    idx = torch.full((T, dims.topk), 7, dtype=torch.int32, device=DEV)
+    csa.csa_indexer_topk(dims, qI.to(DEV), dims.nhI * dims.cI, wI.to(DEV), dims.nhI, KI.to(DEV), cu.to(DEV),
+                         cb.to(DEV), len(lens), T, NB, max(lens), idx)
+    assert csa.csa_get_device_status() == 0
+    idx = idx.cpu().numpy()
+    q64, w64, K64 = f64(qI).reshape(T, dims.nhI, dims.cI), f64(wI), f64(KI)
+    kinds = {"exact": 0, "valid": 0}
+    for b, L in enumerate(lens):
+        for t in range(L):
+            row = int(cu[b]) + t
+            sc = orc.indexer_scores(q64[row], w64[row], K64[int(cb[b]):int(cb[b]) + t // dims.m])
+            kinds[check_topk_row(idx[row], sc, dims.topk)] += 1
+            if zero_w:
+                keff = min(dims.topk, t // dims.m)
+                assert idx[row].tolist() == list(range(keff)) + [-1] * (dims.topk - keff)
+    return kinds
+
+
+@pytest.mark.parametrize("dtype", [csa.CSA_F32, csa.CSA_BF16])
+def test_stage_indexer_topk(dtype):
+    dims = csa.Dims(d=64, c=64, m=4, cI=64, nhI=8, nh=2, dc=64, topk=16, dtype=dtype)
+    kinds = _indexer_case(dims, [1000, 130, 2, 67], 41)
+    assert kinds["exact"] > 0.95 * sum(kinds.values())
+
+
+def test_stage_indexer_ties_take_lowest_blocks():
+    dims = csa.Dims(d=64, c=64, m=4, cI=32, nhI=4, nh=2, dc=64, topk=5, dtype=csa.CSA_BF16)
+    _indexer_case(dims, [300], 42, zero_w=True)
+
+
+def test_stage_indexer_large_k():
+    dims = csa.Dims(d=64, c=64, m=4, cI=128, nhI=16, nh=2, dc=64, topk=600, dtype=csa.CSA_BF16)
+    kinds = _indexer_case(dims, [4096, 2500], 43)
+    assert kinds["exact"] > 0.5 * sum(kinds.values())
+
+
+def _mqa_case(dims, lens, seed, idx_fn):
+    T = sum(lens)
+    cu, cb = csa.cu_from_lengths(lens, dims.m)
+    NB = int(cb[-1])
+    q = synth.make_normal((T, dims.nh * dims.c), dims, seed)
+    C = synth.make_normal((max(NB, 1), dims.c), dims, seed + 1)
+    idx = torch.full((T, dims.topk), -1, dtype=torch.int32)
+    for b, L in enumerate(lens):
+        for t in range(L):
+            idx[int(cu[b]) + t] = torch.as_tensor(idx_fn(t // dims.m, dims.topk, int(cu[b]) + t))
+    O = torch.empty(T, dims.nh * dims.c, dtype=q.dtype, device=DEV)
+    csa.csa_sparse_mqa(dims, q.to(DEV), dims.nh * dims.c, C.to(DEV), idx.to(DEV), cu.to(DEV), cb.to(DEV),
+                       len(lens), T, NB, O)
+    status = csa.csa_get_device_status()
+    q64 = f64(q).reshape(T, dims.nh, dims.c)
+    C64 = f64(C)
+    want = np.zeros((T, dims.nh, dims.c))
+    for b, L in enumerate(lens):
+        for t in range(L):
+            row = int(cu[b]) + t
+            sel = idx[row].numpy()
+            sel = sel[(sel >= 0) & (sel < t // dims.m)]
+            want[row] = orc.core_attn(q64[row], C64[int(cb[b]) + sel])
+    compare_dense(f64(O.cpu()).reshape(T, dims.nh, dims.c), want, dims.dtype, "mqa")
+    return status
+
+
+def _first_k(avail, k, row):
+    keff = min(avail, k)
+    return list(range(keff)) + [-1] * (k - keff)
+
+
+def _strided(avail, k, row):
+    sel = sorted(set((np.arange(min(avail, k)) * 7 + row) % max(avail, 1))) if avail else []
+    return sel + [-1] * (k - len(sel))
+
+
+@pytest.mark.parametrize("dtype", [csa.CSA_F32, csa.CSA_BF16])
+def test_stage_sparse_mqa(dtype):
+    dims = csa.Dims(d=64, c=512, m=4, cI=32, nhI=4, nh=6, dc=64, topk=40, dtype=dtype)
+    assert _mqa_case(dims, [300, 9, 1], 51, _strided) == 0
+    assert _mqa_case(dims, [200], 52, _first_k) == 0
+
+
+def test_stage_sparse_mqa_flags_bad_index_without_fault():
+    """An index >= floor(t/m) is skipped and reported through the status word."""
+    dims = csa.Dims(d=64, c=64, m=4, cI=32, nhI=4, nh=2, dc=64, topk=4, dtype=csa.CSA_BF16)
+
+    def bad(avail, k, row):
+        return [0, avail + 3, -1, -1] if avail else [-1] * k
+
+    assert _mqa_case(dims, [64], 53, bad) == 5   # CSA_ERR_BAD_INDEX
+    assert csa.csa_get_device_status() == 0      # cleared by the read
+
+
+# ---------------------------------------------------------------- decode
+
+def decode_case(dims, B, pos0, cap, steps, seed, check):
+    """`steps` decode steps of B sequences starting at token pos0 (GPU) vs
+    the oracle's decode step on the sequences listed in `check`."""
+    m, c, cI = dims.m, dims.c, dims.cI
+    W = synth.make_weights(dims, seed)
+    packed = gpu_pack(dims, W)
+    RW = csa.csa_ring_row_elems(dims)
+    Cc = synth.make_normal((B, cap, c), dims, seed + 1)
+    Kc = synth.make_normal((B, cap, cI), dims, seed + 2)
+    ring = synth.make_normal((B, 2 * m, RW), dims, seed + 3)
+    pos = torch.full((B,), pos0, dtype=torch.int32)
+    clen = torch.full((B,), pos0 // m, dtype=torch.int32)
+    d_Cc, d_Kc, d_ring, d_clen = Cc.to(DEV), Kc.to(DEV), ring.to(DEV), clen.to(DEV)
+    o_Cc, o_Kc, o_ring = f64(Cc[check]), f64(Kc[check]), f64(ring[check])
+    o_clen = clen[check].numpy().astype(np.int64)
+    W64 = weights_f64(W)
+    ws = torch.empty(csa.csa_decode_workspace_bytes(dims, B), dtype=torch.uint8, device=DEV)
+    for step in range(steps):
+        h = synth.make_normal((B, dims.d), dims, seed + 100 + step)
+        O = torch.empty(B, dims.nh * c, dtype=h.dtype, device=DEV)
+        idx = torch.empty(B, dims.topk, dtype=torch.int32, device=DEV)
+        csa.csa_decode(dims, packed, h.to(DEV), pos.to(DEV), d_ring, d_Cc, d_Kc, d_clen, cap, B, O, idx, ws)
+        assert csa.csa_get_device_status() == 0
+        detail = {}
+        oO, oidx = orc.csa_decode_step(f64(h[check]), pos[check].numpy(), o_Cc, o_Kc, o_clen, o_ring, W64,
+                                       odims(dims), store=store_mode(dims), detail=detail)
+        gidx = idx.cpu().numpy()[check]
+        want = np.zeros_like(oO)
+        for r in range(len(check)):
+            check_topk_row(gidx[r], detail["scores"][r], dims.topk)
+            sel = gidx[r][gidx[r] >= 0]
+            want[r] = orc.core_attn(detail["q"][r], o_Cc[r][sel])
+        compare_dense(f64(O.cpu()).reshape(B, dims.nh, c)[check], want, dims.dtype, f"decode O step {step}")
+        pos += 1
+    assert np.array_equal(d_clen.cpu().numpy()[check], o_clen)
+    nb = int(o_clen.max())
+    compare_dense(f64(d_Cc.cpu()[check][:, :nb]), o_Cc[:, :nb], dims.dtype, "C cache")
+    compare_dense(f64(d_Kc.cpu()[check][:, :nb]), o_Kc[:, :nb], dims.dtype, "K cache")
+
+
+def test_decode_small_across_appends():
+    dims = csa.Dims(d=256, c=128, m=4, cI=64, nhI=8, nh=4, dc=128, topk=16, dtype=csa.CSA_BF16)
+    decode_case(dims, B=5, pos0=61, cap=40, steps=9, seed=61, check=[0, 2, 4])
+
+
+def test_decode_small_fp32_from_start():
+    dims = csa.Dims(d=128, c=64, m=2, cI=32, nhI=4, nh=4, dc=64, topk=3, dtype=csa.CSA_F32)
+    decode_case(dims, B=3, pos0=0, cap=16, steps=11, seed=62, check=[0, 1, 2])
+
+
+def test_decode_full_size_sampled_sequences():
+    """The decode workload at full size (64 sequences, 16384 cached entries,
+    n_h = 128, k = 2048); sampled sequences checked against the oracle."""
+    w = synth.workloads()["decode"]
+    decode_case(w.dims, B=w.decode_batch, pos0=w.decode_pos, cap=w.cache_cap, steps=1, seed=w.seed,
+                check=[0, 17, 63])
