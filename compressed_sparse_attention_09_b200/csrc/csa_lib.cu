@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "compress.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tcgen05.cuh"
 #include "indexer_simt.cuh"
 #include "mqa_simt.cuh"
 #include "pack.cuh"
@@ -105,14 +106,95 @@ FwdLayout fwd_layout(const csa_dims* d, int T) {
 
 inline char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
 
+// ------------------------------------------------------------------ device facts
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [outer, inner] with row stride row_bytes, read in
+// boxes of box_inner (= 64, one 128-byte swizzle span) x box_outer rows.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                    uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  if (reinterpret_cast<uintptr_t>(base) % 16 || row_bytes % 16) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ launchers
+template <int BN, int kStages>
+csa_status launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& g, cudaStream_t st) {
+  using Cfg = TcGemmCfg<BN, kStages>;
+  auto k = gemm_tc_kernel<BN, kStages>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) != cudaSuccess)
+    return CSA_ERR_CUDA;
+  const int tiles = ((g.M + Cfg::BM - 1) / Cfg::BM) * ((g.N + BN - 1) / BN);
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  k<<<grid, 192, Cfg::SMEM, st>>>(ta, tb, g);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+// D[M, N] = A[M, K] . B[N, K]^T routed to `out`.  A: activations (row stride
+// lda), B: packed K-major weights with at least round_up(N, 256) rows.
 csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const void* B, long long ldb,
                        int M, int N, int K, const GemmOut& out, cudaStream_t st) {
   if (M == 0) return CSA_OK;
+  if (d->dtype == CSA_BF16) {
+    CUtensorMap ta, tb;
+    TcGemmArgs g;
+    g.K = K;
+    g.out = out;
+    if (M >= 128) {  // activations as the M operand, 128 x 256 tiles
+      const uint64_t nrows_b = (uint64_t)round_up_int(N, 256);
+      if (!make_tmap_bf16(&ta, A, K, M, lda * 2, 64, 128) || !make_tmap_bf16(&tb, B, K, nrows_b, ldb * 2, 64, 256))
+        return CSA_ERR_UNSUPPORTED;
+      g.M = M; g.N = N; g.transpose_out = 0;
+      return launch_tc_gemm<256, 4>(ta, tb, g, st);
+    }
+    // few rows (decode): swap A and B so the weights fill the 128-row MMA
+    // operand and the tokens are the N = 64 operand; the epilogue transposes.
+    const uint64_t nrows_w = (uint64_t)round_up_int(N, 256);
+    if (!make_tmap_bf16(&ta, B, K, nrows_w, ldb * 2, 64, 128) || !make_tmap_bf16(&tb, A, K, M, lda * 2, 64, 64))
+      return CSA_ERR_UNSUPPORTED;
+    g.M = N; g.N = M; g.transpose_out = 1;
+    if (M <= 64) return launch_tc_gemm<64, 8>(ta, tb, g, st);
+    return CSA_ERR_UNSUPPORTED;
+  }
   SimtGemmArgs g{A, lda, B, ldb, M, N, K, out};
   dim3 grid((N + 127) / 128, (M + 127) / 128);
-  if (d->dtype == CSA_BF16) gemm_simt_kernel<bf16><<<grid, 256, 0, st>>>(g);
-  else gemm_simt_kernel<float><<<grid, 256, 0, st>>>(g);
+  gemm_simt_kernel<float><<<grid, 256, 0, st>>>(g);
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }

@@ -1,0 +1,189 @@
+// Tensor-core projection GEMM for sm_100a:  D[M, N] = A[M, K] . B[N, K]^T,
+// bf16 operands, fp32 accumulation in TMEM, routed epilogue (gemm_simt.cuh's
+// GemmOut).  This carries eqs. (1), (2), (5), (7) (A = H, B = packed H-side
+// weights) and eqs. (6), (10) (A = c^Q, B = packed up-projections) of
+// "Compressed Sparse Attention" (cnblogs).
+//
+// Persistent, warp-specialised CTA (one per SM, 192 threads):
+//   warp 0      TMA producer: 128 x 64 A tiles and BN x 64 B tiles, both
+//               K-major with 128-byte swizzle, into a kStages-deep ring;
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M = 128,
+//               N = BN, K = 16) and commits stage releases / tile completions;
+//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, conversion, and
+//               vectorised stores routed to the output segments.
+// Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap
+// the main loop of tile i+1.  Tiles are visited M-fastest so that the CTAs
+// running at one time share the same few B (weight) column blocks in L2.
+// Every wait is bounded (sm100::mbar_wait); a wait that runs out records a
+// timeout in the status word and the CTA leaves its loop.
+#pragma once
+#include "gemm_simt.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+
+struct TcGemmArgs {
+  int M, N, K;
+  GemmOut out;
+  int transpose_out;   // 1: D[i][j] is stored at output row j, column i (swap-AB use)
+};
+
+template <int BN, int kStages>
+struct TcGemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;       // two accumulators
+  static constexpr size_t SMEM = 1024 /*align slack*/ + (size_t)kStages * STAGE_BYTES + 256 /*barriers*/;
+};
+
+template <typename T>
+__device__ __forceinline__ void store_chunk32(const GemmOut& o, long long row, int col0, int N, const float* v) {
+  // fast path: the 32 columns lie in one segment and are in range
+  for (int s = 0; s < o.nseg; ++s) {
+    const OutSeg& sg = o.seg[s];
+    if (col0 >= sg.col0 && col0 + 32 <= sg.col0 + sg.ncols && col0 + 32 <= N) {
+      const long long off = row * sg.ld + (col0 - sg.col0);
+      const uintptr_t addr = reinterpret_cast<uintptr_t>(sg.ptr) + (uintptr_t)off * (sg.f32 ? 4 : sizeof(T));
+      if (addr % 16) break;   // unaligned destination: per-element stores below
+      if (sg.f32) {
+        float4* p = reinterpret_cast<float4*>(static_cast<float*>(sg.ptr) + off);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) p[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {
+        uint4* p = reinterpret_cast<uint4*>(static_cast<T*>(sg.ptr) + off);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          Vec16<T> pk;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pk.e[e] = from_f32<T>(v[8 * q + e]);
+          p[q] = pk.u;
+        }
+      }
+      return;
+    }
+  }
+  for (int j = 0; j < 32; ++j)
+    if (col0 + j < N) store_out<T>(o, row, col0 + j, v[j]);
+}
+
+template <int BN, int kStages>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcGemmArgs g) {
+  using Cfg = TcGemmCfg<BN, kStages>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smA = smem;
+  uint8_t* smB = smem + kStages * Cfg::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tiles = (g.M + Cfg::BM - 1) / Cfg::BM;
+  const int n_tiles = (g.N + BN - 1) / BN;
+  const int k_blocks = (g.K + Cfg::BK - 1) / Cfg::BK;
+  const int total = m_tiles * n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        const int mt = tile % m_tiles, nt = tile / m_tiles;
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
+          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          tma_load_2d(&tmA, &full[stage], smA + stage * Cfg::A_BYTES, kb * Cfg::BK, mt * Cfg::BM);
+          tma_load_2d(&tmB, &full[stage], smB + stage * Cfg::B_BYTES, kb * Cfg::BK, nt * BN);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---------------- MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(Cfg::BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smA + stage * Cfg::A_BYTES);
+          const uint32_t b0 = smem_u32(smB + stage * Cfg::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < Cfg::BK / 16; ++k)
+            mma_bf16(d_tmem, sdesc_k_sw128(a0 + k * 32), sdesc_k_sw128(b0 + k * 32), idesc, (kb | k) != 0);
+          mma_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        mma_commit(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {  // ---------------- epilogue warps 2..5
+    const int sub = warp & 3;   // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+      const int mt = tile % m_tiles, nt = tile / m_tiles;
+      if (!mbar_wait(&tfull[acc], acc_phase)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const int r = mt * Cfg::BM + sub * 32 + lane;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN + ch * 32), v);
+        const int c0 = nt * BN + ch * 32;
+        if (!g.transpose_out) {
+          if (r < g.M && c0 < g.N) store_chunk32<__nv_bfloat16>(g.out, r, c0, g.N, v);
+        } else if (r < g.M) {
+          for (int j = 0; j < 32; ++j)
+            if (c0 + j < g.N) store_out<__nv_bfloat16>(g.out, c0 + j, r, v[j]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace csa

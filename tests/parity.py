@@ -5,9 +5,14 @@ Comparison protocol (tolerances of the bf16 and fp32 configurations):
 * top-k sets: where the oracle's k-th / (k+1)-th score gap exceeds 1e-3
   relative, the GPU set must equal the oracle's exactly; below that gap the
   set must be valid (k_eff distinct visible blocks, each with an oracle score
-  within 1e-3 relative of the k-th score).  Relative here means relative to
+  within the bar of the k-th score).  Relative here means relative to
   max(|I_(k)|, 1e-2 * max_s |I_s|), so that a k-th score that happens to sit
-  near zero does not demand more than fp32 can resolve.
+  near zero does not demand more than fp32 can resolve.  Stage tests feed
+  both sides bit-identical inputs and use exactly this bar.  End-to-end bf16
+  tests widen it by the score perturbation that bf16 storage rounding itself
+  causes in the oracle (rounding_sensitivity): there both sides round their
+  own projections to bf16 and a few stored elements legitimately land on
+  neighbouring bf16 values.
 * outputs: the GPU output o_t is compared with eq. (11) evaluated by the
   oracle on the GPU's own index set (this isolates the attention error from
   the selection): bf16 max-abs <= 2e-2 and relative L2 <= 1e-2; fp32
@@ -81,8 +86,12 @@ def compare_dense(got, want, dtype, what=""):
     return max_abs, rel
 
 
-def check_topk_row(gpu_row, scores, k):
-    """Check one GPU top-k row against the oracle's fp64 scores; returns 'exact'/'valid'."""
+def check_topk_row(gpu_row, scores, k, extra_tol=0.0):
+    """Check one GPU top-k row against the oracle's fp64 scores; returns 'exact'/'valid'.
+
+    extra_tol (absolute) widens the gap bar where the two sides do not see
+    bit-identical inputs (end-to-end runs, where both round their own fp32 /
+    fp64 projections to bf16 and so may store neighbouring bf16 values)."""
     gpu_row = np.asarray(gpu_row, dtype=np.int64)
     avail = len(scores)
     keff = min(k, avail)
@@ -97,18 +106,17 @@ def check_topk_row(gpu_row, scores, k):
     srt = np.sort(scores)[::-1]
     Ik, Ik1 = srt[keff - 1], srt[keff]
     denom = max(abs(Ik), 1e-2 * float(np.abs(scores).max()), 1e-300)
-    if (Ik - Ik1) / denom > GAP_REL:
-        assert np.array_equal(sel, want), f"set differs with gap {(Ik - Ik1) / denom:.2e}"
+    bar = max(GAP_REL * denom, extra_tol)
+    if Ik - Ik1 > bar:
+        assert np.array_equal(sel, want), f"set differs with gap {(Ik - Ik1) / denom:.2e} (bar {bar / denom:.2e})"
         return "exact"
-    assert np.all(scores[sel] >= Ik - GAP_REL * denom), "a chosen block scores below the k-th"
+    assert np.all(scores[sel] >= Ik - bar), "a chosen block scores below the k-th"
     return "valid"
 
 
-def oracle_attn_on_idx(q_rows, C_comp_seq, idx_rows):
-    """Eq. (11) by the oracle on given index rows (local block indices, -1 padded)."""
-    out = np.zeros(q_rows.shape)
-    for r in range(q_rows.shape[0]):
-        sel = np.asarray(idx_rows[r])
-        sel = sel[sel >= 0]
-        out[r] = orc.core_attn(q_rows[r], C_comp_seq[r][sel] if isinstance(C_comp_seq, list) else C_comp_seq[sel])
-    return out
+def rounding_sensitivity(scores_bf16, scores_exact):
+    """Score perturbation caused by bf16 storage rounding alone, from the oracle:
+    max_s |I_bf16(t, s) - I_exact(t, s)| over one row (0 for an empty row)."""
+    if len(scores_bf16) == 0:
+        return 0.0
+    return float(np.abs(np.asarray(scores_bf16) - np.asarray(scores_exact)).max())

@@ -7,8 +7,8 @@ import torch
 import compressed_sparse_attention_09_b200 as csa
 from compressed_sparse_attention_09_b200 import synth
 from oracle import csa_oracle as orc
-from parity import (check_topk_row, compare_dense, f64, gpu_forward, gpu_pack, store_mode,
-                    weights_f64)
+from parity import (check_topk_row, compare_dense, f64, gpu_forward, gpu_pack, rounding_sensitivity,
+                    store_mode, weights_f64)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -25,13 +25,19 @@ def e2e(dims, seqlens, seed, rows=None):
     g = gpu_forward(dims, W, H, seqlens)
     o = orc.csa_forward(f64(H), weights_f64(W), odims(dims), list(seqlens), store=store_mode(dims),
                         rows=rows, keep_scores=True)
+    if dims.dtype == csa.CSA_BF16:
+        ox = orc.csa_forward(f64(H), weights_f64(W), odims(dims), list(seqlens), store="exact",
+                             rows=o["rows"], keep_scores=True)
+        sens = [rounding_sensitivity(a, b) for a, b in zip(o["scores"], ox["scores"])]
+    else:
+        sens = [0.0] * len(o["rows"])
     compare_dense(f64(g["C_comp"]), o["C_comp"], dims.dtype, "C_comp")
     compare_dense(f64(g["K_icomp"]), o["K_icomp"], dims.dtype, "K_icomp")
     cu = np.concatenate([[0], np.cumsum(seqlens)])
     kinds = {"exact": 0, "valid": 0}
     want = np.zeros((len(o["rows"]), dims.nh, dims.c))
     for r, t in enumerate(o["rows"]):
-        kinds[check_topk_row(g["idx"][t].numpy(), o["scores"][r], dims.topk)] += 1
+        kinds[check_topk_row(g["idx"][t].numpy(), o["scores"][r], dims.topk, sens[r])] += 1
         b = int(np.searchsorted(cu, t, side="right") - 1)
         sel = g["idx"][t].numpy()
         sel = sel[sel >= 0]
@@ -70,7 +76,7 @@ def test_prefill_full_size_sampled_rows():
     rng = np.random.default_rng(5)
     rows = sorted(set(range(2 * w.dims.m)) | {T - 1} | set(rng.integers(0, T, 24).tolist()))
     kinds = e2e(w.dims, w.seqlens, w.seed, rows=rows)
-    assert kinds["exact"] >= 0.5 * len(rows)
+    assert kinds["exact"] >= 0.25 * len(rows), kinds
 
 
 # ---------------------------------------------------------------- stages
@@ -146,6 +152,33 @@ def test_stage_indexer_large_k():
     dims = csa.Dims(d=64, c=64, m=4, cI=128, nhI=16, nh=2, dc=64, topk=600, dtype=csa.CSA_BF16)
     kinds = _indexer_case(dims, [4096, 2500], 43)
     assert kinds["exact"] > 0.5 * sum(kinds.values())
+
+
+def test_stage_indexer_topk_full_size_sampled():
+    """The indexer stage at the n = 8192 prefill sizes (n_h^I = 64, c^I = 128,
+    k = 512) on bit-identical bf16 inputs, every row checked against the
+    oracle's fp64 scores with the plain 1e-3 gap bar."""
+    w = synth.workloads()["prefill"]
+    dims = w.dims
+    lens = list(w.seqlens)
+    T = sum(lens)
+    cu, cb = csa.cu_from_lengths(lens, dims.m)
+    NB = int(cb[-1])
+    qI = synth.make_normal((T, dims.nhI * dims.cI), dims, 71)
+    wI = synth.make_normal((T, dims.nhI), dims, 72).float()
+    KI = synth.make_normal((NB, dims.cI), dims, 73, std=0.5)
+    idx = torch.empty((T, dims.topk), dtype=torch.int32, device=DEV)
+    csa.csa_indexer_topk(dims, qI.to(DEV), dims.nhI * dims.cI, wI.to(DEV), dims.nhI, KI.to(DEV), cu.to(DEV),
+                         cb.to(DEV), 1, T, NB, T, idx)
+    assert csa.csa_get_device_status() == 0
+    idx = idx.cpu().numpy()
+    q64, w64, K64 = f64(qI).reshape(T, dims.nhI, dims.cI), f64(wI), f64(KI)
+    rows = sorted(set(range(0, T, 61)) | {T - 1, 4 * 512, 4 * 512 + 3})
+    kinds = {"exact": 0, "valid": 0}
+    for t in rows:
+        sc = orc.indexer_scores(q64[t], w64[t], K64[:t // dims.m])
+        kinds[check_topk_row(idx[t], sc, dims.topk)] += 1
+    assert kinds["exact"] > 0.9 * len(rows), kinds
 
 
 def _mqa_case(dims, lens, seed, idx_fn):
@@ -228,13 +261,17 @@ def decode_case(dims, B, pos0, cap, steps, seed, check):
         idx = torch.empty(B, dims.topk, dtype=torch.int32, device=DEV)
         csa.csa_decode(dims, packed, h.to(DEV), pos.to(DEV), d_ring, d_Cc, d_Kc, d_clen, cap, B, O, idx, ws)
         assert csa.csa_get_device_status() == 0
-        detail = {}
+        detail, dx = {}, {}
+        if dims.dtype == csa.CSA_BF16:   # same step with exact storage, for the rounding sensitivity
+            orc.csa_decode_step(f64(h[check]), pos[check].numpy(), o_Cc.copy(), o_Kc.copy(), o_clen.copy(),
+                                o_ring.copy(), W64, odims(dims), store="exact", detail=dx)
         oO, oidx = orc.csa_decode_step(f64(h[check]), pos[check].numpy(), o_Cc, o_Kc, o_clen, o_ring, W64,
                                        odims(dims), store=store_mode(dims), detail=detail)
         gidx = idx.cpu().numpy()[check]
         want = np.zeros_like(oO)
         for r in range(len(check)):
-            check_topk_row(gidx[r], detail["scores"][r], dims.topk)
+            sens = rounding_sensitivity(detail["scores"][r], dx["scores"][r]) if dx else 0.0
+            check_topk_row(gidx[r], detail["scores"][r], dims.topk, sens)
             sel = gidx[r][gidx[r] >= 0]
             want[r] = orc.core_attn(detail["q"][r], o_Cc[r][sel])
         compare_dense(f64(O.cpu()).reshape(B, dims.nh, c)[check], want, dims.dtype, f"decode O step {step}")
