@@ -4,9 +4,9 @@ csa_project_query, against fp64 products of the same inputs.
 
 A bf16 output must be the fp64 product rounded to bf16, up to one bf16 ulp
 (the fp32 accumulation can move a value across a rounding boundary) plus a
-small absolute term for values near 0 (this term also covers a c^Q element
-that the two sides stored on neighbouring bf16 values); fp32 outputs within
-1e-5 relative to the row scale."""
+small absolute term for values near 0; fp32 outputs within 1e-5 relative to
+the row scale.  Each GEMM gets seeded inputs that both sides share (H for the
+first, a seeded c^Q with a padded row stride for the second)."""
 import numpy as np
 import pytest
 import torch
@@ -46,8 +46,10 @@ def test_projections(dtype, T):
     wI = torch.empty(T, dims.nhI, dtype=torch.float32, device=DEV)
     Y2 = torch.empty(T, N2, dtype=H.dtype, device=DEV)
     csa.csa_project_hidden(dims, packed, H.to(DEV), T, Y1, wI)
-    cq_off = 4 * dims.c + 4 * dims.cI
-    csa.csa_project_query(dims, packed, Y1.data_ptr() + cq_off * Y1.element_size(), N1b, T, Y2)
+    # the second GEMM gets a seeded c^Q (row stride ld_cq), identical on both sides
+    ld_cq = dims.dc + 24
+    cQ = synth.make_normal((T, ld_cq), dims, 190 + T)
+    csa.csa_project_query(dims, packed, cQ.to(DEV), ld_cq, T, Y2)
     assert csa.csa_get_device_status() == 0
     W64 = {k: f64(v) for k, v in W.items()}
     H64 = f64(H)
@@ -55,7 +57,7 @@ def test_projections(dtype, T):
     want1 = orc.storage_round(np.concatenate([orc.project(H64, W64[n]) for n in H_SIDE], axis=1), store)
     check(f64(Y1.cpu()), want1, dtype, "Y1")
     check(wI.cpu().double().numpy(), orc.project(H64, W64["W_w"]), csa.CSA_F32, "wI")   # fp32 output
-    cQ = want1[:, cq_off:cq_off + dims.dc]               # the oracle's own stored c^Q
-    want2 = orc.storage_round(np.concatenate([orc.project(cQ, W64["W_IUQ"]), orc.project(cQ, W64["W_UQ"])],
+    cQ64 = f64(cQ)[:, :dims.dc]
+    want2 = orc.storage_round(np.concatenate([orc.project(cQ64, W64["W_IUQ"]), orc.project(cQ64, W64["W_UQ"])],
                                              axis=1), store)
     check(f64(Y2.cpu()), want2, dtype, "Y2")
