@@ -15,6 +15,7 @@
 #include "gemm_tcgen05.cuh"
 #include "indexer_simt.cuh"
 #include "mqa_simt.cuh"
+#include "mqa_tcgen05.cuh"
 #include "pack.cuh"
 
 using namespace csa;
@@ -271,6 +272,24 @@ csa_status mqa_launch(const MqaArgs& a, int rows, cudaStream_t st) {
 csa_status launch_mqa(const csa_dims* d, const MqaArgs& a, int rows, cudaStream_t st) {
   if (rows == 0) return CSA_OK;
   const bool b = d->dtype == CSA_BF16;
+  if (b && d->c == mqa::kC && d->nh % mqa::kHeads == 0 && a.ld_q % 8 == 0 && a.ld_O % 8 == 0 &&
+      reinterpret_cast<uintptr_t>(a.q) % 16 == 0 && reinterpret_cast<uintptr_t>(a.O) % 16 == 0 &&
+      reinterpret_cast<uintptr_t>(a.C) % 16 == 0) {
+    // tensor-core path: c = 512, heads in groups of 64
+    MqaTcArgs t;
+    t.q = static_cast<const bf16*>(a.q); t.ld_q = a.ld_q;
+    t.C = static_cast<const bf16*>(a.C); t.idx = a.idx;
+    t.O = static_cast<bf16*>(a.O); t.ld_O = a.ld_O;
+    t.topk = a.topk; t.nh = a.nh; t.rows = rows; t.scale_log2 = a.scale_log2; t.rm = a.rm;
+    if (cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mqa::kSmem) !=
+        cudaSuccess)
+      return CSA_ERR_CUDA;
+    const long long items = (long long)rows * (d->nh / mqa::kHeads);
+    const int grid = items < sm_count() ? (int)items : sm_count();
+    mqa_tc_kernel<<<grid, mqa::kThreads, mqa::kSmem, st>>>(t);
+    CSA_CHECK_LAUNCH();
+    return CSA_OK;
+  }
   switch (d->c / 32) {
     case 2: return b ? mqa_launch<bf16, 2>(a, rows, st) : mqa_launch<float, 2>(a, rows, st);
     case 4: return b ? mqa_launch<bf16, 4>(a, rows, st) : mqa_launch<float, 4>(a, rows, st);
