@@ -176,6 +176,8 @@ class PrefillRunner:
         self.Cc = torch.empty(max(self.NB, 1), d.c, dtype=dt, device=dev)
         self.KI = torch.empty(max(self.NB, 1), d.cI, dtype=dt, device=dev)
         self.idx = torch.empty(self.T, d.topk, dtype=torch.int32, device=dev)
+        self.iws = torch.empty(csa.csa_indexer_workspace_bytes(d, self.T, self.nseq, self.maxlen), dtype=torch.uint8,
+                               device=dev)
 
     def forward(self):
         d = self.dims
@@ -209,7 +211,7 @@ class PrefillRunner:
             "A3_compress": a3,
             "A4_indexer_topk": lambda: csa.csa_indexer_topk(d, self.Y2, self.Y2.shape[1], self.wI, d.nhI, self.KI,
                                                             self.cu, self.cb, self.nseq, T, self.NB, self.maxlen,
-                                                            self.idx),
+                                                            self.idx, self.iws),
             "A5_sparse_mqa": lambda: csa.csa_sparse_mqa(d, self.Y2.data_ptr() + d.nhI * cI * es, self.Y2.shape[1],
                                                         self.Cc, self.idx, self.cu, self.cb, self.nseq, T,
                                                         self.NB, self.O),

@@ -26,7 +26,7 @@ EXPORTS = (
     "csa_sparse_mqa", "csa_forward_workspace_bytes", "csa_forward", "csa_ring_row_elems",
     "csa_cache_append", "csa_decode_workspace_bytes", "csa_decode", "csa_get_device_status",
     "csa_status_string", "csa_hidden_row_elems", "csa_query_row_elems", "csa_project_hidden",
-    "csa_project_query", "csa_launch_count",
+    "csa_project_query", "csa_launch_count", "csa_indexer_workspace_bytes",
 )
 
 
@@ -80,7 +80,8 @@ def lib() -> ctypes.CDLL:
             "csa_packed_weights_bytes": (sz, [D]),
             "csa_pack_weights": (i, [D, ctypes.POINTER(csa_weights), vp, sz, vp]),
             "csa_compress": (i, [D, vp, vp, vp, vp, i, vp, vp, i, vp, vp, i, i, i, vp, vp]),
-            "csa_indexer_topk": (i, [D, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp, vp]),
+            "csa_indexer_topk": (i, [D, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]),
+            "csa_indexer_workspace_bytes": (sz, [D, i, i, i]),
             "csa_sparse_mqa": (i, [D, vp, i, vp, vp, vp, vp, i, i, i, vp, vp]),
             "csa_forward_workspace_bytes": (sz, [D, i, i]),
             "csa_forward": (i, [D, vp, vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp]),
@@ -154,10 +155,15 @@ def csa_compress(dims: Dims, Ca, Cb, Za, Zb, ld, Ba, Bb, width, cu_seqlens, cu_b
                               _stream(stream)), "csa_compress")
 
 
+def csa_indexer_workspace_bytes(dims: Dims, total_tokens: int, nseq: int, max_seqlen: int) -> int:
+    return lib().csa_indexer_workspace_bytes(_d(dims), total_tokens, nseq, max_seqlen)
+
+
 def csa_indexer_topk(dims: Dims, qI, ld_qI, wI, ld_wI, KI, cu_seqlens, cu_blocks, nseq, total_tokens,
-                     total_blocks, max_seqlen, idx, stream=None):
+                     total_blocks, max_seqlen, idx, ws=None, stream=None):
     _check(lib().csa_indexer_topk(_d(dims), _p(qI), ld_qI, _p(wI), ld_wI, _p(KI), _p(cu_seqlens),
                                   _p(cu_blocks), nseq, total_tokens, total_blocks, max_seqlen, _p(idx),
+                                  _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                   _stream(stream)), "csa_indexer_topk")
 
 

@@ -14,6 +14,7 @@
 #include "gemm_simt.cuh"
 #include "gemm_tcgen05.cuh"
 #include "indexer_simt.cuh"
+#include "indexer_tcgen05.cuh"
 #include "mqa_simt.cuh"
 #include "mqa_tcgen05.cuh"
 #include "pack.cuh"
@@ -56,6 +57,19 @@ csa_status check_dims(const csa_dims* d) {
   return CSA_OK;
 }
 
+// ------------------------------------------------------------------ device facts
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
 // ------------------------------------------------------------------ layouts
 struct PackLayout {
   int N1b;    // bf16/f32 block of the H-side output: C^a C^b Z^a Z^b C^aI C^bI Z^aI Z^bI c^Q
@@ -86,7 +100,7 @@ PackLayout pack_layout(const csa_dims* d) {
 }
 
 struct FwdLayout {
-  size_t y1, wI, y2, ccomp, kicomp, idx, total;
+  size_t y1, wI, y2, ccomp, kicomp, idx, scratch, total;
 };
 
 FwdLayout fwd_layout(const csa_dims* d, int T) {
@@ -101,24 +115,12 @@ FwdLayout fwd_layout(const csa_dims* d, int T) {
   L.ccomp = off; off = align_up(off + nbmax * d->c * es);
   L.kicomp = off; off = align_up(off + nbmax * d->cI * es);
   L.idx = off; off = align_up(off + (size_t)T * d->topk * 4);
+  L.scratch = off; off = align_up(off + (size_t)sm_count() * 4 * (size_t)(T / d->m + 1) * 4);
   L.total = off;
   return L;
 }
 
 inline char* at(void* base, size_t off) { return static_cast<char*>(base) + off; }
-
-// ------------------------------------------------------------------ device facts
-int sm_count() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
-  }
-  return cached[dev];
-}
 
 // ------------------------------------------------------------------ TMA descriptors
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -149,6 +151,22 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 tensor [d2, d1, d0] (d0 innermost) with byte strides s1 (between
+// d1 rows) and s2 (between d2 slabs), read in boxes b0 x b1 x b2.
+bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                       uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  if (reinterpret_cast<uintptr_t>(base) % 16 || s1 % 16 || s2 % 16) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -240,6 +258,40 @@ csa_status indexer_launch(const IndexerArgs& a, int rows, size_t smem, cudaStrea
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return CSA_ERR_CUDA;
   k<<<rows, 256, smem, st>>>(a);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+// Whether the tensor-core indexer covers these dims (prefill rows only).
+bool indexer_tc_ok(const csa_dims* d) {
+  return d->dtype == CSA_BF16 && d->m == 4 && (d->nhI == 32 || d->nhI == 64) && (d->cI == 64 || d->cI == 128);
+}
+
+// Scratch of the tensor-core indexer: one row of candidate scores per query
+// of the item, per CTA.
+size_t indexer_scratch_bytes(int sc_cap) { return (size_t)sm_count() * 4 * (size_t)sc_cap * 4; }
+
+csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int NB, void* ws, size_t ws_bytes,
+                             cudaStream_t st) {
+  const int sc_cap = a.sc_cap > 0 ? a.sc_cap : 1;
+  if (!ws || ws_bytes < indexer_scratch_bytes(sc_cap) || reinterpret_cast<uintptr_t>(ws) % 16)
+    return CSA_ERR_WORKSPACE;
+  CUtensorMap tk, tq;
+  const uint64_t krows = NB > 0 ? (uint64_t)NB : 1;
+  if (!make_tmap_bf16(&tk, a.KI, d->cI, krows, (uint64_t)d->cI * 2, 64, idxtc::kM) ||
+      !make_tmap_bf16_3d(&tq, a.qI, d->cI, d->nhI, T, (uint64_t)d->cI * 2, (uint64_t)a.ld_qI * 2, 64, d->nhI, 4))
+    return CSA_ERR_UNSUPPORTED;
+  IdxTcArgs t;
+  t.wI = a.wI; t.ld_wI = a.ld_wI; t.idx = a.idx; t.scratch = static_cast<float*>(ws); t.sc_cap = sc_cap;
+  t.topk = d->topk; t.nhI = d->nhI; t.cI = d->cI;
+  t.cu_seqlens = a.rm.cu_seqlens; t.cu_blocks = a.rm.cu_blocks; t.nseq = a.rm.nseq; t.total_blocks = NB;
+  t.total_tokens = T;
+  if (cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)idxtc::kSmem) !=
+      cudaSuccess)
+    return CSA_ERR_CUDA;
+  const long long items = (long long)NB + a.rm.nseq;
+  const int grid = items < sm_count() ? (int)items : sm_count();
+  indexer_tc_kernel<<<grid, idxtc::kThreads, idxtc::kSmem, st>>>(tk, tq, t);
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }
@@ -480,9 +532,15 @@ csa_status csa_compress(const csa_dims* d, const void* Ca, const void* Cb, const
   return launch_compress(d, a, (cudaStream_t)stream);
 }
 
+size_t csa_indexer_workspace_bytes(const csa_dims* d, int total_tokens, int nseq, int max_seqlen) {
+  if (check_dims(d) != CSA_OK || total_tokens < 0 || nseq <= 0 || max_seqlen < 0) return 0;
+  return align_up(indexer_scratch_bytes(max_seqlen / d->m + 1));
+}
+
 csa_status csa_indexer_topk(const csa_dims* d, const void* qI, int ld_qI, const float* wI, int ld_wI,
                             const void* KI, const int* cu_seqlens, const int* cu_blocks, int nseq,
-                            int total_tokens, int total_blocks, int max_seqlen, int* idx, void* stream) {
+                            int total_tokens, int total_blocks, int max_seqlen, int* idx, void* ws,
+                            size_t ws_bytes, void* stream) {
   csa_status s = check_dims(d);
   if (s != CSA_OK) return s;
   if (!qI || !wI || !KI || !cu_seqlens || !cu_blocks || !idx) return CSA_ERR_INVALID_ARG;
@@ -495,6 +553,11 @@ csa_status csa_indexer_topk(const csa_dims* d, const void* qI, int ld_qI, const 
   a.topk = d->topk; a.nhI = d->nhI;
   a.sc_cap = max_seqlen / d->m;
   a.rm = RowMap{cu_seqlens, cu_blocks, nseq, total_blocks, nullptr, 0, d->m};
+  if (indexer_tc_ok(d) && ld_qI % 8 == 0 && reinterpret_cast<uintptr_t>(qI) % 16 == 0) {
+    if (total_tokens == 0) return CSA_OK;
+    a.sc_cap = max_seqlen / d->m + 1;
+    return launch_indexer_tc(d, a, total_tokens, total_blocks, ws, ws_bytes, (cudaStream_t)stream);
+  }
   return launch_indexer(d, a, total_tokens, (cudaStream_t)stream);
 }
 
@@ -572,7 +635,13 @@ csa_status csa_forward(const csa_dims* d, const void* packed, const void* H, con
   ia.qI = y2; ia.ld_qI = P.N2; ia.wI = wI; ia.ld_wI = d->nhI; ia.KI = KIc; ia.idx = idx;
   ia.topk = d->topk; ia.nhI = d->nhI; ia.sc_cap = max_seqlen / d->m;
   ia.rm = RowMap{cu_seqlens, cu_blocks, nseq, NB, nullptr, 0, d->m};
-  s = launch_indexer(d, ia, T, st);
+  if (indexer_tc_ok(d)) {
+    if (max_seqlen > T) max_seqlen = T;   // scratch rows are sized for T / m blocks
+    ia.sc_cap = max_seqlen / d->m + 1;
+    s = launch_indexer_tc(d, ia, T, NB, at(ws, L.scratch), L.total - L.scratch, st);
+  } else {
+    s = launch_indexer(d, ia, T, st);
+  }
   if (s != CSA_OK) return s;
   // A5: eq. (11)
   MqaArgs ma;

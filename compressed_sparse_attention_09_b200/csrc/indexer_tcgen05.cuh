@@ -1,0 +1,328 @@
+// Lightning indexer (eq. 8) and top-k selector (eq. 9) of "Compressed
+// Sparse Attention" (cnblogs) on the sm_100a tensor cores, prefill form.
+//
+// Work item = the 4 query tokens of one compression block (m = 4): they see
+// the same blocks s < floor(t/m), so they share every K^IComp tile.  Per
+// 128-block tile the MMA computes
+//     D[s, (q, h)] = K^IComp_s . q^I_{t_q, h}      M = 128 blocks, N = 4 x n_h^I, K = c^I
+// into one of two TMEM accumulators, and the epilogue warps (one TMEM lane =
+// one block s per thread) fold it straight into the index score
+//     I[t_q, s] = sum_h w_{t_q, h} ReLU(D[s, (q, h)])
+// so the per-head products never leave the SM.  The four score rows of the
+// item go to a per-CTA scratch row (read back through L2 only; the n x n/m
+// score matrix never exists), then each epilogue warp selects the exact
+// top-k of one query with a warp-level radix select and writes its indices
+// in ascending order (ties to the lower block).  Sequence tails (L mod 4
+// tokens) are extra items with fewer than 4 queries; items whose queries see
+// at most k blocks keep them all without any MMA.
+//
+// Warp roles (192 threads): warp 0 TMA producer (q^I of the item once, then
+// the K^IComp tiles through a kStages ring), warp 1 MMA issuer + TMEM owner,
+// warps 2-5 epilogue + selection.  All waits are bounded.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+
+struct IdxTcArgs {
+  const float* wI; long long ld_wI;   // [T, nhI]
+  int* idx;                           // [T, topk]
+  float* scratch;                     // [gridDim, 4, sc_cap]
+  int sc_cap;                         // >= max blocks of any sequence
+  int topk, nhI, cI;
+  const int* cu_seqlens; const int* cu_blocks;
+  int nseq, total_blocks, total_tokens;
+};
+
+namespace idxtc {
+constexpr int kM = 128;                 // blocks per tile
+constexpr int kStages = 4;
+constexpr int kQChunk = 256 * 128;      // [4 x nhI <= 256 rows x 64 bf16]
+constexpr int kKChunk = kM * 128;       // [128 rows x 64 bf16]
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + 2 * kQChunk;
+constexpr int kOffW = kOffK + kStages * 2 * kKChunk;   // 4 warps x [4 x 64] floats
+constexpr int kOffH = kOffW + 4 * 256 * 4;             // 4 warps x 256 bins
+constexpr int kOffB = kOffH + 4 * 256 * 4;
+constexpr size_t kSmem = 1024 + kOffB + 256;
+constexpr int kThreads = 192;
+}  // namespace idxtc
+
+// Item `it` of the work list: compression blocks from the last one down, then
+// one tail item per sequence.  Returns false for an empty tail item.
+__device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, int& nq, int& avail,
+                                         long long& kbase) {
+  if (it < a.total_blocks) {
+    const int g = a.total_blocks - 1 - it;
+    int lo = 0, hi = a.nseq;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (a.cu_blocks[mid] <= g) lo = mid; else hi = mid;
+    }
+    const int i = g - a.cu_blocks[lo];
+    tok0 = a.cu_seqlens[lo] + 4 * i;
+    nq = 4;
+    avail = i;
+    kbase = a.cu_blocks[lo];
+    return true;
+  }
+  const int b = it - a.total_blocks;
+  const int L = a.cu_seqlens[b + 1] - a.cu_seqlens[b];
+  nq = L & 3;
+  tok0 = a.cu_seqlens[b + 1] - nq;
+  avail = L >> 2;
+  kbase = a.cu_blocks[b];
+  return nq > 0;
+}
+
+// Exact top-k of sc[0..n) (n > k) by one warp, written to out[0..k) as
+// ascending indices; equal scores are taken lowest index first.
+__device__ void warp_topk_ascending(const float* sc, int n, int k, int* out, int* hist) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, mask = 0;
+  int kk = k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = lane; i < 256; i += 32) hist[i] = 0;
+    __syncwarp();
+    for (int s = lane; s < n; s += 32) {
+      const uint32_t key = ordered_key(__ldcg(sc + s));
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncwarp();
+    // lane L owns bins 255-8L .. 248-8L (descending); find the digit holding the kk-th largest
+    int cnt[8], tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - 8 * lane - j]; tot += cnt[j]; }
+    int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    const int excl = incl - tot;
+    const unsigned hit = __ballot_sync(0xffffffffu, excl < kk && incl >= kk);
+    const int src = __ffs(hit) - 1;
+    int digit = 0, before = 0;
+    if (lane == src) {
+      int c = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (c + cnt[j] >= kk) { digit = 255 - 8 * lane - j; before = c; break; }
+        c += cnt[j];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    before = __shfl_sync(0xffffffffu, before, src);
+    prefix |= (uint32_t)digit << shift;
+    mask |= 255u << shift;
+    kk -= before;
+    __syncwarp();
+  }
+  const uint32_t thr = prefix;
+  const int need_eq = kk;
+  int out_off = 0, eq_seen = 0;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = 0; base < n; base += 32) {
+    const int s = base + lane;
+    const uint32_t key = s < n ? ordered_key(__ldcg(sc + s)) : 0u;
+    const bool gt = s < n && key > thr;
+    const bool eq = s < n && key == thr;
+    const unsigned beq = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
+    const unsigned btk = __ballot_sync(0xffffffffu, take);
+    const int p = out_off + __popc(btk & lt);
+    if (take && p < k) out[p] = s;
+    out_off += __popc(btk);
+    eq_seen += __popc(beq);
+  }
+}
+
+__global__ void __launch_bounds__(idxtc::kThreads, 1)
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IdxTcArgs a) {
+  using namespace sm100;
+  using namespace idxtc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_s = sm + kOffQ;
+  uint8_t* k_s = sm + kOffK;
+  float* w_s = reinterpret_cast<float*>(sm + kOffW);
+  int* h_s = reinterpret_cast<int*>(sm + kOffH);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffB);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;                 // [kStages]
+  uint64_t* k_empty = k_full + kStages;        // [kStages]
+  uint64_t* t_full = k_empty + kStages;        // [2]
+  uint64_t* t_empty = t_full + 2;              // [2]
+  uint64_t* sc_done = t_empty + 2;             // scores of the item written (4 warps)
+  uint64_t* sel_done = sc_done + 1;            // selection of the item done (4 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sel_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = 4 * a.nhI;                      // MMA N: (query, head) pairs
+  const int kchunks = a.cI / 64;
+  const uint32_t tmem_cols = N <= 128 ? 256 : 512;
+  const int items = a.total_blocks + a.nseq;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&t_full[s], 1);
+      mbar_init(&t_empty[s], 4);
+    }
+    mbar_init(sc_done, 4);
+    mbar_init(sel_done, 4);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmQ);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t g = 0, qi = 0;
+      for (int it = blockIdx.x; it < items && !*abort_flag; it += gridDim.x) {
+        int tok0, nq, avail;
+        long long kbase;
+        if (!idx_item(a, it, tok0, nq, avail, kbase) || avail <= a.topk) continue;
+        const int ntiles = (avail + kM - 1) / kM;
+        if (!mbar_wait(q_empty, (qi & 1) ^ 1)) { *abort_flag = 1; break; }
+        mbar_arrive_expect_tx(q_full, (uint32_t)(kchunks * N * 128));
+        for (int c = 0; c < kchunks; ++c) tma_load_3d(&tmQ, q_full, q_s + c * kQChunk, 64 * c, 0, tok0);
+        ++qi;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j, ++g) {
+          const int st = g % kStages;
+          if (!mbar_wait(&k_empty[st], ((g / kStages) & 1) ^ 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[st], (uint32_t)(kchunks * kKChunk));
+          for (int c = 0; c < kchunks; ++c)
+            tma_load_2d(&tmK, &k_full[st], k_s + (st * 2 + c) * kKChunk, 64 * c, (int)(kbase + (long long)kM * j));
+        }
+        if (!ok) { *abort_flag = 1; break; }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kM, N);
+      uint32_t g = 0, qi = 0, acc_it = 0;
+      for (int it = blockIdx.x; it < items && !*abort_flag; it += gridDim.x) {
+        int tok0, nq, avail;
+        long long kbase;
+        if (!idx_item(a, it, tok0, nq, avail, kbase) || avail <= a.topk) continue;
+        const int ntiles = (avail + kM - 1) / kM;
+        if (!mbar_wait(q_full, qi & 1)) { *abort_flag = 1; break; }
+        ++qi;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j, ++g, ++acc_it) {
+          const int st = g % kStages, acc = acc_it & 1;
+          if (!mbar_wait(&k_full[st], (g / kStages) & 1) || !mbar_wait(&t_empty[acc], ((acc_it >> 1) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ka = smem_u32(k_s + st * 2 * kKChunk), qa = smem_u32(q_s);
+          for (int c = 0; c < kchunks; ++c)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              mma_bf16(tmem + (uint32_t)(acc * N), sdesc_k_sw128(ka + c * kKChunk + ks * 32),
+                       sdesc_k_sw128(qa + c * kQChunk + ks * 32), idesc, (c | ks) != 0);
+          mma_commit(&k_empty[st]);
+          mma_commit(&t_full[acc]);
+        }
+        if (!ok) { *abort_flag = 1; break; }
+        mma_commit(q_empty);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue + selection (warps 2-5)
+    const int sub = warp & 3;            // TMEM lane quarter; also the query this warp selects for
+    const int ew = warp - 2;             // epilogue warp index: private smem slices
+    float* w_my = w_s + ew * 256;
+    int* hist = h_s + ew * 256;
+    float* scr = a.scratch + (size_t)blockIdx.x * 4 * a.sc_cap;
+    const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
+    uint32_t acc_it = 0, wi = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+      if (warp_aborted(abort_flag)) break;
+      int tok0, nq, avail;
+      long long kbase;
+      if (!idx_item(a, it, tok0, nq, avail, kbase)) continue;
+      if (avail <= a.topk) {   // every visible block is kept
+        if (sub < nq) {
+          int* out = a.idx + (long long)(tok0 + sub) * a.topk;
+          for (int j = lane; j < a.topk; j += 32) out[j] = j < avail ? j : -1;
+        }
+        continue;
+      }
+      const int ntiles = (avail + kM - 1) / kM;
+      // this item's head weights, one private copy per warp
+      for (int e = lane; e < 4 * a.nhI; e += 32) {
+        const int q = e / a.nhI, h = e - q * a.nhI;
+        w_my[q * 64 + h] = q < nq ? a.wI[(long long)(tok0 + q) * a.ld_wI + h] : 0.f;
+      }
+      __syncwarp();
+      // the previous item's selection must be over before its scratch rows are overwritten
+      if (wi > 0 && !warp_wait(sel_done, (wi - 1) & 1)) { *abort_flag = 1; break; }
+      bool ok = true;
+      for (int j = 0; j < ntiles; ++j, ++acc_it) {
+        const int acc = acc_it & 1;
+        if (!warp_wait(&t_full[acc], (acc_it >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const int s = j * kM + 32 * sub + lane;
+        for (int q = 0; q < nq; ++q) {
+          float acc_s = 0.f;
+          for (int hc = 0; hc < a.nhI; hc += 32) {
+            float v[32];
+            tmem_ld_32x32b_x32(tmem + lane_base + (uint32_t)(acc * N + q * a.nhI + hc), v);
+            const float4* w4 = reinterpret_cast<const float4*>(w_my + q * 64 + hc);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float4 w = w4[e];
+              acc_s = fmaf(w.x, fmaxf(v[4 * e + 0], 0.f), acc_s);
+              acc_s = fmaf(w.y, fmaxf(v[4 * e + 1], 0.f), acc_s);
+              acc_s = fmaf(w.z, fmaxf(v[4 * e + 2], 0.f), acc_s);
+              acc_s = fmaf(w.w, fmaxf(v[4 * e + 3], 0.f), acc_s);
+            }
+          }
+          if (s < avail) __stcg(scr + (size_t)q * a.sc_cap + s, acc_s);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&t_empty[acc]);
+      }
+      if (!ok) { *abort_flag = 1; break; }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sc_done);
+      if (!warp_wait(sc_done, wi & 1)) { *abort_flag = 1; break; }
+      if (sub < nq)
+        warp_topk_ascending(scr + (size_t)sub * a.sc_cap, avail, a.topk, a.idx + (long long)(tok0 + sub) * a.topk,
+                            hist);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sel_done);
+      ++wi;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+}  // namespace csa

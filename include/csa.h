@@ -157,11 +157,17 @@ csa_status csa_compress(const csa_dims* dims, const void* Ca, const void* Cb, co
  * max_seqlen [host] : an upper bound of every sequence length (it sizes the
  *             per-query candidate storage; a longer sequence is clamped and
  *             flags CSA_ERR_BAD_METADATA).
+ * ws [dev]  : workspace of ws_bytes >= csa_indexer_workspace_bytes(), 256-byte
+ *             aligned, no initialisation needed.
  * The score matrix is never written to memory. */
 csa_status csa_indexer_topk(const csa_dims* dims, const void* qI, int ld_qI, const float* wI,
                             int ld_wI, const void* KI, const int* cu_seqlens, const int* cu_blocks,
                             int nseq, int total_tokens, int total_blocks, int max_seqlen, int* idx,
-                            void* stream);
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes csa_indexer_topk needs (per-CTA rows of candidate scores,
+ * kept on chip / in L2; 0 if the dims are invalid). */
+size_t csa_indexer_workspace_bytes(const csa_dims* dims, int total_tokens, int nseq, int max_seqlen);
 
 /* Shared-KV MQA over the selected entries, eqs. (10)-(11).
  * q [dev]     : [total_tokens, nh*c] (row stride ld_q), heads concatenated.

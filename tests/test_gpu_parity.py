@@ -119,8 +119,9 @@ def _indexer_case(dims, lens, seed, zero_w=False):
         wI.zero_()
     KI = synth.make_normal((NB, dims.cI), dims, seed + 2, std=0.5)
     idx = torch.full((T, dims.topk), 7, dtype=torch.int32, device=DEV)
+    ws = torch.empty(csa.csa_indexer_workspace_bytes(dims, T, len(lens), max(lens)), dtype=torch.uint8, device=DEV)
     csa.csa_indexer_topk(dims, qI.to(DEV), dims.nhI * dims.cI, wI.to(DEV), dims.nhI, KI.to(DEV), cu.to(DEV),
-                         cb.to(DEV), len(lens), T, NB, max(lens), idx)
+                         cb.to(DEV), len(lens), T, NB, max(lens), idx, ws)
     assert csa.csa_get_device_status() == 0
     idx = idx.cpu().numpy()
     q64, w64, K64 = f64(qI).reshape(T, dims.nhI, dims.cI), f64(wI), f64(KI)
@@ -154,6 +155,21 @@ def test_stage_indexer_large_k():
     assert kinds["exact"] > 0.5 * sum(kinds.values())
 
 
+@pytest.mark.parametrize("nhI,cI", [(64, 128), (32, 64)])
+@pytest.mark.parametrize("topk", [16, 100])
+def test_stage_indexer_topk_tensor_core(nhI, cI, topk):
+    """The tcgen05 indexer (m = 4): ragged packed sequences with tails of 1-3
+    tokens, sequences shorter than m, queries with fewer blocks than k."""
+    dims = csa.Dims(d=64, c=64, m=4, cI=cI, nhI=nhI, nh=2, dc=64, topk=topk, dtype=csa.CSA_BF16)
+    kinds = _indexer_case(dims, [1000, 130, 2, 67, 515, 1], 44 + topk)
+    assert kinds["exact"] > 0.8 * sum(kinds.values()), kinds
+
+
+def test_stage_indexer_tensor_core_ties_take_lowest_blocks():
+    dims = csa.Dims(d=64, c=64, m=4, cI=128, nhI=64, nh=2, dc=64, topk=37, dtype=csa.CSA_BF16)
+    _indexer_case(dims, [700, 9], 45, zero_w=True)
+
+
 def test_stage_indexer_topk_full_size_sampled():
     """The indexer stage at the n = 8192 prefill sizes (n_h^I = 64, c^I = 128,
     k = 512) on bit-identical bf16 inputs, every row checked against the
@@ -168,8 +184,9 @@ def test_stage_indexer_topk_full_size_sampled():
     wI = synth.make_normal((T, dims.nhI), dims, 72).float()
     KI = synth.make_normal((NB, dims.cI), dims, 73, std=0.5)
     idx = torch.empty((T, dims.topk), dtype=torch.int32, device=DEV)
+    ws = torch.empty(csa.csa_indexer_workspace_bytes(dims, T, 1, T), dtype=torch.uint8, device=DEV)
     csa.csa_indexer_topk(dims, qI.to(DEV), dims.nhI * dims.cI, wI.to(DEV), dims.nhI, KI.to(DEV), cu.to(DEV),
-                         cb.to(DEV), 1, T, NB, T, idx)
+                         cb.to(DEV), 1, T, NB, T, idx, ws)
     assert csa.csa_get_device_status() == 0
     idx = idx.cpu().numpy()
     q64, w64, K64 = f64(qI).reshape(T, dims.nhI, dims.cI), f64(wI), f64(KI)
