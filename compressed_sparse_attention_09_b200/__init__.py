@@ -9,5 +9,6 @@ from .capi import (CSA_BF16, CSA_F32, CsaError, Dims, csa_cache_append, csa_comp
                    csa_get_device_status, csa_indexer_topk, csa_pack_weights, csa_packed_weights_bytes,
                    csa_ring_row_elems, csa_sparse_mqa, lib, status_string,
                    csa_hidden_row_elems, csa_query_row_elems, csa_project_hidden, csa_project_query,
-                   csa_launch_count, csa_indexer_workspace_bytes)
+                   csa_launch_count, csa_indexer_workspace_bytes,
+                   csa_indexer_topk_noalloc)
 from .meta import cu_from_lengths  # noqa: F401

@@ -26,7 +26,7 @@ EXPORTS = (
     "csa_sparse_mqa", "csa_forward_workspace_bytes", "csa_forward", "csa_ring_row_elems",
     "csa_cache_append", "csa_decode_workspace_bytes", "csa_decode", "csa_get_device_status",
     "csa_status_string", "csa_hidden_row_elems", "csa_query_row_elems", "csa_project_hidden",
-    "csa_project_query", "csa_launch_count", "csa_indexer_workspace_bytes",
+    "csa_project_query", "csa_launch_count", "csa_indexer_workspace_bytes", "csa_indexer_topk_noalloc",
 )
 
 
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
             "csa_compress": (i, [D, vp, vp, vp, vp, i, vp, vp, i, vp, vp, i, i, i, vp, vp]),
             "csa_indexer_topk": (i, [D, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]),
             "csa_indexer_workspace_bytes": (sz, [D, i, i, i]),
+            "csa_indexer_topk_noalloc": (i, [D, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp, vp]),
             "csa_sparse_mqa": (i, [D, vp, i, vp, vp, vp, vp, i, i, i, vp, vp]),
             "csa_forward_workspace_bytes": (sz, [D, i, i]),
             "csa_forward": (i, [D, vp, vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp]),
@@ -165,6 +166,14 @@ def csa_indexer_topk(dims: Dims, qI, ld_qI, wI, ld_wI, KI, cu_seqlens, cu_blocks
                                   _p(cu_blocks), nseq, total_tokens, total_blocks, max_seqlen, _p(idx),
                                   _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                   _stream(stream)), "csa_indexer_topk")
+
+
+def csa_indexer_topk_noalloc(dims: Dims, qI, ld_qI, wI, ld_wI, KI, cu_seqlens, cu_blocks, nseq, total_tokens,
+                             total_blocks, max_seqlen, idx, stream=None):
+    """csa_indexer_topk without a workspace argument (see include/csa.h)."""
+    _check(lib().csa_indexer_topk_noalloc(_d(dims), _p(qI), ld_qI, _p(wI), ld_wI, _p(KI), _p(cu_seqlens),
+                                          _p(cu_blocks), nseq, total_tokens, total_blocks, max_seqlen, _p(idx),
+                                          _stream(stream)), "csa_indexer_topk_noalloc")
 
 
 def csa_sparse_mqa(dims: Dims, q, ld_q, Ccomp, idx, cu_seqlens, cu_blocks, nseq, total_tokens,

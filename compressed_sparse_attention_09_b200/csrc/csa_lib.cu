@@ -578,6 +578,62 @@ csa_status csa_sparse_mqa(const csa_dims* d, const void* q, int ld_q, const void
   return launch_mqa(d, a, total_tokens, (cudaStream_t)stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------- indexer without a caller workspace
+// Scratch of csa_indexer_topk_noalloc: the tensor-core indexer's per-CTA
+// score rows (4 rows of up to kNoAllocMaxBlocks scores for each of up to
+// kNoAllocMaxCtas CTAs), held in module memory for the life of the process
+// on every GPU that loads the library (10 MiB).
+constexpr int kNoAllocMaxCtas = 160;
+constexpr int kNoAllocMaxBlocks = 4096;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxCtas * 4 * kNoAllocMaxBlocks];
+
+namespace {
+// Device address of g_noalloc_scratch on the current device.  The host-side
+// name is only a stand-in, so the address is looked up once per device (with
+// that device current) and cached.
+float* noalloc_scratch() {
+  static std::atomic<float*> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  float* p = cached[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    p = static_cast<float*>(q);
+    cached[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+}  // namespace
+
+extern "C" {
+
+csa_status csa_indexer_topk_noalloc(const csa_dims* d, const void* qI, int ld_qI, const float* wI, int ld_wI,
+                                    const void* KI, const int* cu_seqlens, const int* cu_blocks, int nseq,
+                                    int total_tokens, int total_blocks, int max_seqlen, int* idx, void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!qI || !wI || !KI || !cu_seqlens || !cu_blocks || !idx) return CSA_ERR_INVALID_ARG;
+  if (nseq <= 0 || total_tokens < 0 || total_blocks < 0 || max_seqlen < 0) return CSA_ERR_INVALID_ARG;
+  if (ld_qI < d->nhI * d->cI || ld_wI < d->nhI) return CSA_ERR_INVALID_ARG;
+  if (!indexer_tc_ok(d) || ld_qI % 8 || reinterpret_cast<uintptr_t>(qI) % 16 ||
+      reinterpret_cast<uintptr_t>(KI) % 16)
+    return CSA_ERR_UNSUPPORTED;
+  const int sc_cap = max_seqlen / d->m + 1;
+  if (sc_cap > kNoAllocMaxBlocks || sm_count() > kNoAllocMaxCtas) return CSA_ERR_UNSUPPORTED;
+  float* scratch = noalloc_scratch();
+  if (!scratch) return CSA_ERR_CUDA;
+  if (total_tokens == 0) return CSA_OK;
+  IndexerArgs a;
+  a.qI = qI; a.ld_qI = ld_qI; a.wI = wI; a.ld_wI = ld_wI; a.KI = KI; a.idx = idx;
+  a.topk = d->topk; a.nhI = d->nhI; a.sc_cap = sc_cap;
+  a.rm = RowMap{cu_seqlens, cu_blocks, nseq, total_blocks, nullptr, 0, d->m};
+  return launch_indexer_tc(d, a, total_tokens, total_blocks, scratch, sizeof(g_noalloc_scratch),
+                           (cudaStream_t)stream);
+}
+
 size_t csa_forward_workspace_bytes(const csa_dims* d, int total_tokens, int nseq) {
   if (check_dims(d) != CSA_OK || total_tokens < 0 || nseq <= 0) return 0;
   return fwd_layout(d, total_tokens).total;

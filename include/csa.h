@@ -169,6 +169,31 @@ csa_status csa_indexer_topk(const csa_dims* dims, const void* qI, int ld_qI, con
  * kept on chip / in L2; 0 if the dims are invalid). */
 size_t csa_indexer_workspace_bytes(const csa_dims* dims, int total_tokens, int nseq, int max_seqlen);
 
+/* csa_indexer_topk for callers that cannot allocate device memory.
+ * The page has no counterpart: this is an interface addition, not a step of
+ * the method.  Some callers own no allocator: code that runs where a
+ * cudaMalloc is not allowed (a process whose device memory is handed out by
+ * another framework's pool, or a latency-critical loop that must not
+ * allocate after start-up) cannot provide the indexer's workspace.  This
+ * entry point takes the same arguments minus the workspace and instead uses
+ * a fixed scratch array that lives in the library's module memory (10 MiB on
+ * every GPU that loads the library, held until the process exits).
+ * Limits: the tensor-core indexer's shapes only (bf16, m = 4, nhI in {32, 64},
+ * cI in {64, 128}, qI and KI 16-byte aligned, ld_qI a multiple of 8) and
+ * max_seqlen / m + 1 <= 4096 (max_seqlen <= 16380 for m = 4); anything else
+ * returns CSA_ERR_UNSUPPORTED before any launch.  It calls no allocating
+ * routine.  The first call on a device looks up the scratch array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  Every call shares the one array: calls
+ * whose kernels overlap on the GPU (e.g. on two streams) race on it; calls in
+ * one stream are safe.  The array's contents carry over between calls; no
+ * part of it needs to start at zero (each score is written before it is
+ * read).  Output identical to csa_indexer_topk. */
+csa_status csa_indexer_topk_noalloc(const csa_dims* dims, const void* qI, int ld_qI, const float* wI,
+                                    int ld_wI, const void* KI, const int* cu_seqlens,
+                                    const int* cu_blocks, int nseq, int total_tokens, int total_blocks,
+                                    int max_seqlen, int* idx, void* stream);
+
 /* Shared-KV MQA over the selected entries, eqs. (10)-(11).
  * q [dev]     : [total_tokens, nh*c] (row stride ld_q), heads concatenated.
  * Ccomp [dev] : [total_blocks, c] compressed entries (keys AND values).
