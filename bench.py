@@ -449,6 +449,29 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_stage(args):
+    """Runs one stage of the prefill workload (after one full forward that fills
+    its inputs) warmup + steps times; for profiling a single kernel."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.workloads()[args.workload]
+    runner = PrefillRunner(w, dev)
+    fn = runner.stages()[args.stage]
+    # inputs of every stage: one pass of the stages in order
+    for name, f in runner.stages().items():
+        f()
+        if name == args.stage:
+            break
+    for _ in range(args.warmup + args.steps):
+        fn()
+    torch.cuda.synchronize()
+    st = csa.csa_get_device_status()
+    print(json.dumps({"stage": args.stage, "workload": args.workload, "launches": args.warmup + args.steps,
+                      "status": csa.status_string(st)}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
+
+
 def runner_T(w):
     return sum(w.seqlens)
 
@@ -464,6 +487,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-stages", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--stage", choices=["A1_project_hidden", "A2_project_query", "A3_compress", "A4_indexer_topk",
+                                        "A5_sparse_mqa"], help="run only this stage (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -472,6 +497,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.stage:
+        run_stage(args)
         return
     if world > 1:
         import datetime
