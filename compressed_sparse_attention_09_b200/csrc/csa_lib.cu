@@ -324,12 +324,16 @@ csa_status mqa_launch(const MqaArgs& a, int rows, cudaStream_t st) {
 csa_status launch_mqa(const csa_dims* d, const MqaArgs& a, int rows, cudaStream_t st) {
   if (rows == 0) return CSA_OK;
   const bool b = d->dtype == CSA_BF16;
-  if (b && d->c == mqa::kC && d->nh % mqa::kHeads == 0 && a.ld_q % 8 == 0 && a.ld_O % 8 == 0 &&
+  if (b && d->c == mqa::kC && d->nh % mqa::kHeads == 0 && a.topk <= mqa::kMaxTopk && a.ld_q % 8 == 0 &&
+      a.ld_O % 8 == 0 &&
       reinterpret_cast<uintptr_t>(a.q) % 16 == 0 && reinterpret_cast<uintptr_t>(a.O) % 16 == 0 &&
       reinterpret_cast<uintptr_t>(a.C) % 16 == 0) {
-    // tensor-core path: c = 512, heads in groups of 64
+    // tensor-core path: c = 512, heads in groups of 64, q read through a 3-D tensor map
+    CUtensorMap tq;
+    if (!make_tmap_bf16_3d(&tq, a.q, mqa::kC, d->nh, rows, (uint64_t)mqa::kC * 2, (uint64_t)a.ld_q * 2, 64,
+                           mqa::kHeads, 1))
+      return CSA_ERR_UNSUPPORTED;
     MqaTcArgs t;
-    t.q = static_cast<const bf16*>(a.q); t.ld_q = a.ld_q;
     t.C = static_cast<const bf16*>(a.C); t.idx = a.idx;
     t.O = static_cast<bf16*>(a.O); t.ld_O = a.ld_O;
     t.topk = a.topk; t.nh = a.nh; t.rows = rows; t.scale_log2 = a.scale_log2; t.rm = a.rm;
@@ -338,7 +342,7 @@ csa_status launch_mqa(const csa_dims* d, const MqaArgs& a, int rows, cudaStream_
       return CSA_ERR_CUDA;
     const long long items = (long long)rows * (d->nh / mqa::kHeads);
     const int grid = items < sm_count() ? (int)items : sm_count();
-    mqa_tc_kernel<<<grid, mqa::kThreads, mqa::kSmem, st>>>(t);
+    mqa_tc_kernel<<<grid, mqa::kThreads, mqa::kSmem, st>>>(tq, t);
     CSA_CHECK_LAUNCH();
     return CSA_OK;
   }

@@ -3,10 +3,10 @@
 //
 // Work item = one query row and a group of 64 of its heads (decode rows with
 // n_h = 128 make two items).  For each item the CTA gathers the selected
-// entries 64 at a time and, per tile,
-//     S  = q . C_tile^T          tcgen05.mma M=64 (heads) N=64 (entries) K=512
+// entries 32 at a time and, per tile,
+//     S  = q . C_tile^T          tcgen05.mma M=64 (heads) N=32 (entries) K=512
 //     P  = exp2(S * log2e/sqrt(c) - m)     online softmax, one head per thread
-//     O += P . C_tile            tcgen05.mma M=64 (heads) N=256 (x2)  K=64
+//     O += P . C_tile            tcgen05.mma M=64 (heads) N=256 (x2)  K=32
 // The gathered tile sits in shared memory once, in the 128-byte-swizzled
 // layout; the S product reads it as a K-major operand (rows = entries) and
 // the O product reads the very same bytes as an MN-major operand (rows =
@@ -14,16 +14,17 @@
 // key and value.  With M = 64 the accumulator occupies half of each TMEM lane
 // quarter, so the 64 x 512 fp32 O lives in 256 columns (channels 0-255 in the
 // lower 16 lanes of every quarter, 256-511 in the upper 16) next to two
-// 64-column S buffers.  Each softmax thread owns one head row of S: max, sum
+// 32-column S buffers.  Each softmax thread owns one head row of S: max, sum
 // and the P row need no cross-thread reduction.  O is rescaled (TMEM load,
 // multiply, store) only when a head's running maximum grows by more than 8 in
 // log2 units; otherwise the stale maximum is kept, which is exact because O
 // and the normaliser l share it.
 //
-// Warp roles (288 threads): warps 0-3 gather q and the entry tiles with
-// 16-byte cp.async (zero-filling rows past the selection), warp 4 issues the
-// MMAs (one thread) and owns TMEM, warps 5-8 run the softmax and the output
-// epilogue.  All waits are bounded (sm100::mbar_wait).
+// Warp roles (224 threads): warps 0-1 gather the entry tiles with 16-byte
+// cp.async into a 4-deep ring (completion is tracked by the stage's mbarrier,
+// so the gathers never block); thread 0 also loads q with a 3-D TMA; warp 2
+// issues the MMAs (one thread) and owns TMEM; warps 3-6 run the softmax and
+// the output epilogue.  All waits are bounded (sm100::mbar_wait).
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -31,7 +32,6 @@
 namespace csa {
 
 struct MqaTcArgs {
-  const __nv_bfloat16* q; long long ld_q;   // [rows, nh*512]
   const __nv_bfloat16* C;                   // entries [*, 512]
   const int* idx;                           // [rows, topk]
   __nv_bfloat16* O; long long ld_O;         // [rows, nh*512]
@@ -41,18 +41,22 @@ struct MqaTcArgs {
 };
 
 namespace mqa {
-constexpr int kC = 512, kHeads = 64, kTile = 64;
-constexpr int kChunk = 64 * 128;            // [64 rows x 64 bf16], 128-byte rows, swizzled
-constexpr int kQBytes = 8 * kChunk;         // 64 x 512
-constexpr int kCBytes = 8 * kChunk;         // one tile: 64 entries x 512
-constexpr int kPBytes = kChunk;             // 64 heads x 64 entries
+constexpr int kC = 512, kHeads = 64, kTile = 32, kStages = 4;
+constexpr int kQChunk = 64 * 128;           // [64 heads x 64 bf16], 128-byte rows, swizzled
+constexpr int kCChunk = kTile * 128;        // [32 entries x 64 bf16]
+constexpr int kQBytes = 8 * kQChunk;        // 64 x 512
+constexpr int kCBytes = 8 * kCChunk;        // one tile: 32 entries x 512
+constexpr int kPBytes = 64 * 128;           // 64 heads x 32 entries (rows padded to 128 B), swizzled
+constexpr int kMaxTopk = 4096;
+constexpr int kProducers = 64;              // threads of warps 0-1
 constexpr int kOffQ = 0;
 constexpr int kOffC = kOffQ + kQBytes;
-constexpr int kOffP = kOffC + 2 * kCBytes;
-constexpr int kOffMisc = kOffP + 2 * kPBytes;
+constexpr int kOffP = kOffC + kStages * kCBytes;
+constexpr int kOffIdx = kOffP + 2 * kPBytes;
+constexpr int kOffMisc = kOffIdx + kMaxTopk * 4;
 constexpr int kMiscBytes = 256;
 constexpr size_t kSmem = 1024 + kOffMisc + kMiscBytes;
-constexpr int kThreads = 288;
+constexpr int kThreads = 224;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256;
 }  // namespace mqa
@@ -60,7 +64,7 @@ constexpr uint32_t kColO = 0, kColS = 256;
 // byte offset of 16-byte unit u (0..7) of row r in a 128-byte-swizzled chunk
 __device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
-// Number of 64-entry tiles a query row needs: up to its last valid slot
+// Number of kTile-entry tiles a query row needs: up to its last valid slot
 // (0 <= s < avail).  Every warp role derives it on its own from the index
 // row, so no role depends on another's shared-memory copy of it.
 __device__ __forceinline__ int mqa_ntiles(const int* ir, int topk, int avail) {
@@ -74,7 +78,8 @@ __device__ __forceinline__ int mqa_ntiles(const int* ir, int topk, int avail) {
   return (last + mqa::kTile) / mqa::kTile;
 }
 
-__global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
+__global__ void __launch_bounds__(mqa::kThreads, 1)
+    mqa_tc_kernel(const __grid_constant__ CUtensorMap tmQ, MqaTcArgs a) {
   using namespace sm100;
   using namespace mqa;
   extern __shared__ uint8_t smem_raw[];
@@ -82,48 +87,53 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
   uint8_t* q_s = sm + kOffQ;
   uint8_t* c_s = sm + kOffC;
   uint8_t* p_s = sm + kOffP;
+  int* idx_s = reinterpret_cast<int*>(sm + kOffIdx);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffMisc);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* c_full = bars + 2;      // [2]
-  uint64_t* s_full = bars + 4;      // [2]
-  uint64_t* s_free = bars + 6;      // [2]
-  uint64_t* p_full = bars + 8;      // [2]
-  uint64_t* t_done = bars + 10;     // [2]  O of the tile done: frees its C stage and P buffer
-  uint64_t* o_free = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
-  uint32_t* mask_s = reinterpret_cast<uint32_t*>(bars + 14);   // [2 stages][2 words]: valid rows of the tile
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 16);
+  uint64_t* c_full = bars + 2;                 // [kStages]
+  uint64_t* t_done = c_full + kStages;         // [kStages]  O of the tile done: frees its C stage
+  uint64_t* s_full = t_done + kStages;         // [2]
+  uint64_t* s_free = s_full + 2;               // [2]
+  uint64_t* p_full = s_free + 2;               // [2]
+  uint64_t* o_free = p_full + 2;
+  uint64_t* i_free = o_free + 1;               // both producer warps done with an item's idx copy
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(i_free + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hgroups = a.nh / kHeads;
   const int items = a.rows * hgroups;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 128);
+    mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&c_full[s], kProducers);
+      mbar_init(&t_done[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&c_full[s], 128);
       mbar_init(&s_full[s], 1);
       mbar_init(&s_free[s], 4);
       mbar_init(&p_full[s], 4);
-      mbar_init(&t_done[s], 1);
     }
     mbar_init(o_free, 4);
+    mbar_init(i_free, 2);
     *abort_flag = 0;
     fence_barrier_init();
+    tma_prefetch_desc(&tmQ);
   }
-  if (warp == 4) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 2) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
-    // ------------------------------------------------------------ producers (warps 0-3)
-    const int tid = threadIdx.x;
-    uint32_t g = 0, qi = 0;
-    for (int it = blockIdx.x; it < items; it += gridDim.x, ++qi) {
+  if (warp < 2) {
+    // ------------------------------------------------------------ producers (warps 0-1)
+    const int tid = threadIdx.x;   // 0..63
+    uint32_t g = 0, qw = 0, ii = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x, ++ii) {
       if (warp_aborted(abort_flag)) break;
       const int row = a.rows - 1 - it / hgroups, hg = it % hgroups;
       long long base;
@@ -131,54 +141,53 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
       row_entries(a.rm, row, base, avail);
       const int* ir = a.idx + (long long)row * a.topk;
       const int ntiles = mqa_ntiles(ir, a.topk, avail);
-      if (!warp_wait(q_empty, (qi & 1) ^ 1)) { *abort_flag = 1; break; }
-      if (ntiles > 0) {
-        const __nv_bfloat16* qrow = a.q + (long long)row * a.ld_q + (long long)hg * kHeads * kC;
-        for (int i = 0; i < 32; ++i) {
-          const int u = tid + 128 * i, r = u >> 6, c16 = u & 63;
-          cp_async16(q_s + (c16 >> 3) * kChunk + sw128(r, c16 & 7), qrow + (long long)r * kC + c16 * 8, 16);
-        }
+      // both producer warps must be done reading the previous item's idx copy
+      if (ii > 0 && !warp_wait(i_free, (ii - 1) & 1)) { *abort_flag = 1; break; }
+      // each warp writes the whole copy (identical values), so its own reads need only __syncwarp
+      for (int j = lane; j < ntiles * kTile; j += 32) {
+        const int s = j < a.topk ? ir[j] : -1;
+        const bool v = s >= 0 && s < avail;
+        if (warp == 0 && !v && s != -1) flag_status(kStatusBadIndex);
+        idx_s[j] = v ? s : -1;
       }
-      cp_async_commit();
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(q_full);
+      __syncwarp();
+      if (ntiles > 0) {
+        if (tid == 0) {
+          if (!mbar_wait(q_empty, (qw & 1) ^ 1)) {
+            *abort_flag = 1;
+          } else {
+            mbar_arrive_expect_tx(q_full, (uint32_t)kQBytes);
+            for (int kc = 0; kc < 8; ++kc) tma_load_3d(&tmQ, q_full, q_s + kc * kQChunk, 64 * kc, 64 * hg, row);
+          }
+        }
+        ++qw;
+      }
       bool ok = true;
       for (int j = 0; j < ntiles; ++j, ++g) {
-        const int st = g & 1;
-        if (!warp_wait(&t_done[st], ((g >> 1) & 1) ^ 1)) { ok = false; break; }
-        if (warp < 2) {   // rows 32*warp .. 32*warp+31 of the tile: validity bits
-          const int e = j * kTile + tid;
-          const int s = e < a.topk ? ir[e] : -1;
-          const bool v = s >= 0 && s < avail;
-          if (!v && s != -1) flag_status(kStatusBadIndex);
-          const unsigned bal = __ballot_sync(0xffffffffu, v);
-          if (lane == 0) mask_s[st * 2 + warp] = bal;
-        }
+        const int st = g % kStages;
+        if (!warp_wait(&t_done[st], ((g / kStages) & 1) ^ 1)) { ok = false; break; }
         uint8_t* cst = c_s + st * kCBytes;
-        for (int i = 0; i < 32; ++i) {
-          const int u = tid + 128 * i, r = u >> 6, c16 = u & 63;
-          const int e = j * kTile + r;
-          const int s = e < a.topk ? ir[e] : -1;
-          const bool v = s >= 0 && s < avail;
-          const __nv_bfloat16* src = v ? a.C + (base + s) * kC + c16 * 8 : a.C;
-          cp_async16(cst + (c16 >> 3) * kChunk + sw128(r, c16 & 7), src, v ? 16u : 0u);
+#pragma unroll 4
+        for (int i = 0; i < kTile * 64 / kProducers; ++i) {
+          const int u = tid + kProducers * i, r = u >> 6, c16 = u & 63;
+          const int s = idx_s[j * kTile + r];
+          const __nv_bfloat16* src = s >= 0 ? a.C + (base + s) * kC + c16 * 8 : a.C;
+          cp_async16(cst + (c16 >> 3) * kCChunk + sw128(r, c16 & 7), src, s >= 0 ? 16u : 0u);
         }
-        cp_async_commit();
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(&c_full[st]);
+        cp_async_arrive_noinc(&c_full[st]);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(i_free);
       if (!ok) { *abort_flag = 1; break; }
     }
     cp_async_wait_all();
-  } else if (warp == 4) {
-    // ------------------------------------------------------------ MMA issuer (warp 4, lane 0 issues)
-    constexpr uint32_t idS = idesc_bf16_f32(64, 64);
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ MMA issuer (warp 2, lane 0 issues)
+    constexpr uint32_t idS = idesc_bf16_f32(64, kTile);
     constexpr uint32_t idO = idesc_bf16_f32_bmn(64, 256);
     const uint32_t q_addr = smem_u32(q_s);
-    uint32_t g = 0, qi = 0;
-    for (int it = blockIdx.x; it < items; it += gridDim.x, ++qi) {
+    uint32_t g = 0, qw = 0, oi = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x, ++oi) {
       if (warp_aborted(abort_flag)) break;
       const int row = a.rows - 1 - it / hgroups;
       long long base;
@@ -187,12 +196,12 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
       const int ntiles = mqa_ntiles(a.idx + (long long)row * a.topk, a.topk, avail);
       int ok = 1;
       if (lane == 0) {
-        auto issue_o = [&](uint32_t gj, int jj) -> bool {
-          const int st = gj & 1;
-          if (!mbar_wait(&p_full[st], (gj >> 1) & 1)) return false;
-          if (jj == 0 && !mbar_wait(o_free, (qi & 1) ^ 1)) return false;
+        auto issue_o = [&](uint32_t gj, uint32_t jj) -> bool {
+          const int st = gj % kStages, pb = gj & 1;
+          if (!mbar_wait(&p_full[pb], (gj >> 1) & 1)) return false;
+          if (jj == 0 && !mbar_wait(o_free, (oi & 1) ^ 1)) return false;   // previous item's O stored
           tc_fence_after();
-          const uint32_t pa = smem_u32(p_s + st * kPBytes);
+          const uint32_t pa = smem_u32(p_s + pb * kPBytes);
           const uint32_t ca = smem_u32(c_s + st * kCBytes);
 #pragma unroll
           for (int ks = 0; ks < kTile / 16; ++ks) {
@@ -200,34 +209,34 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
               mma_bf16(tmem + ((uint32_t)(16 * hh) << 16) + kColO, ad,
-                       sdesc_mn_sw128(ca + 4 * hh * kChunk + ks * 2048, kChunk, 1024), idO, (jj > 0 || ks > 0));
+                       sdesc_mn_sw128(ca + 4 * hh * kCChunk + ks * 2048, kCChunk, 1024), idO, (jj > 0 || ks > 0));
           }
           mma_commit(&t_done[st]);
           return true;
         };
-        if (!mbar_wait(q_full, qi & 1)) {
+        if (ntiles == 0) {
+          if (!mbar_wait(o_free, (oi & 1) ^ 1)) ok = 0;     // keep one o_free phase per item
+        } else if (!mbar_wait(q_full, qw & 1)) {
           ok = 0;
-        } else if (ntiles == 0) {
-          mma_commit(q_empty);
-          if (!mbar_wait(o_free, (qi & 1) ^ 1)) ok = 0;
         } else {
           tc_fence_after();
           for (int j = 0; j < ntiles && ok; ++j) {
             const uint32_t gj = g + j;
-            const int st = gj & 1;
-            if (!mbar_wait(&c_full[st], (gj >> 1) & 1) || !mbar_wait(&s_free[st], ((gj >> 1) & 1) ^ 1)) {
+            const int st = gj % kStages, sb = gj & 1;
+            if (!mbar_wait(&c_full[st], (gj / kStages) & 1) || !mbar_wait(&s_free[sb], ((gj >> 1) & 1) ^ 1)) {
               ok = 0;
               break;
             }
+            fence_proxy_async_smem();
             tc_fence_after();
             const uint32_t ca = smem_u32(c_s + st * kCBytes);
 #pragma unroll
             for (int kc = 0; kc < 8; ++kc)
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + kColS + 64 * st, sdesc_k_sw128(q_addr + kc * kChunk + ks * 32),
-                         sdesc_k_sw128(ca + kc * kChunk + ks * 32), idS, (kc | ks) != 0);
-            mma_commit(&s_full[st]);
+                mma_bf16(tmem + kColS + kTile * sb, sdesc_k_sw128(q_addr + kc * kQChunk + ks * 32),
+                         sdesc_k_sw128(ca + kc * kCChunk + ks * 32), idS, (kc | ks) != 0);
+            mma_commit(&s_full[sb]);
             if (j == ntiles - 1) mma_commit(q_empty);
             if (j >= 1 && !issue_o(gj - 1, j - 1)) ok = 0;
           }
@@ -236,22 +245,24 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) { if (lane == 0) *abort_flag = 1; break; }
+      if (ntiles > 0) ++qw;
       g += ntiles;
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue (warps 5-8)
+    // ------------------------------------------------------------ softmax + epilogue (warps 3-6)
     const int sub = warp & 3;                  // TMEM lane quarter of this warp
     const int hrow = 16 * sub + (lane & 15);   // head row (within the group) of lanes 0-15
     const int half = lane >> 4;                // O channel half held by this lane
     const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
-    uint32_t g = 0, qi = 0;
-    for (int it = blockIdx.x; it < items; it += gridDim.x, ++qi) {
+    uint32_t g = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
       if (warp_aborted(abort_flag)) break;
       const int row = a.rows - 1 - it / hgroups, hg = it % hgroups;
       long long base;
       int avail;
       row_entries(a.rm, row, base, avail);
-      const int ntiles = mqa_ntiles(a.idx + (long long)row * a.topk, a.topk, avail);
+      const int* ir = a.idx + (long long)row * a.topk;
+      const int ntiles = mqa_ntiles(ir, a.topk, avail);
       __nv_bfloat16* orow = a.O + (long long)row * a.ld_O + (long long)(hg * kHeads + hrow) * kC + half * 256;
       if (ntiles == 0) {
         const uint4 z = make_uint4(0, 0, 0, 0);
@@ -264,29 +275,31 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
       bool ok = true;
       for (int j = 0; j < ntiles; ++j) {
         const uint32_t gj = g + j;
-        const int st = gj & 1;
-        if (!warp_wait(&s_full[st], (gj >> 1) & 1) || !warp_wait(&c_full[st], (gj >> 1) & 1)) { ok = false; break; }
+        const int sb = gj & 1;
+        // validity of this tile's 32 rows, from the index row itself
+        const int e = j * kTile + lane;
+        const int sidx = e < a.topk ? ir[e] : -1;
+        const uint32_t vmask = __ballot_sync(0xffffffffu, sidx >= 0 && sidx < avail);
+        if (!warp_wait(&s_full[sb], (gj >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        float sv[64];
-        tmem_ld_32x32b_x32(tmem + lane_base + kColS + 64 * st, sv);
-        tmem_ld_32x32b_x32(tmem + lane_base + kColS + 64 * st + 32, sv + 32);
+        float sv[kTile];
+        tmem_ld_32x32b_x32(tmem + lane_base + kColS + kTile * sb, sv);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[st]);
-        const uint32_t mlo = mask_s[st * 2], mhi = mask_s[st * 2 + 1];
+        if (lane == 0) mbar_arrive(&s_free[sb]);
         float tmax = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          const bool v = ((e < 32 ? mlo >> e : mhi >> (e - 32)) & 1u) != 0;
-          sv[e] = v ? sv[e] * a.scale_log2 : -INFINITY;
-          tmax = fmaxf(tmax, sv[e]);
+        for (int q = 0; q < kTile; ++q) {
+          sv[q] = ((vmask >> q) & 1u) ? sv[q] * a.scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, sv[q]);
         }
         const float m_new = fmaxf(m_run, tmax);
         const bool grow = half == 0 && m_new > m_run + 8.f;   // also true on the first finite tile
         const float m_use = grow ? m_new : m_run;
         if (__any_sync(0xffffffffu, grow && j > 0)) {
           // rescale O: the O MMAs of the earlier tiles must have completed
-          if (!warp_wait(&t_done[(gj - 1) & 1], ((gj - 1) >> 1) & 1)) { ok = false; break; }
+          const uint32_t gp = gj - 1;
+          if (!warp_wait(&t_done[gp % kStages], (gp / kStages) & 1)) { ok = false; break; }
           tc_fence_after();
           float alpha = grow ? exp2f(m_run - m_new) : 1.f;    // exp2(-inf) = 0 when nothing was seen
           alpha = __shfl_sync(0xffffffffu, alpha, lane & 15);
@@ -295,7 +308,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
             float v[32];
             tmem_ld_32x32b_x32(tmem + lane_base + kColO + ch * 32, v);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= alpha;
+            for (int q = 0; q < 32; ++q) v[q] *= alpha;
             tmem_st_32x32b_x32(tmem + lane_base + kColO + ch * 32, v);
           }
           tmem_st_wait();
@@ -304,19 +317,22 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
         }
         m_run = m_use;
         // P rows (lanes 0-15), once the P buffer's previous reader (tile gj-2) is done
-        if (gj >= 2 && !warp_wait(&t_done[st], ((gj >> 1) & 1) ^ 1)) { ok = false; break; }
+        if (gj >= 2) {
+          const uint32_t gp = gj - 2;
+          if (!warp_wait(&t_done[gp % kStages], (gp / kStages) & 1)) { ok = false; break; }
+        }
         if (half == 0) {
-          uint8_t* prow = p_s + st * kPBytes;
+          uint8_t* prow = p_s + sb * kPBytes;
           float sum = 0.f;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
+          for (int u = 0; u < kTile / 8; ++u) {
             Vec16<__nv_bfloat16> pk;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float x = sv[8 * u + e];
+            for (int q = 0; q < 8; ++q) {
+              const float x = sv[8 * u + q];
               const float p = (x == -INFINITY) ? 0.f : exp2f(x - m_use);
               sum += p;
-              pk.e[e] = __float2bfloat16_rn(p);
+              pk.e[q] = __float2bfloat16_rn(p);
             }
             *reinterpret_cast<uint4*>(prow + sw128(hrow, u)) = pk.u;
           }
@@ -324,12 +340,12 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[st]);
+        if (lane == 0) mbar_arrive(&p_full[sb]);
       }
       if (!ok) { *abort_flag = 1; break; }
       // epilogue: O / l for this warp's 16 heads
       const uint32_t glast = g + ntiles - 1;
-      if (!warp_wait(&t_done[glast & 1], (glast >> 1) & 1)) { *abort_flag = 1; break; }
+      if (!warp_wait(&t_done[glast % kStages], (glast / kStages) & 1)) { *abort_flag = 1; break; }
       tc_fence_after();
       float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       inv = __shfl_sync(0xffffffffu, inv, lane & 15);
@@ -341,7 +357,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
         for (int qd = 0; qd < 4; ++qd) {
           Vec16<__nv_bfloat16> pk;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) pk.e[e] = __float2bfloat16_rn(v[8 * qd + e] * inv);
+          for (int q = 0; q < 8; ++q) pk.e[q] = __float2bfloat16_rn(v[8 * qd + q] * inv);
           reinterpret_cast<uint4*>(orow + ch * 32)[qd] = pk.u;
         }
       }
@@ -353,7 +369,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1) mqa_tc_kernel(MqaTcArgs a) {
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
