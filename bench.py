@@ -239,7 +239,7 @@ class DecodeRunner:
         self.pos = torch.full((self.B,), w.decode_pos, dtype=torch.int32, device=dev)
         self.clen = torch.full((self.B,), w.decode_pos // d.m, dtype=torch.int32, device=dev)
         self.O = torch.empty(self.B, d.nh * d.c, dtype=dt, device=dev)
-        self.ws = torch.empty(csa.csa_decode_workspace_bytes(d, self.B), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(csa.csa_decode_workspace_bytes(d, self.B, self.cap), dtype=torch.uint8, device=dev)
 
     def step(self):
         csa.csa_decode(self.dims, self.packed, self.h, self.pos, self.ring, self.Cc, self.Kc, self.clen,

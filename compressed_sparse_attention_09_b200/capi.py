@@ -88,7 +88,7 @@ def lib() -> ctypes.CDLL:
             "csa_forward": (i, [D, vp, vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp]),
             "csa_ring_row_elems": (i, [D]),
             "csa_cache_append": (i, [D, vp, vp, vp, vp, vp, vp, vp, i, i, vp]),
-            "csa_decode_workspace_bytes": (sz, [D, i]),
+            "csa_decode_workspace_bytes": (sz, [D, i, i]),
             "csa_decode": (i, [D, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, sz, vp]),
             "csa_get_device_status": (i, [vp]),
             "csa_status_string": (ctypes.c_char_p, [i]),
@@ -204,8 +204,8 @@ def csa_cache_append(dims: Dims, packed, rows, pos, ring, Ccache, KIcache, cache
                                   _p(KIcache), _p(cache_len), cap, B, _stream(stream)), "csa_cache_append")
 
 
-def csa_decode_workspace_bytes(dims: Dims, B: int) -> int:
-    return lib().csa_decode_workspace_bytes(_d(dims), B)
+def csa_decode_workspace_bytes(dims: Dims, B: int, cap: int) -> int:
+    return lib().csa_decode_workspace_bytes(_d(dims), B, cap)
 
 
 def csa_decode(dims: Dims, packed, h, pos, ring, Ccache, KIcache, cache_len, cap, B, O, idx_out=None,

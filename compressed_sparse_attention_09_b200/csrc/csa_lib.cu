@@ -115,7 +115,7 @@ FwdLayout fwd_layout(const csa_dims* d, int T) {
   L.ccomp = off; off = align_up(off + nbmax * d->c * es);
   L.kicomp = off; off = align_up(off + nbmax * d->cI * es);
   L.idx = off; off = align_up(off + (size_t)T * d->topk * 4);
-  L.scratch = off; off = align_up(off + (size_t)sm_count() * 4 * (size_t)(T / d->m + 1) * 4);
+  L.scratch = off; off = align_up(off + (size_t)sm_count() * 2 * 4 * (size_t)(T / d->m + 1) * 4);
   L.total = off;
   return L;
 }
@@ -267,9 +267,9 @@ bool indexer_tc_ok(const csa_dims* d) {
   return d->dtype == CSA_BF16 && d->m == 4 && (d->nhI == 32 || d->nhI == 64) && (d->cI == 64 || d->cI == 128);
 }
 
-// Scratch of the tensor-core indexer: one row of candidate scores per query
-// of the item, per CTA.
-size_t indexer_scratch_bytes(int sc_cap) { return (size_t)sm_count() * 4 * (size_t)sc_cap * 4; }
+// Scratch of the tensor-core indexer: two buffers of one row of candidate
+// scores per query of an item, per CTA.
+size_t indexer_scratch_bytes(int sc_cap) { return (size_t)sm_count() * 2 * 4 * (size_t)sc_cap * 4; }
 
 csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int NB, void* ws, size_t ws_bytes,
                              cudaStream_t st) {
@@ -586,12 +586,12 @@ csa_status csa_sparse_mqa(const csa_dims* d, const void* q, int ld_q, const void
 
 // ---------------------------------------------------------------- indexer without a caller workspace
 // Scratch of csa_indexer_topk_noalloc: the tensor-core indexer's per-CTA
-// score rows (4 rows of up to kNoAllocMaxBlocks scores for each of up to
-// kNoAllocMaxCtas CTAs), held in module memory for the life of the process
-// on every GPU that loads the library (10 MiB).
+// score rows (2 buffers x 4 rows of up to kNoAllocMaxBlocks scores for each
+// of up to kNoAllocMaxCtas CTAs), held in module memory for the life of the
+// process on every GPU that loads the library (20 MiB).
 constexpr int kNoAllocMaxCtas = 160;
 constexpr int kNoAllocMaxBlocks = 4096;
-static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxCtas * 4 * kNoAllocMaxBlocks];
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxCtas * 2 * 4 * kNoAllocMaxBlocks];
 
 namespace {
 // Device address of g_noalloc_scratch on the current device.  The host-side
@@ -750,9 +750,9 @@ csa_status launch_append(const csa_dims* d, const void* packed, const void* rows
 }
 
 struct DecLayout {
-  size_t y1, wI, y2, idx, total;
+  size_t y1, wI, y2, idx, scratch, total;
 };
-DecLayout dec_layout(const csa_dims* d, int B) {
+DecLayout dec_layout(const csa_dims* d, int B, int cap) {
   const PackLayout P = pack_layout(d);
   const size_t es = elem_size(d);
   DecLayout L;
@@ -761,8 +761,37 @@ DecLayout dec_layout(const csa_dims* d, int B) {
   L.wI = off; off = align_up(off + (size_t)B * d->nhI * 4);
   L.y2 = off; off = align_up(off + (size_t)B * P.N2 * es);
   L.idx = off; off = align_up(off + (size_t)B * d->topk * 4);
+  L.scratch = off; off = align_up(off + (size_t)B * (size_t)cap * 4);
   L.total = off;
   return L;
+}
+
+// Decode rows through the tensor-core indexer: split-s scores into the
+// workspace, then one selection CTA per sequence.
+csa_status launch_indexer_decode_tc(const csa_dims* d, const IndexerArgs& a, int B, int cap, float* scratch,
+                                    cudaStream_t st) {
+  CUtensorMap tk, tq;
+  if (!make_tmap_bf16(&tk, a.KI, d->cI, (uint64_t)B * cap, (uint64_t)d->cI * 2, 64, idxdec::kM) ||
+      !make_tmap_bf16_3d(&tq, a.qI, d->cI, d->nhI, B, (uint64_t)d->cI * 2, (uint64_t)a.ld_qI * 2, 64, d->nhI, 1))
+    return CSA_ERR_UNSUPPORTED;
+  IdxDecArgs t;
+  t.wI = a.wI; t.ld_wI = a.ld_wI; t.pos = a.rm.pos; t.scratch = scratch; t.B = B; t.cap = cap; t.m = d->m;
+  t.nhI = d->nhI; t.cI = d->cI; t.tiles_per_seq = (cap + idxdec::kM - 1) / idxdec::kM;
+  if (cudaFuncSetAttribute(indexer_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)idxdec::kSmem) != cudaSuccess)
+    return CSA_ERR_CUDA;
+  const long long items = (long long)B * t.tiles_per_seq;
+  const int grid = items < sm_count() ? (int)items : sm_count();
+  indexer_decode_tc_kernel<<<grid, idxdec::kThreads, idxdec::kSmem, st>>>(tk, tq, t);
+  CSA_CHECK_LAUNCH();
+  const size_t smem = (size_t)cap * 4 + 256 * 4 + 40 * 4;
+  if (smem > kMaxSmem) return CSA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return CSA_ERR_CUDA;
+  decode_select_kernel<<<B, 512, smem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
 }
 }  // namespace
 
@@ -777,9 +806,9 @@ csa_status csa_cache_append(const csa_dims* d, const void* packed, const void* r
                        (cudaStream_t)stream);
 }
 
-size_t csa_decode_workspace_bytes(const csa_dims* d, int B) {
-  if (check_dims(d) != CSA_OK || B < 0) return 0;
-  return dec_layout(d, B).total;
+size_t csa_decode_workspace_bytes(const csa_dims* d, int B, int cap) {
+  if (check_dims(d) != CSA_OK || B < 0 || cap <= 0) return 0;
+  return dec_layout(d, B, cap).total;
 }
 
 csa_status csa_decode(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
@@ -791,7 +820,7 @@ csa_status csa_decode(const csa_dims* d, const void* packed, const void* h, cons
   if (cap <= 0 || B < 0) return CSA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(ws) % kPtrAlign || reinterpret_cast<uintptr_t>(packed) % kPtrAlign)
     return CSA_ERR_INVALID_ARG;
-  const DecLayout L = dec_layout(d, B);
+  const DecLayout L = dec_layout(d, B, cap);
   if (ws_bytes < L.total) return CSA_ERR_WORKSPACE;
   if (B == 0) return CSA_OK;
   const PackLayout P = pack_layout(d);
@@ -812,7 +841,11 @@ csa_status csa_decode(const csa_dims* d, const void* packed, const void* h, cons
   ia.qI = y2; ia.ld_qI = P.N2; ia.wI = wI; ia.ld_wI = d->nhI; ia.KI = KIcache; ia.idx = idx;
   ia.topk = d->topk; ia.nhI = d->nhI; ia.sc_cap = cap;
   ia.rm = RowMap{nullptr, nullptr, 0, 0, pos, cap, d->m};
-  s = launch_indexer(d, ia, B, st);
+  if (d->dtype == CSA_BF16 && (d->nhI == 32 || d->nhI == 64) && (d->cI == 64 || d->cI == 128) &&
+      reinterpret_cast<uintptr_t>(KIcache) % 16 == 0)
+    s = launch_indexer_decode_tc(d, ia, B, cap, reinterpret_cast<float*>(at(ws, L.scratch)), st);
+  else
+    s = launch_indexer(d, ia, B, st);
   if (s != CSA_OK) return s;
   MqaArgs ma;
   ma.q = y2 + (size_t)d->nhI * cI * es; ma.ld_q = P.N2; ma.C = Ccache; ma.idx = idx;

@@ -9,26 +9,30 @@
 // one block s per thread) fold it straight into the index score
 //     I[t_q, s] = sum_h w_{t_q, h} ReLU(D[s, (q, h)])
 // so the per-head products never leave the SM.  The four score rows of the
-// item go to a per-CTA scratch row (read back through L2 only; the n x n/m
-// score matrix never exists), then each epilogue warp selects the exact
-// top-k of one query with a warp-level radix select and writes its indices
-// in ascending order (ties to the lower block).  Sequence tails (L mod 4
-// tokens) are extra items with fewer than 4 queries; items whose queries see
-// at most k blocks keep them all without any MMA.
+// item go to one of two per-CTA scratch buffers (written and read back
+// through L2 only; the n x n/m score matrix never exists), and four
+// selection warps each pick the exact top-k of one query with a warp-level
+// radix select, writing its indices in ascending order (ties to the lower
+// block), while the epilogue warps already fill the other buffer with the
+// next item's scores.  Sequence tails (L mod 4 tokens) are extra items with
+// fewer than 4 queries; items whose queries see at most k blocks keep them
+// all without any MMA.
 //
-// Warp roles (192 threads): warp 0 TMA producer (q^I of the item once, then
+// Warp roles (320 threads): warp 0 TMA producer (q^I of the item once, then
 // the K^IComp tiles through a kStages ring), warp 1 MMA issuer + TMEM owner,
-// warps 2-5 epilogue + selection.  All waits are bounded.
+// warps 2-5 epilogue (TMEM -> scores), warps 6-9 selection.  All waits are
+// bounded.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
+#include "topk.cuh"
 
 namespace csa {
 
 struct IdxTcArgs {
   const float* wI; long long ld_wI;   // [T, nhI]
   int* idx;                           // [T, topk]
-  float* scratch;                     // [gridDim, 4, sc_cap]
+  float* scratch;                     // [gridDim, 2 buffers, 4, sc_cap]
   int sc_cap;                         // >= max blocks of any sequence
   int topk, nhI, cI;
   const int* cu_seqlens; const int* cu_blocks;
@@ -46,7 +50,7 @@ constexpr int kOffW = kOffK + kStages * 2 * kKChunk;   // 4 warps x [4 x 64] flo
 constexpr int kOffH = kOffW + 4 * 256 * 4;             // 4 warps x 256 bins
 constexpr int kOffB = kOffH + 4 * 256 * 4;
 constexpr size_t kSmem = 1024 + kOffB + 256;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 }  // namespace idxtc
 
 // Item `it` of the work list: compression blocks from the last one down, then
@@ -156,9 +160,9 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
   uint64_t* k_empty = k_full + kStages;        // [kStages]
   uint64_t* t_full = k_empty + kStages;        // [2]
   uint64_t* t_empty = t_full + 2;              // [2]
-  uint64_t* sc_done = t_empty + 2;             // scores of the item written (4 warps)
-  uint64_t* sel_done = sc_done + 1;            // selection of the item done (4 warps)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sel_done + 1);
+  uint64_t* sc_full = t_empty + 2;             // [2] score buffer written (4 epilogue warps)
+  uint64_t* sc_free = sc_full + 2;             // [2] score buffer selected from (4 selection warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sc_free + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -178,8 +182,10 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
       mbar_init(&t_full[s], 1);
       mbar_init(&t_empty[s], 4);
     }
-    mbar_init(sc_done, 4);
-    mbar_init(sel_done, 4);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sc_full[s], 4);
+      mbar_init(&sc_free[s], 4);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
@@ -248,36 +254,28 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
         mma_commit(q_empty);
       }
     }
-  } else {
-    // ------------------------------------------------------------ epilogue + selection (warps 2-5)
-    const int sub = warp & 3;            // TMEM lane quarter; also the query this warp selects for
-    const int ew = warp - 2;             // epilogue warp index: private smem slices
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue (warps 2-5): TMEM -> scores
+    const int sub = warp & 3;            // TMEM lane quarter
+    const int ew = warp - 2;             // private smem slice for the head weights
     float* w_my = w_s + ew * 256;
-    int* hist = h_s + ew * 256;
-    float* scr = a.scratch + (size_t)blockIdx.x * 4 * a.sc_cap;
     const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
     uint32_t acc_it = 0, wi = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x) {
       if (warp_aborted(abort_flag)) break;
       int tok0, nq, avail;
       long long kbase;
-      if (!idx_item(a, it, tok0, nq, avail, kbase)) continue;
-      if (avail <= a.topk) {   // every visible block is kept
-        if (sub < nq) {
-          int* out = a.idx + (long long)(tok0 + sub) * a.topk;
-          for (int j = lane; j < a.topk; j += 32) out[j] = j < avail ? j : -1;
-        }
-        continue;
-      }
+      if (!idx_item(a, it, tok0, nq, avail, kbase) || avail <= a.topk) continue;
       const int ntiles = (avail + kM - 1) / kM;
-      // this item's head weights, one private copy per warp
+      const int buf = wi & 1;
+      float* scr = a.scratch + ((size_t)blockIdx.x * 2 + buf) * 4 * a.sc_cap;
       for (int e = lane; e < 4 * a.nhI; e += 32) {
         const int q = e / a.nhI, h = e - q * a.nhI;
         w_my[q * 64 + h] = q < nq ? a.wI[(long long)(tok0 + q) * a.ld_wI + h] : 0.f;
       }
       __syncwarp();
-      // the previous item's selection must be over before its scratch rows are overwritten
-      if (wi > 0 && !warp_wait(sel_done, (wi - 1) & 1)) { *abort_flag = 1; break; }
+      // the selection of the item that used this buffer before must be over
+      if (!warp_wait(&sc_free[buf], ((wi >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
       bool ok = true;
       for (int j = 0; j < ntiles; ++j, ++acc_it) {
         const int acc = acc_it & 1;
@@ -307,13 +305,33 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
       }
       if (!ok) { *abort_flag = 1; break; }
       __syncwarp();
-      if (lane == 0) mbar_arrive(sc_done);
-      if (!warp_wait(sc_done, wi & 1)) { *abort_flag = 1; break; }
-      if (sub < nq)
-        warp_topk_ascending(scr + (size_t)sub * a.sc_cap, avail, a.topk, a.idx + (long long)(tok0 + sub) * a.topk,
-                            hist);
+      if (lane == 0) mbar_arrive(&sc_full[buf]);
+      ++wi;
+    }
+  } else {
+    // ------------------------------------------------------------ selection (warps 6-9): one query each
+    const int q = warp - 6;
+    int* hist = h_s + q * 256;
+    uint32_t wi = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+      if (warp_aborted(abort_flag)) break;
+      int tok0, nq, avail;
+      long long kbase;
+      if (!idx_item(a, it, tok0, nq, avail, kbase)) continue;
+      if (avail <= a.topk) {   // every visible block is kept
+        if (q < nq) {
+          int* out = a.idx + (long long)(tok0 + q) * a.topk;
+          for (int j = lane; j < a.topk; j += 32) out[j] = j < avail ? j : -1;
+        }
+        continue;
+      }
+      const int buf = wi & 1;
+      const float* scr = a.scratch + ((size_t)blockIdx.x * 2 + buf) * 4 * a.sc_cap;
+      if (!warp_wait(&sc_full[buf], (wi >> 1) & 1)) { *abort_flag = 1; break; }
+      if (q < nq)
+        warp_topk_ascending(scr + (size_t)q * a.sc_cap, avail, a.topk, a.idx + (long long)(tok0 + q) * a.topk, hist);
       __syncwarp();
-      if (lane == 0) mbar_arrive(sel_done);
+      if (lane == 0) mbar_arrive(&sc_free[buf]);
       ++wi;
     }
   }
@@ -323,6 +341,184 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
   }
+}
+
+}  // namespace csa
+
+namespace csa {
+
+// ---------------------------------------------------------------- decode form
+// One new query per sequence over that sequence's cached K^IComp: the score
+// row I[b, s] = sum_h w_{b,h} ReLU(q^I_{b,h} . K^IComp_{b,s}) is split over
+// all SMs in 128-block tiles (work item = (sequence, tile)), each tile one
+// tcgen05.mma group D[128 blocks x n_h^I] with the ReLU / head weighting in
+// the epilogue; the row goes to a [B, cap] scratch and decode_select_kernel
+// then picks its exact top-k.  The cache streams from HBM once.
+struct IdxDecArgs {
+  const float* wI; long long ld_wI;   // [B, nhI]
+  const int* pos;                     // [B]
+  float* scratch;                     // [B, cap]
+  int B, cap, m, nhI, cI, tiles_per_seq;
+};
+
+namespace idxdec {
+constexpr int kM = 128, kStages = 4;
+constexpr int kQBytes = 64 * 128 * 2;    // up to [64 heads x 128] bf16 as two 64-column chunks
+constexpr int kKBytes = kM * 128 * 2;    // [128 blocks x 128] bf16 as two chunks
+constexpr int kStageBytes = kQBytes + kKBytes;
+constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 4 * 64 * 4 + 256;
+constexpr int kThreads = 192;
+}  // namespace idxdec
+
+__global__ void __launch_bounds__(idxdec::kThreads, 1)
+    indexer_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                             IdxDecArgs a) {
+  using namespace sm100;
+  using namespace idxdec;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* w_s = reinterpret_cast<float*>(sm + kStages * kStageBytes);     // 4 warps x 64
+  uint64_t* bars = reinterpret_cast<uint64_t*>(w_s + 4 * 64);
+  uint64_t* full = bars;                   // [kStages]
+  uint64_t* empty = full + kStages;        // [kStages]
+  uint64_t* t_full = empty + kStages;      // [2]
+  uint64_t* t_empty = t_full + 2;          // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.nhI;
+  const int kchunks = a.cI / 64;
+  const int items = a.B * a.tiles_per_seq;
+  const int qchunk = N * 128, kchunk = kM * 128;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&t_full[s], 1); mbar_init(&t_empty[s], 4); }
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmQ);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // items of this CTA: a contiguous range, so consecutive items share a sequence
+  const int per = (items + gridDim.x - 1) / gridDim.x;
+  const int it0 = blockIdx.x * per, it1 = min(items, it0 + per);
+  auto item_ok = [&](int it, int& b, int& j, int& avail) {
+    b = it / a.tiles_per_seq;
+    j = it - b * a.tiles_per_seq;
+    const int t = a.pos[b];
+    avail = t >= 0 ? t / a.m : 0;
+    if (avail > a.cap) avail = a.cap;
+    return j * kM < avail;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t g = 0;
+      for (int it = it0; it < it1 && !*abort_flag; ++it) {
+        int b, j, avail;
+        if (!item_ok(it, b, j, avail)) continue;
+        const int st = g % kStages;
+        if (!mbar_wait(&empty[st], ((g / kStages) & 1) ^ 1)) { *abort_flag = 1; break; }
+        uint8_t* stage = sm + st * kStageBytes;
+        mbar_arrive_expect_tx(&full[st], (uint32_t)(kchunks * (qchunk + kchunk)));
+        for (int c = 0; c < kchunks; ++c) {
+          tma_load_3d(&tmQ, &full[st], stage + c * qchunk, 64 * c, 0, b);
+          tma_load_2d(&tmK, &full[st], stage + kQBytes + c * kchunk, 64 * c, b * a.cap + j * kM);
+        }
+        ++g;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kM, N);
+      uint32_t g = 0;
+      for (int it = it0; it < it1 && !*abort_flag; ++it) {
+        int b, j, avail;
+        if (!item_ok(it, b, j, avail)) continue;
+        const int st = g % kStages, acc = g & 1;
+        if (!mbar_wait(&full[st], (g / kStages) & 1) || !mbar_wait(&t_empty[acc], ((g >> 1) & 1) ^ 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sm + st * kStageBytes), ka = qa + kQBytes;
+        for (int c = 0; c < kchunks; ++c)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(tmem + (uint32_t)(acc * 64), sdesc_k_sw128(ka + c * kchunk + ks * 32),
+                     sdesc_k_sw128(qa + c * qchunk + ks * 32), idesc, (c | ks) != 0);
+        mma_commit(&empty[st]);
+        mma_commit(&t_full[acc]);
+        ++g;
+      }
+    }
+  } else {
+    const int sub = warp & 3;
+    float* w_my = w_s + (warp - 2) * 64;
+    const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
+    uint32_t g = 0;
+    int wb = -1;
+    for (int it = it0; it < it1; ++it) {
+      if (warp_aborted(abort_flag)) break;
+      int b, j, avail;
+      if (!item_ok(it, b, j, avail)) continue;
+      if (b != wb) {
+        for (int h = lane; h < N; h += 32) w_my[h] = a.wI[(long long)b * a.ld_wI + h];
+        __syncwarp();
+        wb = b;
+      }
+      const int acc = g & 1;
+      if (!warp_wait(&t_full[acc], (g >> 1) & 1)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      float sc = 0.f;
+      for (int hc = 0; hc < N; hc += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem + lane_base + (uint32_t)(acc * 64 + hc), v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sc = fmaf(w_my[hc + e], fmaxf(v[e], 0.f), sc);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&t_empty[acc]);
+      const int s = j * kM + 32 * sub + lane;
+      if (s < avail) __stcg(a.scratch + (long long)b * a.cap + s, sc);
+      ++g;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// Exact top-k of each decode row's score row (one CTA per sequence; the row
+// is staged in shared memory).
+__global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch, const int* pos, int cap, int m,
+                                                            int topk, int* idx) {
+  extern __shared__ __align__(16) float sc_s[];   // [cap] then hist[256], ws[40]
+  unsigned* hist = reinterpret_cast<unsigned*>(sc_s + cap);
+  int* ws = reinterpret_cast<int*>(hist + 256);
+  const int b = blockIdx.x;
+  const int t = pos[b];
+  int avail = t >= 0 ? t / m : 0;
+  if (avail > cap) avail = cap;
+  int* out = idx + (long long)b * topk;
+  if (avail <= topk) {
+    for (int j = threadIdx.x; j < topk; j += blockDim.x) out[j] = j < avail ? j : -1;
+    return;
+  }
+  const float* row = scratch + (long long)b * cap;
+  for (int s = threadIdx.x; s < avail; s += blockDim.x) sc_s[s] = __ldcg(row + s);
+  __syncthreads();
+  cta_topk_ascending(sc_s, avail, topk, out, hist, ws);
 }
 
 }  // namespace csa

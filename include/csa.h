@@ -176,7 +176,7 @@ size_t csa_indexer_workspace_bytes(const csa_dims* dims, int total_tokens, int n
  * another framework's pool, or a latency-critical loop that must not
  * allocate after start-up) cannot provide the indexer's workspace.  This
  * entry point takes the same arguments minus the workspace and instead uses
- * a fixed scratch array that lives in the library's module memory (10 MiB on
+ * a fixed scratch array that lives in the library's module memory (20 MiB on
  * every GPU that loads the library, held until the process exits).
  * Limits: the tensor-core indexer's shapes only (bf16, m = 4, nhI in {32, 64},
  * cI in {64, 128}, qI and KI 16-byte aligned, ld_qI a multiple of 8) and
@@ -252,8 +252,9 @@ csa_status csa_cache_append(const csa_dims* dims, const void* packed, const void
                             const int* pos, void* ring, void* Ccache, void* KIcache,
                             int* cache_len, int cap, int B, void* stream);
 
-/* Workspace bytes csa_decode needs for B sequences. */
-size_t csa_decode_workspace_bytes(const csa_dims* dims, int B);
+/* Workspace bytes csa_decode needs for B sequences with caches of capacity
+ * cap entries. */
+size_t csa_decode_workspace_bytes(const csa_dims* dims, int B, int cap);
 
 /* One decode step: each of B independent sequences gets one new token h_b
  * at position pos[b] and attends over its cached entries s < floor(t/m).

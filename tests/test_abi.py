@@ -42,7 +42,7 @@ def test_sizes_and_strings():
     assert csa.csa_packed_weights_bytes(TINY) > 0
     assert csa.csa_forward_workspace_bytes(TINY, 256, 1) > 0
     assert csa.csa_ring_row_elems(TINY) == 4 * 64 + 4 * 32
-    assert csa.csa_decode_workspace_bytes(TINY, 3) > 0
+    assert csa.csa_decode_workspace_bytes(TINY, 3, 40) > 0
     assert csa.status_string(0) == "ok"
     bad = csa.Dims(d=256, c=63, m=4, cI=32, nhI=4, nh=8, dc=128, topk=16, dtype=csa.CSA_F32)
     assert csa.csa_packed_weights_bytes(bad) == 0

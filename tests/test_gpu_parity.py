@@ -271,7 +271,7 @@ def decode_case(dims, B, pos0, cap, steps, seed, check):
     o_Cc, o_Kc, o_ring = f64(Cc[check]), f64(Kc[check]), f64(ring[check])
     o_clen = clen[check].numpy().astype(np.int64)
     W64 = weights_f64(W)
-    ws = torch.empty(csa.csa_decode_workspace_bytes(dims, B), dtype=torch.uint8, device=DEV)
+    ws = torch.empty(csa.csa_decode_workspace_bytes(dims, B, cap), dtype=torch.uint8, device=DEV)
     for step in range(steps):
         h = synth.make_normal((B, dims.d), dims, seed + 100 + step)
         O = torch.empty(B, dims.nh * c, dtype=h.dtype, device=DEV)
@@ -345,3 +345,11 @@ def test_stage_sparse_mqa_tensor_core_bad_index():
 
     assert _mqa_case(dims, [400], 57, bad) == 5
     assert csa.csa_get_device_status() == 0
+
+
+@pytest.mark.parametrize("m", [4, 2])
+def test_decode_tensor_core_indexer(m):
+    """Decode rows through the split-s tcgen05 indexer (n_h^I = 64, c^I = 128)
+    and the per-sequence selection, across cache appends."""
+    dims = csa.Dims(d=256, c=128, m=m, cI=128, nhI=64, nh=4, dc=128, topk=16, dtype=csa.CSA_BF16)
+    decode_case(dims, B=5, pos0=301, cap=400, steps=6, seed=63 + m, check=[0, 3, 4])
