@@ -3,35 +3,28 @@
 //
 // Work item = one query row and a group of 64 of its heads (decode rows with
 // n_h = 128 make two items).  For each item the CTA gathers the selected
-// entries 128 at a time and, per tile,
-//     S  = q . C_tile^T          tcgen05.mma M=64 (heads) N=128 (entries) K=512
+// entries 32 at a time and, per tile,
+//     S  = q . C_tile^T          tcgen05.mma M=64 (heads) N=32 (entries) K=512
 //     P  = exp2(S * log2e/sqrt(c) - m)     online softmax, one head per thread
-//     O += P . C_tile            tcgen05.mma M=64 (heads) N=256 (x2)  K=128
-// Every instruction is at least M64 x N128: on sm_100a a tcgen05.mma costs
-// at least ~54 cycles to issue, so smaller shapes (N = 32, 64) would leave
-// the tensor core idle between instructions.  The gathered tile sits in
-// shared memory once, in the 128-byte-swizzled layout, as 8 channel chunks
-// of [128 entries x 64 channels]; the S product reads it as a K-major
-// operand (rows = entries) and the O product reads the very same bytes as an
-// MN-major operand (rows = entries = K, channels contiguous): every entry is
-// loaded once and serves as key and value.  A 128-entry tile is 128 KB, so
-// there is one tile buffer whose chunks are released one by one: the next
-// tile's gather of channels 0-255 starts as soon as the O product has
-// consumed them, while it still runs on channels 256-511.
-// With M = 64 the accumulator occupies half of each TMEM lane quarter, so the
-// 64 x 512 fp32 O lives in 256 columns (channels 0-255 in the lower 16 lanes
-// of every quarter, 256-511 in the upper 16) next to a 128-column S.  Each
-// softmax thread owns one head row of S: max, sum and the P row need no
-// cross-thread reduction.  O is rescaled (TMEM load, multiply, store) only
-// when a head's running maximum grows by more than 8 in log2 units;
-// otherwise the stale maximum is kept, which is exact because O and the
-// normaliser l share it.
+//     O += P . C_tile            tcgen05.mma M=64 (heads) N=256 (x2)  K=32
+// The gathered tile sits in shared memory once, in the 128-byte-swizzled
+// layout; the S product reads it as a K-major operand (rows = entries) and
+// the O product reads the very same bytes as an MN-major operand (rows =
+// entries = K, channels contiguous): every entry is loaded once and serves as
+// key and value.  With M = 64 the accumulator occupies half of each TMEM lane
+// quarter, so the 64 x 512 fp32 O lives in 256 columns (channels 0-255 in the
+// lower 16 lanes of every quarter, 256-511 in the upper 16) next to two
+// 32-column S buffers.  Each softmax thread owns one head row of S: max, sum
+// and the P row need no cross-thread reduction.  O is rescaled (TMEM load,
+// multiply, store) only when a head's running maximum grows by more than 8 in
+// log2 units; otherwise the stale maximum is kept, which is exact because O
+// and the normaliser l share it.
 //
-// Warp roles (224 threads): warps 0-1 gather the entry chunks with 16-byte
-// cp.async (completion is tracked by the chunk's mbarrier, so the gathers
-// never block); thread 0 also loads q with a 3-D TMA; warp 2 issues the MMAs
-// (one thread) and owns TMEM; warps 3-6 run the softmax and the output
-// epilogue.  All waits are bounded (sm100::mbar_wait).
+// Warp roles (224 threads): warps 0-1 gather the entry tiles with 16-byte
+// cp.async into a 4-deep ring (completion is tracked by the stage's mbarrier,
+// so the gathers never block); thread 0 also loads q with a 3-D TMA; warp 2
+// issues the MMAs (one thread) and owns TMEM; warps 3-6 run the softmax and
+// the output epilogue.  All waits are bounded (sm100::mbar_wait).
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -48,19 +41,18 @@ struct MqaTcArgs {
 };
 
 namespace mqa {
-constexpr int kC = 512, kHeads = 64, kTile = 128;
+constexpr int kC = 512, kHeads = 64, kTile = 32, kStages = 4;
 constexpr int kQChunk = 64 * 128;           // [64 heads x 64 bf16], 128-byte rows, swizzled
-constexpr int kCChunk = kTile * 128;        // [128 entries x 64 bf16]
-constexpr int kPChunk = 64 * 128;           // [64 heads x 64 entries]
+constexpr int kCChunk = kTile * 128;        // [32 entries x 64 bf16]
 constexpr int kQBytes = 8 * kQChunk;        // 64 x 512
-constexpr int kCBytes = 8 * kCChunk;        // one tile: 128 entries x 512
-constexpr int kPBytes = 2 * kPChunk;        // 64 heads x 128 entries
+constexpr int kCBytes = 8 * kCChunk;        // one tile: 32 entries x 512
+constexpr int kPBytes = 64 * 128;           // 64 heads x 32 entries (rows padded to 128 B), swizzled
 constexpr int kMaxTopk = 4096;
 constexpr int kProducers = 64;              // threads of warps 0-1
 constexpr int kOffQ = 0;
 constexpr int kOffC = kOffQ + kQBytes;
-constexpr int kOffP = kOffC + kCBytes;
-constexpr int kOffIdx = kOffP + kPBytes;
+constexpr int kOffP = kOffC + kStages * kCBytes;
+constexpr int kOffIdx = kOffP + 2 * kPBytes;
 constexpr int kOffMisc = kOffIdx + kMaxTopk * 4;
 constexpr int kMiscBytes = 256;
 constexpr size_t kSmem = 1024 + kOffMisc + kMiscBytes;
@@ -99,13 +91,12 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffMisc);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
-  uint64_t* c_full = bars + 2;                 // [8] channel chunk of the tile gathered
-  uint64_t* c_free = c_full + 8;               // [8] chunk consumed by the tile's MMAs
-  uint64_t* s_full = c_free + 8;
-  uint64_t* s_free = s_full + 1;
-  uint64_t* p_full = s_free + 1;
-  uint64_t* t_done = p_full + 1;               // O of the tile done (P buffer free)
-  uint64_t* o_free = t_done + 1;
+  uint64_t* c_full = bars + 2;                 // [kStages]
+  uint64_t* t_done = c_full + kStages;         // [kStages]  O of the tile done: frees its C stage
+  uint64_t* s_full = t_done + kStages;         // [2]
+  uint64_t* s_free = s_full + 2;               // [2]
+  uint64_t* p_full = s_free + 2;               // [2]
+  uint64_t* o_free = p_full + 2;
   uint64_t* i_free = o_free + 1;               // both producer warps done with an item's idx copy
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(i_free + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -117,14 +108,15 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int c = 0; c < 8; ++c) {
-      mbar_init(&c_full[c], kProducers);
-      mbar_init(&c_free[c], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&c_full[s], kProducers);
+      mbar_init(&t_done[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, 4);
-    mbar_init(p_full, 4);
-    mbar_init(t_done, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 4);
+      mbar_init(&p_full[s], 4);
+    }
     mbar_init(o_free, 4);
     mbar_init(i_free, 2);
     *abort_flag = 0;
@@ -171,19 +163,18 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
         ++qw;
       }
       bool ok = true;
-      for (int j = 0; j < ntiles && ok; ++j, ++g) {
-        for (int kc = 0; kc < 8; ++kc) {
-          if (!warp_wait(&c_free[kc], (g & 1) ^ 1)) { ok = false; break; }
-          uint8_t* dst = c_s + kc * kCChunk;
+      for (int j = 0; j < ntiles; ++j, ++g) {
+        const int st = g % kStages;
+        if (!warp_wait(&t_done[st], ((g / kStages) & 1) ^ 1)) { ok = false; break; }
+        uint8_t* cst = c_s + st * kCBytes;
 #pragma unroll 4
-          for (int i = 0; i < kTile * 8 / kProducers; ++i) {
-            const int u = tid + kProducers * i, r = u >> 3, unit = u & 7;
-            const int s = idx_s[j * kTile + r];
-            const __nv_bfloat16* src = s >= 0 ? a.C + (base + s) * kC + kc * 64 + unit * 8 : a.C;
-            cp_async16(dst + sw128(r, unit), src, s >= 0 ? 16u : 0u);
-          }
-          cp_async_arrive_noinc(&c_full[kc]);
+        for (int i = 0; i < kTile * 64 / kProducers; ++i) {
+          const int u = tid + kProducers * i, r = u >> 6, c16 = u & 63;
+          const int s = idx_s[j * kTile + r];
+          const __nv_bfloat16* src = s >= 0 ? a.C + (base + s) * kC + c16 * 8 : a.C;
+          cp_async16(cst + (c16 >> 3) * kCChunk + sw128(r, c16 & 7), src, s >= 0 ? 16u : 0u);
         }
+        cp_async_arrive_noinc(&c_full[st]);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(i_free);
@@ -194,7 +185,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
     // ------------------------------------------------------------ MMA issuer (warp 2, lane 0 issues)
     constexpr uint32_t idS = idesc_bf16_f32(64, kTile);
     constexpr uint32_t idO = idesc_bf16_f32_bmn(64, 256);
-    const uint32_t q_addr = smem_u32(q_s), c_addr = smem_u32(c_s), p_addr = smem_u32(p_s);
+    const uint32_t q_addr = smem_u32(q_s);
     uint32_t g = 0, qw = 0, oi = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++oi) {
       if (warp_aborted(abort_flag)) break;
@@ -205,45 +196,51 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       const int ntiles = mqa_ntiles(a.idx + (long long)row * a.topk, a.topk, avail);
       int ok = 1;
       if (lane == 0) {
+        auto issue_o = [&](uint32_t gj, uint32_t jj) -> bool {
+          const int st = gj % kStages, pb = gj & 1;
+          if (!mbar_wait(&p_full[pb], (gj >> 1) & 1)) return false;
+          if (jj == 0 && !mbar_wait(o_free, (oi & 1) ^ 1)) return false;   // previous item's O stored
+          tc_fence_after();
+          const uint32_t pa = smem_u32(p_s + pb * kPBytes);
+          const uint32_t ca = smem_u32(c_s + st * kCBytes);
+#pragma unroll
+          for (int ks = 0; ks < kTile / 16; ++ks) {
+            const uint64_t ad = sdesc_k_sw128(pa + ks * 32);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+              mma_bf16(tmem + ((uint32_t)(16 * hh) << 16) + kColO, ad,
+                       sdesc_mn_sw128(ca + 4 * hh * kCChunk + ks * 2048, kCChunk, 1024), idO, (jj > 0 || ks > 0));
+          }
+          mma_commit(&t_done[st]);
+          return true;
+        };
         if (ntiles == 0) {
           if (!mbar_wait(o_free, (oi & 1) ^ 1)) ok = 0;     // keep one o_free phase per item
         } else if (!mbar_wait(q_full, qw & 1)) {
           ok = 0;
         } else {
+          tc_fence_after();
           for (int j = 0; j < ntiles && ok; ++j) {
             const uint32_t gj = g + j;
-            const uint32_t ph = gj & 1;
-            // S = q . C_tile^T, chunk by chunk as the gathers land
-            if (!mbar_wait(s_free, ph ^ 1)) { ok = 0; break; }
-            for (int kc = 0; kc < 8 && ok; ++kc) {
-              if (!mbar_wait(&c_full[kc], ph)) { ok = 0; break; }
-              fence_proxy_async_smem();
-              tc_fence_after();
+            const int st = gj % kStages, sb = gj & 1;
+            if (!mbar_wait(&c_full[st], (gj / kStages) & 1) || !mbar_wait(&s_free[sb], ((gj >> 1) & 1) ^ 1)) {
+              ok = 0;
+              break;
+            }
+            fence_proxy_async_smem();
+            tc_fence_after();
+            const uint32_t ca = smem_u32(c_s + st * kCBytes);
+#pragma unroll
+            for (int kc = 0; kc < 8; ++kc)
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + kColS, sdesc_k_sw128(q_addr + kc * kQChunk + ks * 32),
-                         sdesc_k_sw128(c_addr + kc * kCChunk + ks * 32), idS, (kc | ks) != 0);
-            }
-            if (!ok) break;
-            mma_commit(s_full);
+                mma_bf16(tmem + kColS + kTile * sb, sdesc_k_sw128(q_addr + kc * kQChunk + ks * 32),
+                         sdesc_k_sw128(ca + kc * kCChunk + ks * 32), idS, (kc | ks) != 0);
+            mma_commit(&s_full[sb]);
             if (j == ntiles - 1) mma_commit(q_empty);
-            // O += P . C_tile, channels 0-255 then 256-511, releasing the chunks as they are consumed
-            if (!mbar_wait(p_full, ph)) { ok = 0; break; }
-            if (j == 0 && !mbar_wait(o_free, (oi & 1) ^ 1)) { ok = 0; break; }   // previous item's O stored
-            tc_fence_after();
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-              for (int ks = 0; ks < kTile / 16; ++ks)
-                mma_bf16(tmem + ((uint32_t)(16 * hh) << 16) + kColO,
-                         sdesc_k_sw128(p_addr + (ks >> 2) * kPChunk + (ks & 3) * 32),
-                         sdesc_mn_sw128(c_addr + 4 * hh * kCChunk + ks * 2048, kCChunk, 1024), idO,
-                         (j > 0 || ks > 0));
-#pragma unroll
-              for (int kc = 0; kc < 4; ++kc) mma_commit(&c_free[4 * hh + kc]);
-            }
-            mma_commit(t_done);
+            if (j >= 1 && !issue_o(gj - 1, j - 1)) ok = 0;
           }
+          if (ok && !issue_o(g + ntiles - 1, ntiles - 1)) ok = 0;
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -277,35 +274,32 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       float m_run = -INFINITY, l_run = 0.f;
       bool ok = true;
       for (int j = 0; j < ntiles; ++j) {
-        const uint32_t gj = g + j, ph = gj & 1;
-        // validity of this tile's 128 rows, from the index row itself
-        uint32_t vm[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const int e = j * kTile + 32 * w + lane;
-          const int sidx = e < a.topk ? ir[e] : -1;
-          vm[w] = __ballot_sync(0xffffffffu, sidx >= 0 && sidx < avail);
-        }
-        if (!warp_wait(s_full, ph)) { ok = false; break; }
+        const uint32_t gj = g + j;
+        const int sb = gj & 1;
+        // validity of this tile's 32 rows, from the index row itself
+        const int e = j * kTile + lane;
+        const int sidx = e < a.topk ? ir[e] : -1;
+        const uint32_t vmask = __ballot_sync(0xffffffffu, sidx >= 0 && sidx < avail);
+        if (!warp_wait(&s_full[sb], (gj >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         float sv[kTile];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) tmem_ld_32x32b_x32(tmem + lane_base + kColS + 32 * w, sv + 32 * w);
+        tmem_ld_32x32b_x32(tmem + lane_base + kColS + kTile * sb, sv);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
+        if (lane == 0) mbar_arrive(&s_free[sb]);
         float tmax = -INFINITY;
 #pragma unroll
         for (int q = 0; q < kTile; ++q) {
-          sv[q] = ((vm[q >> 5] >> (q & 31)) & 1u) ? sv[q] * a.scale_log2 : -INFINITY;
+          sv[q] = ((vmask >> q) & 1u) ? sv[q] * a.scale_log2 : -INFINITY;
           tmax = fmaxf(tmax, sv[q]);
         }
         const float m_new = fmaxf(m_run, tmax);
         const bool grow = half == 0 && m_new > m_run + 8.f;   // also true on the first finite tile
         const float m_use = grow ? m_new : m_run;
-        // the previous tile's O MMAs must be done: P is single-buffered, and O may need rescaling
-        if (j > 0 && !warp_wait(t_done, (gj - 1) & 1)) { ok = false; break; }
         if (__any_sync(0xffffffffu, grow && j > 0)) {
+          // rescale O: the O MMAs of the earlier tiles must have completed
+          const uint32_t gp = gj - 1;
+          if (!warp_wait(&t_done[gp % kStages], (gp / kStages) & 1)) { ok = false; break; }
           tc_fence_after();
           float alpha = grow ? exp2f(m_run - m_new) : 1.f;    // exp2(-inf) = 0 when nothing was seen
           alpha = __shfl_sync(0xffffffffu, alpha, lane & 15);
@@ -322,7 +316,13 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
           l_run *= alpha;
         }
         m_run = m_use;
+        // P rows (lanes 0-15), once the P buffer's previous reader (tile gj-2) is done
+        if (gj >= 2) {
+          const uint32_t gp = gj - 2;
+          if (!warp_wait(&t_done[gp % kStages], (gp / kStages) & 1)) { ok = false; break; }
+        }
         if (half == 0) {
+          uint8_t* prow = p_s + sb * kPBytes;
           float sum = 0.f;
 #pragma unroll
           for (int u = 0; u < kTile / 8; ++u) {
@@ -334,18 +334,18 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
               sum += p;
               pk.e[q] = __float2bfloat16_rn(p);
             }
-            *reinterpret_cast<uint4*>(p_s + (u >> 3) * kPChunk + sw128(hrow, u & 7)) = pk.u;
+            *reinterpret_cast<uint4*>(prow + sw128(hrow, u)) = pk.u;
           }
           l_run += sum;
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[sb]);
       }
       if (!ok) { *abort_flag = 1; break; }
       // epilogue: O / l for this warp's 16 heads
       const uint32_t glast = g + ntiles - 1;
-      if (!warp_wait(t_done, glast & 1)) { *abort_flag = 1; break; }
+      if (!warp_wait(&t_done[glast % kStages], (glast / kStages) & 1)) { *abort_flag = 1; break; }
       tc_fence_after();
       float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       inv = __shfl_sync(0xffffffffu, inv, lane & 15);
