@@ -4,11 +4,13 @@
 // Z^b + B^b) weighting the matching C^a / C^b rows.
 //
 // The work is a pure stream: each C/Z element is read once and each entry
-// written once, so the kernel is HBM-bound.  One thread owns one 16-byte
-// channel vector of one entry: its 4m row loads are 16-byte vector loads,
-// coalesced across the warp (neighbouring threads own neighbouring channel
-// vectors of the same rows), and the 2m-wide softmax and the weighted sum run
-// in fp32 registers.
+// written once, so the kernel is HBM-bound.  One thread owns 4 channels of
+// one entry: its 4m row loads are 4-element vector loads (8 bytes for bf16,
+// 16 for fp32), coalesced across the warp (neighbouring threads own
+// neighbouring channels of the same rows), and the 2m-wide softmax and the
+// weighted sum run in fp32 registers.  Four channels per thread keep the
+// live registers low enough for many resident warps, which is what keeps
+// enough loads in flight to stream at HBM rate.
 #pragma once
 #include "common.cuh"
 
@@ -60,8 +62,8 @@ struct CompressSeg {
 struct CompressArgs {
   CompressSeg seg[2];
   int nseg;
-  int vecs0;           // 16-byte vectors per entry row of segment 0
-  int vecs_total;      // vectors per entry over all segments
+  int vecs0;           // 4-channel groups per entry row of segment 0
+  int vecs_total;      // 4-channel groups per entry over all segments
   const int* cu_seqlens;
   const int* cu_blocks;
   int nseq;
@@ -69,10 +71,36 @@ struct CompressArgs {
   int total_blocks;
 };
 
-// grid-stride over (entry, vector) pairs of all segments
+// 4 consecutive elements as fp32 (one 8-byte or 16-byte load)
+template <typename T> __device__ __forceinline__ void load4(const T* p, float* o);
+template <> __device__ __forceinline__ void load4<float>(const float* p, float* o) {
+  const float4 v = *reinterpret_cast<const float4*>(p);
+  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+}
+template <> __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float* o) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+  const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  o[0] = fa.x; o[1] = fa.y; o[2] = fb.x; o[3] = fb.y;
+}
+template <typename T> __device__ __forceinline__ void store4(T* p, const float* v);
+template <> __device__ __forceinline__ void store4<float>(float* p, const float* v) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, const float* v) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+  uint2 u;
+  u.x = *reinterpret_cast<const uint32_t*>(&a);
+  u.y = *reinterpret_cast<const uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+// grid-stride over (entry, 4-channel group) pairs of all segments
 template <typename T, int M>
 __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
-  constexpr int V = Vec16<T>::V;
+  constexpr int V = 4;
   const long long n_items = (long long)a.total_blocks * a.vecs_total;
   for (long long it = (long long)blockIdx.x * blockDim.x + threadIdx.x; it < n_items;
        it += (long long)gridDim.x * blockDim.x) {
@@ -99,26 +127,21 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
 #pragma unroll
     for (int r = 0; r < M; ++r) {
       const long long ra = (tok + r) * sg.ld + col;
-      load_vec_f32<T>(static_cast<const T*>(sg.Za) + ra, la[r]);
-      load_vec_f32<T>(static_cast<const T*>(sg.Ca) + ra, ca[r]);
-      const float4* bia = reinterpret_cast<const float4*>(sg.Ba + (long long)r * sg.width + col);
-#pragma unroll
-      for (int q = 0; q < V / 4; ++q) {
-        float4 b4 = bia[q];
-        la[r][4 * q + 0] += b4.x; la[r][4 * q + 1] += b4.y;
-        la[r][4 * q + 2] += b4.z; la[r][4 * q + 3] += b4.w;
-      }
+      load4<T>(static_cast<const T*>(sg.Za) + ra, la[r]);
+      load4<T>(static_cast<const T*>(sg.Ca) + ra, ca[r]);
       if (has_prev) {
         const long long rb = (tok - M + r) * sg.ld + col;
-        load_vec_f32<T>(static_cast<const T*>(sg.Zb) + rb, lb[r]);
-        load_vec_f32<T>(static_cast<const T*>(sg.Cb) + rb, cb[r]);
-        const float4* bib = reinterpret_cast<const float4*>(sg.Bb + (long long)r * sg.width + col);
+        load4<T>(static_cast<const T*>(sg.Zb) + rb, lb[r]);
+        load4<T>(static_cast<const T*>(sg.Cb) + rb, cb[r]);
+      }
+    }
 #pragma unroll
-        for (int q = 0; q < V / 4; ++q) {
-          float4 b4 = bib[q];
-          lb[r][4 * q + 0] += b4.x; lb[r][4 * q + 1] += b4.y;
-          lb[r][4 * q + 2] += b4.z; lb[r][4 * q + 3] += b4.w;
-        }
+    for (int r = 0; r < M; ++r) {
+      const float4 ba = *reinterpret_cast<const float4*>(sg.Ba + (long long)r * sg.width + col);
+      la[r][0] += ba.x; la[r][1] += ba.y; la[r][2] += ba.z; la[r][3] += ba.w;
+      if (has_prev) {
+        const float4 bb = *reinterpret_cast<const float4*>(sg.Bb + (long long)r * sg.width + col);
+        lb[r][0] += bb.x; lb[r][1] += bb.y; lb[r][2] += bb.z; lb[r][3] += bb.w;
       }
     }
     float res[V];
@@ -133,7 +156,7 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
       }
       res[e] = compress_channel<M>(l_a, l_b, c_a, c_b, has_prev);
     }
-    store_vec_f32<T>(static_cast<T*>(sg.out) + (long long)g * sg.width + col, res);
+    store4<T>(static_cast<T*>(sg.out) + (long long)g * sg.width + col, res);
   }
 }
 

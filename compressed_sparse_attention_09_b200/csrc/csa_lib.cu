@@ -221,7 +221,8 @@ csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const vo
 template <typename T, int M>
 void compress_launch(const CompressArgs& a, long long items, cudaStream_t st) {
   long long blocks = (items + 255) / 256;
-  if (blocks > 148LL * 16) blocks = 148LL * 16;
+  const long long cap = (long long)sm_count() * 8;   // grid-stride beyond 8 CTAs per SM
+  if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   compress_kernel<T, M><<<(unsigned)blocks, 256, 0, st>>>(a);
 }
@@ -524,14 +525,15 @@ csa_status csa_compress(const csa_dims* d, const void* Ca, const void* Cb, const
   if (!Ca || !Cb || !Za || !Zb || !Ba || !Bb || !cu_seqlens || !cu_blocks || !out) return CSA_ERR_INVALID_ARG;
   if (nseq <= 0 || total_tokens < 0 || total_blocks < 0 || width <= 0 || ld < width) return CSA_ERR_INVALID_ARG;
   if (total_blocks > total_tokens / d->m) return CSA_ERR_INVALID_ARG;
-  const int v = 16 / (int)elem_size(d);
-  if (width % v || ld % v) return CSA_ERR_UNSUPPORTED;
-  for (const void* p : {Ca, Cb, Za, Zb, (const void*)Ba, (const void*)Bb, (const void*)out})
-    if (reinterpret_cast<uintptr_t>(p) % 16) return CSA_ERR_UNSUPPORTED;
+  if (width % 4 || ld % 4) return CSA_ERR_UNSUPPORTED;
+  const uintptr_t va = 4 * elem_size(d);   // 4-element vectors
+  for (const void* p : {Ca, Cb, Za, Zb, (const void*)out})
+    if (reinterpret_cast<uintptr_t>(p) % va) return CSA_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(Ba) % 16 || reinterpret_cast<uintptr_t>(Bb) % 16) return CSA_ERR_UNSUPPORTED;
   CompressArgs a = make_compress_args(d, cu_seqlens, cu_blocks, nseq, total_tokens, total_blocks);
   a.seg[0] = {Ca, Cb, Za, Zb, ld, Ba, Bb, width, out};
   a.nseg = 1;
-  a.vecs0 = width / v;
+  a.vecs0 = width / 4;
   a.vecs_total = a.vecs0;
   return launch_compress(d, a, (cudaStream_t)stream);
 }
@@ -685,9 +687,8 @@ csa_status csa_forward(const csa_dims* d, const void* packed, const void* H, con
                reinterpret_cast<const float*>(at((void*)packed, P.baI)),
                reinterpret_cast<const float*>(at((void*)packed, P.bbI)), cI, KIc};
   ca.nseg = 2;
-  const int v = 16 / (int)es;
-  ca.vecs0 = c / v;
-  ca.vecs_total = (c + cI) / v;
+  ca.vecs0 = c / 4;
+  ca.vecs_total = (c + cI) / 4;
   s = launch_compress(d, ca, st);
   if (s != CSA_OK) return s;
   // A4: eqs. (8), (9)
