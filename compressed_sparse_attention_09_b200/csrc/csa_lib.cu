@@ -70,6 +70,12 @@ int sm_count() {
   return cached[dev];
 }
 
+// Scratch of the tensor-core indexer: two buffers of one row of candidate
+// scores per query of an item, per CTA.  Rows are padded to a multiple of 4
+// floats so that every row starts 16-byte aligned.
+inline int padded_cap(int sc_cap) { return (sc_cap + 3) & ~3; }
+size_t indexer_scratch_bytes(int sc_cap) { return (size_t)sm_count() * 2 * 4 * (size_t)padded_cap(sc_cap) * 4; }
+
 // ------------------------------------------------------------------ layouts
 struct PackLayout {
   int N1b;    // bf16/f32 block of the H-side output: C^a C^b Z^a Z^b C^aI C^bI Z^aI Z^bI c^Q
@@ -115,7 +121,7 @@ FwdLayout fwd_layout(const csa_dims* d, int T) {
   L.ccomp = off; off = align_up(off + nbmax * d->c * es);
   L.kicomp = off; off = align_up(off + nbmax * d->cI * es);
   L.idx = off; off = align_up(off + (size_t)T * d->topk * 4);
-  L.scratch = off; off = align_up(off + (size_t)sm_count() * 2 * 4 * (size_t)(T / d->m + 1) * 4);
+  L.scratch = off; off = align_up(off + indexer_scratch_bytes(T / d->m + 1));
   L.total = off;
   return L;
 }
@@ -268,13 +274,10 @@ bool indexer_tc_ok(const csa_dims* d) {
   return d->dtype == CSA_BF16 && d->m == 4 && (d->nhI == 32 || d->nhI == 64) && (d->cI == 64 || d->cI == 128);
 }
 
-// Scratch of the tensor-core indexer: two buffers of one row of candidate
-// scores per query of an item, per CTA.
-size_t indexer_scratch_bytes(int sc_cap) { return (size_t)sm_count() * 2 * 4 * (size_t)sc_cap * 4; }
 
 csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int NB, void* ws, size_t ws_bytes,
                              cudaStream_t st) {
-  const int sc_cap = a.sc_cap > 0 ? a.sc_cap : 1;
+  const int sc_cap = padded_cap(a.sc_cap > 0 ? a.sc_cap : 1);
   if (!ws || ws_bytes < indexer_scratch_bytes(sc_cap) || reinterpret_cast<uintptr_t>(ws) % 16)
     return CSA_ERR_WORKSPACE;
   CUtensorMap tk, tq;

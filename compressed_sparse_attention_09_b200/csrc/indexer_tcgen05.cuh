@@ -41,14 +41,15 @@ struct IdxTcArgs {
 
 namespace idxtc {
 constexpr int kM = 128;                 // blocks per tile
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kQChunk = 256 * 128;      // [4 x nhI <= 256 rows x 64 bf16]
 constexpr int kKChunk = kM * 128;       // [128 rows x 64 bf16]
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + 2 * kQChunk;
 constexpr int kOffW = kOffK + kStages * 2 * kKChunk;   // 4 warps x [4 x 64] floats
 constexpr int kOffH = kOffW + 4 * 256 * 4;             // 4 warps x 256 bins
-constexpr int kOffB = kOffH + 4 * 256 * 4;
+constexpr int kOffS = kOffH + 4 * 256 * 4;             // 4 warps x kSelChunk staged scores
+constexpr int kOffB = kOffS + 4 * 2048 * 4;
 constexpr size_t kSmem = 1024 + kOffB + 256;
 constexpr int kThreads = 320;
 }  // namespace idxtc
@@ -81,20 +82,50 @@ __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, 
 }
 
 // Exact top-k of sc[0..n) (n > k) by one warp, written to out[0..k) as
-// ascending indices; equal scores are taken lowest index first.
-__device__ void warp_topk_ascending(const float* sc, int n, int k, int* out, int* hist) {
+// ascending indices; equal scores are taken lowest index first.  The row is
+// read through `buf` (kSelChunk floats of shared memory) a chunk at a time
+// with 16-byte loads, all in flight together; a row that fits in one chunk
+// is read once and every pass runs on shared memory.  Radix select on the
+// order-preserving 32-bit keys: 4 passes of 8-bit histograms find the k-th
+// largest key and how many keys equal to it are taken, then an ordered pass
+// writes the winners.
+constexpr int kSelChunk = 2048;
+
+__device__ __forceinline__ void warp_stage_chunk(const float* src, int n, float* buf) {
   const int lane = threadIdx.x & 31;
+  // n <= kSelChunk; 16-byte loads where the whole vector is in range
+  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+  if (vec) {
+    const int n4 = n >> 2;
+#pragma unroll 4
+    for (int i = lane; i < n4; i += 32) reinterpret_cast<float4*>(buf)[i] = __ldcg(reinterpret_cast<const float4*>(src) + i);
+    for (int i = (n4 << 2) + lane; i < n; i += 32) buf[i] = __ldcg(src + i);
+  } else {
+#pragma unroll 4
+    for (int i = lane; i < n; i += 32) buf[i] = __ldcg(src + i);
+  }
+  __syncwarp();
+}
+
+__device__ void warp_topk_ascending(const float* sc, int n, int k, int* out, int* hist, float* buf) {
+  const int lane = threadIdx.x & 31;
+  const bool resident = n <= kSelChunk;
+  if (resident) warp_stage_chunk(sc, n, buf);
   uint32_t prefix = 0, mask = 0;
   int kk = k;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int i = lane; i < 256; i += 32) hist[i] = 0;
     __syncwarp();
-    for (int s = lane; s < n; s += 32) {
-      const uint32_t key = ordered_key(__ldcg(sc + s));
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    for (int c0 = 0; c0 < n; c0 += kSelChunk) {
+      const int cn = min(kSelChunk, n - c0);
+      if (!resident) warp_stage_chunk(sc + c0, cn, buf);
+      for (int s = lane; s < cn; s += 32) {
+        const uint32_t key = ordered_key(buf[s]);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+      }
+      __syncwarp();
     }
-    __syncwarp();
     // lane L owns bins 255-8L .. 248-8L (descending); find the digit holding the kk-th largest
     int cnt[8], tot = 0;
 #pragma unroll
@@ -128,18 +159,23 @@ __device__ void warp_topk_ascending(const float* sc, int n, int k, int* out, int
   const int need_eq = kk;
   int out_off = 0, eq_seen = 0;
   const unsigned lt = (1u << lane) - 1u;
-  for (int base = 0; base < n; base += 32) {
-    const int s = base + lane;
-    const uint32_t key = s < n ? ordered_key(__ldcg(sc + s)) : 0u;
-    const bool gt = s < n && key > thr;
-    const bool eq = s < n && key == thr;
-    const unsigned beq = __ballot_sync(0xffffffffu, eq);
-    const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
-    const unsigned btk = __ballot_sync(0xffffffffu, take);
-    const int p = out_off + __popc(btk & lt);
-    if (take && p < k) out[p] = s;
-    out_off += __popc(btk);
-    eq_seen += __popc(beq);
+  for (int c0 = 0; c0 < n; c0 += kSelChunk) {
+    const int cn = min(kSelChunk, n - c0);
+    if (!resident) warp_stage_chunk(sc + c0, cn, buf);
+    for (int base = 0; base < cn; base += 32) {
+      const int s = base + lane;
+      const uint32_t key = s < cn ? ordered_key(buf[s]) : 0u;
+      const bool gt = s < cn && key > thr;
+      const bool eq = s < cn && key == thr;
+      const unsigned beq = __ballot_sync(0xffffffffu, eq);
+      const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
+      const unsigned btk = __ballot_sync(0xffffffffu, take);
+      const int p = out_off + __popc(btk & lt);
+      if (take && p < k) out[p] = c0 + s;
+      out_off += __popc(btk);
+      eq_seen += __popc(beq);
+    }
+    __syncwarp();
   }
 }
 
@@ -153,6 +189,7 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
   uint8_t* k_s = sm + kOffK;
   float* w_s = reinterpret_cast<float*>(sm + kOffW);
   int* h_s = reinterpret_cast<int*>(sm + kOffH);
+  float* sel_s = reinterpret_cast<float*>(sm + kOffS);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffB);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
@@ -329,7 +366,8 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
       const float* scr = a.scratch + ((size_t)blockIdx.x * 2 + buf) * 4 * a.sc_cap;
       if (!warp_wait(&sc_full[buf], (wi >> 1) & 1)) { *abort_flag = 1; break; }
       if (q < nq)
-        warp_topk_ascending(scr + (size_t)q * a.sc_cap, avail, a.topk, a.idx + (long long)(tok0 + q) * a.topk, hist);
+        warp_topk_ascending(scr + (size_t)q * a.sc_cap, avail, a.topk, a.idx + (long long)(tok0 + q) * a.topk, hist,
+                            sel_s + q * kSelChunk);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sc_free[buf]);
       ++wi;
