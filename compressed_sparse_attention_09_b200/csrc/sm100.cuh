@@ -189,6 +189,11 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const float* 
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Instruction descriptor as idesc_bf16_f32 with the A operand MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N) {
+  return idesc_bf16_f32(M, N) | (1u << 15);
+}
+
 // Instruction descriptor as idesc_bf16_f32 with the B operand MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
   return idesc_bf16_f32(M, N) | (1u << 16);
