@@ -3,10 +3,10 @@
 //
 // Work item = one query row and a group of 64 of its heads (decode rows with
 // n_h = 128 make two items).  For each item the CTA gathers the selected
-// entries 64 at a time and, per tile,
-//     S  = q . C_tile^T          tcgen05.mma M=64 (heads) N=64 (entries) K=512
+// entries 32 at a time and, per tile,
+//     S  = q . C_tile^T          tcgen05.mma M=64 (heads) N=32 (entries) K=512
 //     P  = exp2(S * log2e/sqrt(c) - m)     online softmax, one head per thread
-//     O += P . C_tile            tcgen05.mma M=64 (heads) N=256 (x2)  K=64
+//     O += P . C_tile            tcgen05.mma M=64 (heads) N=256 (x2)  K=32
 // The gathered tile sits in shared memory once, in the 128-byte-swizzled
 // layout; the S product reads it as a K-major operand (rows = entries) and
 // the O product reads the very same bytes as an MN-major operand (rows =
@@ -14,14 +14,14 @@
 // key and value.  With M = 64 the accumulator occupies half of each TMEM lane
 // quarter, so the 64 x 512 fp32 O lives in 256 columns (channels 0-255 in the
 // lower 16 lanes of every quarter, 256-511 in the upper 16) next to two
-// 64-column S buffers.  Each softmax thread owns one head row of S: max, sum
+// 32-column S buffers.  Each softmax thread owns one head row of S: max, sum
 // and the P row need no cross-thread reduction.  O is rescaled (TMEM load,
 // multiply, store) only when a head's running maximum grows by more than 8 in
 // log2 units; otherwise the stale maximum is kept, which is exact because O
 // and the normaliser l share it.
 //
 // Warp roles (224 threads): warps 0-1 gather the entry tiles with 16-byte
-// cp.async into a 2-deep ring (completion is tracked by the stage's mbarrier,
+// cp.async into a 4-deep ring (completion is tracked by the stage's mbarrier,
 // so the gathers never block); thread 0 also loads q with a 3-D TMA; warp 2
 // issues the MMAs (one thread) and owns TMEM; warps 3-6 run the softmax and
 // the output epilogue.  All waits are bounded (sm100::mbar_wait).
@@ -41,12 +41,12 @@ struct MqaTcArgs {
 };
 
 namespace mqa {
-constexpr int kC = 512, kHeads = 64, kTile = 64, kStages = 2;
+constexpr int kC = 512, kHeads = 64, kTile = 32, kStages = 4;
 constexpr int kQChunk = 64 * 128;           // [64 heads x 64 bf16], 128-byte rows, swizzled
 constexpr int kCChunk = kTile * 128;        // [32 entries x 64 bf16]
 constexpr int kQBytes = 8 * kQChunk;        // 64 x 512
 constexpr int kCBytes = 8 * kCChunk;        // one tile: 32 entries x 512
-constexpr int kPBytes = 64 * 128;           // 64 heads x 64 entries, swizzled
+constexpr int kPBytes = 64 * 128;           // 64 heads x 32 entries (rows padded to 128 B), swizzled
 constexpr int kMaxTopk = 4096;
 constexpr int kProducers = 64;              // threads of warps 0-1
 constexpr int kOffQ = 0;
@@ -276,26 +276,21 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       for (int j = 0; j < ntiles; ++j) {
         const uint32_t gj = g + j;
         const int sb = gj & 1;
-        // validity of this tile's 64 rows, from the index row itself
-        uint32_t vm[kTile / 32];
-#pragma unroll
-        for (int w = 0; w < kTile / 32; ++w) {
-          const int e = j * kTile + 32 * w + lane;
-          const int sidx = e < a.topk ? ir[e] : -1;
-          vm[w] = __ballot_sync(0xffffffffu, sidx >= 0 && sidx < avail);
-        }
+        // validity of this tile's 32 rows, from the index row itself
+        const int e = j * kTile + lane;
+        const int sidx = e < a.topk ? ir[e] : -1;
+        const uint32_t vmask = __ballot_sync(0xffffffffu, sidx >= 0 && sidx < avail);
         if (!warp_wait(&s_full[sb], (gj >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         float sv[kTile];
-#pragma unroll
-        for (int w = 0; w < kTile / 32; ++w) tmem_ld_32x32b_x32(tmem + lane_base + kColS + kTile * sb + 32 * w, sv + 32 * w);
+        tmem_ld_32x32b_x32(tmem + lane_base + kColS + kTile * sb, sv);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
         float tmax = -INFINITY;
 #pragma unroll
         for (int q = 0; q < kTile; ++q) {
-          sv[q] = ((vm[q >> 5] >> (q & 31)) & 1u) ? sv[q] * a.scale_log2 : -INFINITY;
+          sv[q] = ((vmask >> q) & 1u) ? sv[q] * a.scale_log2 : -INFINITY;
           tmax = fmaxf(tmax, sv[q]);
         }
         const float m_new = fmaxf(m_run, tmax);
