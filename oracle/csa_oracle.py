@@ -42,6 +42,7 @@ __all__ = [
     "core_attn",
     "num_blocks",
     "csa_forward",
+    "csa_forward_sampled",
     "csa_decode_step",
 ]
 
@@ -294,6 +295,74 @@ def csa_forward(H, W, dims, seqlens, store="exact", rows=None, keep_scores=False
     if keep_scores:
         out["scores"] = scores
     return out
+
+
+def csa_forward_sampled(H, W, dims, seqlens, rows, store="bf16", chunk=8192):
+    """``csa_forward`` restricted to ``rows``, for inputs too large to hold in fp64.
+
+    The same equations in the same order; only the bookkeeping differs:
+    H (any array-like of shape [T, d], e.g. a bf16 torch tensor) is widened
+    to fp64 ``chunk`` tokens at a time, and each chunk's eight H-side
+    projections (eqs. 1, 2 and the indexer copies) are stored after storage
+    rounding.  With ``store="bf16"`` they are kept in fp32, which holds every
+    bf16 value exactly; with ``"exact"`` they stay fp64.  Compression, the
+    indexer, top-k and CoreAttn then run as in ``csa_forward``.
+    Returns the same keys as ``csa_forward`` for the requested rows.
+    """
+    m, k = dims["m"], dims["topk"]
+    nh, nhI, c, cI = dims["nh"], dims["nhI"], dims["c"], dims["cI"]
+    T = sum(seqlens)
+    rnd = lambda x: storage_round(x, store)
+    rnd_w = (lambda x: round_f32(x)) if store == "bf16" else rnd
+    keep = np.float32 if store in ("bf16", "f32") else np.float64
+
+    def rows_f64(a, b):
+        x = H[a:b]
+        if hasattr(x, "double"):               # a torch tensor
+            x = x.double().numpy()
+        return np.asarray(x, dtype=np.float64)
+
+    Wcat = np.concatenate([np.asarray(W[n], dtype=np.float64) for n in _HSIDE], axis=1)
+    widths = [c, c, c, c, cI, cI, cI, cI]
+    offs = np.concatenate([[0], np.cumsum(widths)])
+    proj = np.empty((T, int(offs[-1])), dtype=keep)
+    for a in range(0, T, chunk):
+        b = min(T, a + chunk)
+        proj[a:b] = rnd(project(rows_f64(a, b), Wcat))
+    part = lambda j, sl: proj[sl, offs[j]:offs[j + 1]]
+
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int64)
+    cu_blocks = np.concatenate([[0], np.cumsum([num_blocks(L, m) for L in seqlens])]).astype(np.int64)
+    C_parts, K_parts = [], []
+    for b, L in enumerate(seqlens):
+        sl = slice(cu[b], cu[b] + L)
+        C_parts.append(compress(part(0, sl), part(1, sl), part(2, sl), part(3, sl), W["B_a"], W["B_b"], m))
+        K_parts.append(compress(part(4, sl), part(5, sl), part(6, sl), part(7, sl), W["B_a_I"], W["B_b_I"], m))
+    del proj
+    C_comp = rnd(np.concatenate(C_parts, axis=0))
+    K_icomp = rnd(np.concatenate(K_parts, axis=0))
+
+    rows = np.asarray(rows, dtype=np.int64)
+    seq_of = np.searchsorted(cu, rows, side="right") - 1
+    Hr = np.concatenate([rows_f64(int(t), int(t) + 1) for t in rows]) if len(rows) else np.zeros((0, H.shape[1]))
+    cQ = rnd(project(Hr, W["W_DQ"]))
+    wI = rnd_w(project(Hr, W["W_w"]))
+    qI = rnd(project(cQ, W["W_IUQ"])).reshape(len(rows), nhI, cI)
+    q = rnd(project(cQ, W["W_UQ"])).reshape(len(rows), nh, c)
+    idx = np.full((len(rows), k), -1, dtype=np.int64)
+    O = np.zeros((len(rows), nh, c))
+    scores = []
+    for r, (tg, b) in enumerate(zip(rows, seq_of)):
+        t = int(tg - cu[b])
+        avail = t // m
+        base = int(cu_blocks[b])
+        I_t = indexer_scores(qI[r], wI[r], K_icomp[base:base + avail])
+        sel = topk_select(I_t, k)
+        idx[r] = sel
+        O[r] = core_attn(q[r], C_comp[base + sel[sel >= 0]])
+        scores.append(I_t)
+    return {"C_comp": C_comp, "K_icomp": K_icomp, "cu_blocks": cu_blocks, "rows": rows, "idx": idx, "O": O,
+            "cQ": cQ, "wI": wI, "qI": qI, "q": q, "scores": scores}
 
 
 # --------------------------------------------------------------------------

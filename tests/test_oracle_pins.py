@@ -425,3 +425,19 @@ def test_decode_first_block_uses_i0_padding():
         O, idx = orc.csa_decode_step(H[t:t + 1], [t], C_cache, K_cache, cache_len, ring, W, dims)
         np.testing.assert_allclose(O[0], full["O"][t], atol=1e-13)
     np.testing.assert_allclose(C_cache[0, :2], full["C_comp"], atol=1e-13)
+
+
+@pytest.mark.parametrize("store", ["exact", "bf16"])
+def test_forward_sampled_equals_forward(store):
+    """The chunked, memory-light form gives the same rows as csa_forward."""
+    lens = [37, 5, 60]
+    H, W, dims = small_problem(20, lens, topk=4)
+    rows = [0, 4, 36, 40, 41, 70, 101]
+    full = orc.csa_forward(H, W, dims, lens, store=store, rows=rows, keep_scores=True)
+    samp = orc.csa_forward_sampled(H, W, dims, lens, rows, store=store, chunk=16)
+    np.testing.assert_allclose(samp["C_comp"], full["C_comp"], atol=1e-12)
+    np.testing.assert_allclose(samp["K_icomp"], full["K_icomp"], atol=1e-12)
+    np.testing.assert_array_equal(samp["idx"], full["idx"])
+    np.testing.assert_allclose(samp["O"], full["O"], atol=1e-12)
+    for a, b in zip(samp["scores"], full["scores"]):
+        np.testing.assert_allclose(a, b, atol=1e-12)
