@@ -139,11 +139,11 @@ __global__ void __launch_bounds__(192, 1)
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smA + stage * Cfg::A_BYTES);
-          const uint32_t b0 = smem_u32(smB + stage * Cfg::B_BYTES);
+          const uint64_t ad = sdesc_k_sw128(smem_u32(smA + stage * Cfg::A_BYTES));
+          const uint64_t bd = sdesc_k_sw128(smem_u32(smB + stage * Cfg::B_BYTES));
 #pragma unroll
           for (int k = 0; k < Cfg::BK / 16; ++k)
-            mma_bf16(d_tmem, sdesc_k_sw128(a0 + k * 32), sdesc_k_sw128(b0 + k * 32), idesc, (kb | k) != 0);
+            mma_bf16(d_tmem, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc, (kb | k) != 0);
           mma_commit(&empty[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }

@@ -278,12 +278,12 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t ka = smem_u32(k_s + st * 2 * kKChunk), qa = smem_u32(q_s);
+          const uint64_t kd = sdesc_k_sw128(smem_u32(k_s + st * 2 * kKChunk)), qd = sdesc_k_sw128(smem_u32(q_s));
           for (int c = 0; c < kchunks; ++c)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-              mma_bf16(tmem + (uint32_t)(acc * N), sdesc_k_sw128(ka + c * kKChunk + ks * 32),
-                       sdesc_k_sw128(qa + c * kQChunk + ks * 32), idesc, (c | ks) != 0);
+              mma_bf16(tmem + (uint32_t)(acc * N), desc_add(kd, c * kKChunk + ks * 32),
+                       desc_add(qd, c * kQChunk + ks * 32), idesc, (c | ks) != 0);
           mma_commit(&k_empty[st]);
           mma_commit(&t_full[acc]);
         }
@@ -485,12 +485,13 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t qa = smem_u32(sm + st * kStageBytes), ka = qa + kQBytes;
+        const uint32_t qa = smem_u32(sm + st * kStageBytes);
+        const uint64_t qd = sdesc_k_sw128(qa), kd = sdesc_k_sw128(qa + kQBytes);
         for (int c = 0; c < kchunks; ++c)
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(tmem + (uint32_t)(acc * 64), sdesc_k_sw128(ka + c * kchunk + ks * 32),
-                     sdesc_k_sw128(qa + c * qchunk + ks * 32), idesc, (c | ks) != 0);
+            mma_bf16(tmem + (uint32_t)(acc * 64), desc_add(kd, c * kchunk + ks * 32),
+                     desc_add(qd, c * qchunk + ks * 32), idesc, (c | ks) != 0);
         mma_commit(&empty[st]);
         mma_commit(&t_full[acc]);
         ++g;

@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
     // ------------------------------------------------------------ MMA issuer (warp 2, lane 0 issues)
     constexpr uint32_t idS = idesc_bf16_f32(64, kTile);
     constexpr uint32_t idO = idesc_bf16_f32_bmn(64, 256);
-    const uint32_t q_addr = smem_u32(q_s);
+    const uint64_t qd0 = sdesc_k_sw128(smem_u32(q_s));
     uint32_t g = 0, qw = 0, oi = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x, ++oi) {
       if (warp_aborted(abort_flag)) break;
@@ -201,15 +201,14 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
           if (!mbar_wait(&p_full[pb], (gj >> 1) & 1)) return false;
           if (jj == 0 && !mbar_wait(o_free, (oi & 1) ^ 1)) return false;   // previous item's O stored
           tc_fence_after();
-          const uint32_t pa = smem_u32(p_s + pb * kPBytes);
-          const uint32_t ca = smem_u32(c_s + st * kCBytes);
+          const uint64_t pd = sdesc_k_sw128(smem_u32(p_s + pb * kPBytes));
+          const uint64_t cd = sdesc_mn_sw128(smem_u32(c_s + st * kCBytes), kCChunk, 1024);
 #pragma unroll
           for (int ks = 0; ks < kTile / 16; ++ks) {
-            const uint64_t ad = sdesc_k_sw128(pa + ks * 32);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh)
-              mma_bf16(tmem + ((uint32_t)(16 * hh) << 16) + kColO, ad,
-                       sdesc_mn_sw128(ca + 4 * hh * kCChunk + ks * 2048, kCChunk, 1024), idO, (jj > 0 || ks > 0));
+              mma_bf16(tmem + ((uint32_t)(16 * hh) << 16) + kColO, desc_add(pd, ks * 32),
+                       desc_add(cd, 4 * hh * kCChunk + ks * 2048), idO, (jj > 0 || ks > 0));
           }
           mma_commit(&t_done[st]);
           return true;
@@ -229,13 +228,13 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
             }
             fence_proxy_async_smem();
             tc_fence_after();
-            const uint32_t ca = smem_u32(c_s + st * kCBytes);
+            const uint64_t cd = sdesc_k_sw128(smem_u32(c_s + st * kCBytes));
 #pragma unroll
             for (int kc = 0; kc < 8; ++kc)
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tmem + kColS + kTile * sb, sdesc_k_sw128(q_addr + kc * kQChunk + ks * 32),
-                         sdesc_k_sw128(ca + kc * kCChunk + ks * 32), idS, (kc | ks) != 0);
+                mma_bf16(tmem + kColS + kTile * sb, desc_add(qd0, kc * kQChunk + ks * 32),
+                         desc_add(cd, kc * kCChunk + ks * 32), idS, (kc | ks) != 0);
             mma_commit(&s_full[sb]);
             if (j == ntiles - 1) mma_commit(q_empty);
             if (j >= 1 && !issue_o(gj - 1, j - 1)) ok = 0;

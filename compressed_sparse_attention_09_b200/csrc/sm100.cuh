@@ -149,6 +149,12 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t addr) {
          | ((uint64_t)2 << 61);                 // swizzle mode: 128 B
 }
 
+// The descriptor of the same operand layout starting `byte_off` bytes later:
+// the start-address field (address / 16, 14 bits) cannot overflow because
+// shared memory addresses stay below 256 KB.  With constant offsets this is
+// one add, instead of rebuilding the descriptor before every MMA.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t byte_off) { return d + (uint64_t)(byte_off >> 4); }
+
 // 32 consecutive fp32 TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float* v) {
   uint32_t r[32];
