@@ -328,8 +328,7 @@ csa_status mqa_launch(const MqaArgs& a, int rows, cudaStream_t st) {
 csa_status launch_mqa(const csa_dims* d, const MqaArgs& a, int rows, cudaStream_t st) {
   if (rows == 0) return CSA_OK;
   const bool b = d->dtype == CSA_BF16;
-  if (b && d->c == mqa::kC && d->nh % mqa::kHeads == 0 && a.topk <= mqa::kMaxTopk && a.ld_q % 8 == 0 &&
-      a.ld_O % 8 == 0 &&
+  if (b && d->c == mqa::kC && d->nh % mqa::kHeads == 0 && a.topk >= 1 && a.ld_q % 8 == 0 && a.ld_O % 8 == 0 &&
       reinterpret_cast<uintptr_t>(a.q) % 16 == 0 && reinterpret_cast<uintptr_t>(a.O) % 16 == 0 &&
       reinterpret_cast<uintptr_t>(a.C) % 16 == 0) {
     // tensor-core path: c = 512, heads in groups of 64, q read through a 3-D tensor map

@@ -198,12 +198,16 @@ def test_stage_indexer_topk_full_size_sampled():
     assert kinds["exact"] > 0.6 * len(rows), kinds   # the rest passed the validity check
 
 
-def _mqa_case(dims, lens, seed, idx_fn):
+def _mqa_case(dims, lens, seed, idx_fn, q_std=1.0, c_row_scale=None):
     T = sum(lens)
     cu, cb = csa.cu_from_lengths(lens, dims.m)
     NB = int(cb[-1])
-    q = synth.make_normal((T, dims.nh * dims.c), dims, seed)
+    q = synth.make_normal((T, dims.nh * dims.c), dims, seed, std=q_std)
     C = synth.make_normal((max(NB, 1), dims.c), dims, seed + 1)
+    if c_row_scale is not None:   # per-entry scale (given the entry's block index s), applied before rounding
+        s_of_row = np.concatenate([np.arange(int(cb[b + 1]) - int(cb[b])) for b in range(len(lens))] or [[0]])
+        sc = torch.as_tensor(c_row_scale(s_of_row[:C.shape[0]]), dtype=torch.float32)
+        C = (C.float() * sc[:, None]).to(C.dtype)
     idx = torch.full((T, dims.topk), -1, dtype=torch.int32)
     for b, L in enumerate(lens):
         for t in range(L):
@@ -332,6 +336,25 @@ def test_stage_sparse_mqa_tensor_core(nh, topk, fn):
     a partial last tile, rows with no visible block, -1 holes."""
     dims = csa.Dims(d=64, c=512, m=4, cI=32, nhI=4, nh=nh, dc=64, topk=topk, dtype=csa.CSA_BF16)
     assert _mqa_case(dims, [300, 9, 1, 2100], 54 + topk, fn) == 0
+
+
+@pytest.mark.parametrize("fn", [_strided, _holes])
+def test_stage_sparse_mqa_tensor_core_many_blocks(fn):
+    """k = 768 over up to 825 visible entries: three full 256-entry blocks
+    and a ragged fourth, with the running maximum carried across them."""
+    dims = csa.Dims(d=64, c=512, m=4, cI=32, nhI=4, nh=64, dc=64, topk=768, dtype=csa.CSA_BF16)
+    assert _mqa_case(dims, [3300, 5], 58, fn) == 0
+
+
+def test_stage_sparse_mqa_tensor_core_rescale():
+    """Scores that grow along the row (entries s < 256 scaled by 0.025, the
+    rest by 0.5, q with std 6: scaled scores of std ~4 in log2 units after
+    near-zero ones), so the running maximum of most heads rises by far more
+    than the lazy threshold and O and l are rescaled in flight.  The entry
+    scale keeps |O| near unit size, where the absolute bar applies."""
+    dims = csa.Dims(d=64, c=512, m=4, cI=32, nhI=4, nh=64, dc=64, topk=640, dtype=csa.CSA_BF16)
+    assert _mqa_case(dims, [2600], 59, _first_k, q_std=6.0,
+                     c_row_scale=lambda s: np.where(s < 256, 0.025, 0.5)) == 0
 
 
 def test_stage_sparse_mqa_tensor_core_bad_index():
