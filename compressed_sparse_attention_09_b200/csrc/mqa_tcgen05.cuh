@@ -16,10 +16,11 @@
 // Issue rate.  One thread issuing tcgen05.mma waits ~54 cycles per
 // instruction whatever its size below N = 128, so the S product of a 32-entry
 // tile (32 instructions) would leave the tensor pipe three-quarters idle.
-// Four threads (one per issuer warp) therefore issue it together, each over a
-// quarter of the channels (K = 128) into its own partial accumulator; the
-// softmax adds the four partials.  The O product is split by channel half
-// between issuers 0 and 1.
+// Four threads (one per S-issuer warp) therefore issue it together, each over
+// a quarter of the channels (K = 128) into its own partial accumulator; the
+// softmax adds the four partials.  A fifth warp issues the O products only,
+// so the S issuers never wait for the softmax: they run up to four tiles
+// ahead, one S buffer each.
 //
 // Gather rate.  The tiles are gathered with 16-byte cp.async by eight warps
 // into a 4-deep ring (completion tracked by the stage's mbarrier, so the
@@ -27,7 +28,7 @@
 // per warp, and the MMAs consume ~32 bytes/clock.
 //
 // TMEM (512 columns): O (64 x 512 fp32) in columns 0-255 (channels 0-255 in
-// the lower 16 lanes of every lane quarter, 256-511 in the upper 16); two S
+// the lower 16 lanes of every lane quarter, 256-511 in the upper 16); four S
 // buffers of 64 columns, each holding the four partials (issuer i at column
 // offset 32 (i / 2) and lane offset 16 (i % 2)).  A softmax thread owns one
 // head and half of a tile (16 entries).  O is rescaled (TMEM load, multiply,
@@ -35,10 +36,10 @@
 // units; otherwise the stale maximum is kept, which is exact because O and
 // the normaliser l share it.
 //
-// Warp roles (512 threads): warps 0-7 gather the entry tiles (thread 0 also
-// loads q with a 3-D TMA); warps 8-11 issue the MMAs (lane 0 of each; warp 8
-// owns TMEM); warps 12-15 run the softmax and the output epilogue.  All waits
-// are bounded (sm100::mbar_wait).
+// Warp roles (544 threads): warps 0-7 gather the entry tiles (thread 0 also
+// loads q with a 3-D TMA); warps 8-11 issue the S products and warp 12 the O
+// products (lane 0 of each; warp 8 owns TMEM); warps 13-16 run the softmax
+// and the output epilogue.  All waits are bounded (sm100::mbar_wait).
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -62,14 +63,17 @@ constexpr int kQBytes = 8 * kQChunk;        // 64 x 512
 constexpr int kCBytes = 8 * kCChunk;        // one tile: 32 entries x 512
 constexpr int kPBytes = 64 * 128;           // 64 heads x 32 entries (rows padded to 128 B), swizzled
 constexpr int kProducers = 256;             // threads of warps 0-7
-constexpr int kIssuers = 4;                 // warps 8-11
+constexpr int kIssuers = 4;                 // S issuers: warps 8-11
+constexpr int kSBufs = 4;                   // S buffers in TMEM
 constexpr int kOffQ = 0;
 constexpr int kOffC = kOffQ + kQBytes;
 constexpr int kOffP = kOffC + kStages * kCBytes;
-constexpr int kOffMisc = kOffP + 2 * kPBytes;
+constexpr int kStageBytes = 4 * 32 * 128;     // O staging: 32 rows of 128 B per softmax warp
+constexpr int kOffStage = kOffP + 2 * kPBytes;
+constexpr int kOffMisc = kOffStage + kStageBytes;
 constexpr int kMiscBytes = 256;
 constexpr size_t kSmem = 1024 + kOffMisc + kMiscBytes;
-constexpr int kThreads = 512;
+constexpr int kThreads = 544;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256;
 }  // namespace mqa
@@ -79,13 +83,21 @@ __device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 
 
 // Number of kTile-entry tiles a query row needs: up to its last valid slot
 // (0 <= s < avail).  Called by a whole warp; every warp role derives it on
-// its own from the index row.
+// its own from the index row.  The loads go out 16 per lane at a time, so a
+// row of up to 512 slots costs one memory latency.
 __device__ __forceinline__ int mqa_ntiles(const int* ir, int topk, int avail) {
   const int lane = threadIdx.x & 31;
   int last = -1;
-  for (int j = lane; j < topk; j += 32) {
-    const int s = ir[j];
-    if (s >= 0 && s < avail) last = j;
+  for (int j0 = 0; j0 < topk; j0 += 32 * 16) {
+    int v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int j = j0 + 32 * u + lane;
+      v[u] = j < topk ? __ldg(ir + j) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      if (v[u] >= 0 && v[u] < avail) last = j0 + 32 * u + lane;
   }
   last = __reduce_max_sync(0xffffffffu, last);
   return (last + mqa::kTile) / mqa::kTile;
@@ -101,14 +113,15 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
   uint8_t* q_s = sm + kOffQ;
   uint8_t* c_s = sm + kOffC;
   uint8_t* p_s = sm + kOffP;
+  uint8_t* o_stage = sm + kOffStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffMisc);
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;                // every issuer's last S of the item done with q
   uint64_t* c_full = bars + 2;                 // [kStages]
-  uint64_t* t_done = c_full + kStages;         // [kStages] every MMA reading the stage done (frees it)
-  uint64_t* s_full = t_done + kStages;         // [2]  all four S partials written
-  uint64_t* s_free = s_full + 2;               // [2]
-  uint64_t* p_full = s_free + 2;               // [2]
+  uint64_t* t_done = c_full + kStages;         // [kStages] O product of the stage's tile done (frees it)
+  uint64_t* s_full = t_done + kStages;         // [kSBufs] all four S partials written
+  uint64_t* s_free = s_full + kSBufs;          // [kSBufs]
+  uint64_t* p_full = s_free + kSBufs;          // [2]
   uint64_t* o_free = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -122,13 +135,13 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
     mbar_init(q_empty, kIssuers);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&c_full[s], kProducers);
-      mbar_init(&t_done[s], kIssuers);
+      mbar_init(&t_done[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&s_full[s], kIssuers);
       mbar_init(&s_free[s], 4);
-      mbar_init(&p_full[s], 4);
     }
+    for (int s = 0; s < 2; ++s) mbar_init(&p_full[s], 4);
     mbar_init(o_free, 4);
     *abort_flag = 0;
     fence_barrier_init();
@@ -188,17 +201,14 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
     if (!ok && lane == 0) *abort_flag = 1;
     cp_async_wait_all();
   } else if (warp < 12) {
-    // ------------------------------------------------------------ MMA issuers (warps 8-11, lane 0 issues)
+    // ------------------------------------------------------------ S issuers (warps 8-11, lane 0 issues)
     const int iw = warp - 8;
     constexpr uint32_t idS = idesc_bf16_f32(64, kTile);
-    constexpr uint32_t idO = idesc_bf16_f32_bmn(64, 256);
     const uint64_t qd0 = sdesc_k_sw128(smem_u32(q_s));
-    const uint64_t cd0 = sdesc_k_sw128(smem_u32(c_s));                  // stages as K-major operands (S)
-    const uint64_t od0 = sdesc_mn_sw128(smem_u32(c_s), kCChunk, 1024);  // stages as MN-major operands (O)
-    const uint64_t pd0 = sdesc_k_sw128(smem_u32(p_s));
+    const uint64_t cd0 = sdesc_k_sw128(smem_u32(c_s));   // stages as K-major operands
     // this issuer's S partial: channels 128 iw .. + 127 (K chunks 2 iw and 2 iw + 1)
     const uint32_t s_col = tmem + kColS + 32u * (uint32_t)(iw >> 1) + ((uint32_t)(16 * (iw & 1)) << 16);
-    uint32_t g = 0, qw = 0, oi = 0;
+    uint32_t g = 0, qw = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x) {
       if (warp_aborted(abort_flag)) break;
       const int row = a.rows - 1 - it / hgroups;
@@ -209,27 +219,15 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       if (ntiles == 0) continue;
       int ok = 1;
       if (lane == 0) {
-        // O product of tile gj (issuers 0 and 1: channel half iw), once its P is written
-        auto issue_o = [&](uint32_t gj, uint32_t jj) -> bool {
-          const int st = (int)(gj % kStages), pb = (int)(gj & 1);
-          if (!mbar_wait(&p_full[pb], (gj >> 1) & 1)) return false;
-          if (jj == 0 && !mbar_wait(o_free, (oi & 1) ^ 1)) return false;   // previous item's O stored
-          tc_fence_after();
-#pragma unroll
-          for (int ks = 0; ks < kTile / 16; ++ks)
-            mma_bf16(tmem + ((uint32_t)(16 * iw) << 16) + kColO, desc_add(pd0, pb * kPBytes + ks * 32),
-                     desc_add(od0, st * kCBytes + 4 * iw * kCChunk + ks * 2048), idO, (jj > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(&t_done[st]);
-          return true;
-        };
         if (!mbar_wait(q_full, qw & 1)) {
           ok = 0;
         } else {
           tc_fence_after();
-          for (int j = 0; j < ntiles && ok; ++j) {
+          for (int j = 0; j < ntiles; ++j) {
             const uint32_t gj = g + j;
-            const int st = (int)(gj % kStages), sb = (int)(gj & 1);
-            if (!mbar_wait(&c_full[st], (gj / kStages) & 1) || !mbar_wait(&s_free[sb], ((gj >> 1) & 1) ^ 1)) {
+            const int st = (int)(gj % kStages), sb = (int)(gj % kSBufs);
+            if (!mbar_wait(&c_full[st], (gj / kStages) & 1) ||
+                !mbar_wait(&s_free[sb], ((gj / kSBufs) & 1) ^ 1)) {
               ok = 0;
               break;
             }
@@ -245,13 +243,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
               }
             mma_commit(&s_full[sb]);
             if (j == ntiles - 1) mma_commit(q_empty);
-            if (iw >= 2) {
-              mma_commit(&t_done[st]);          // the S partial is this issuer's only use of the stage
-            } else if (j >= 1 && !issue_o(gj - 1, j - 1)) {
-              ok = 0;
-            }
           }
-          if (ok && iw < 2 && !issue_o(g + ntiles - 1, ntiles - 1)) ok = 0;
         }
       }
       ok = __shfl_sync(kFull, ok, 0);
@@ -260,15 +252,60 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
         break;
       }
       ++qw;
+      g += ntiles;
+    }
+  } else if (warp == 12) {
+    // ------------------------------------------------------------ O issuer (warp 12, lane 0 issues)
+    // The stage of a tile is released after its O product, which is issued
+    // only once P is written, i.e. after all four S partials have completed.
+    constexpr uint32_t idO = idesc_bf16_f32_bmn(64, 256);
+    const uint64_t od0 = sdesc_mn_sw128(smem_u32(c_s), kCChunk, 1024);  // stages as MN-major operands
+    const uint64_t pd0 = sdesc_k_sw128(smem_u32(p_s));
+    uint32_t g = 0, oi = 0;
+    for (int it = blockIdx.x; it < items; it += gridDim.x) {
+      if (warp_aborted(abort_flag)) break;
+      const int row = a.rows - 1 - it / hgroups;
+      long long base;
+      int avail;
+      row_entries(a.rm, row, base, avail);
+      const int ntiles = mqa_ntiles(a.idx + (long long)row * a.topk, a.topk, avail);
+      if (ntiles == 0) continue;
+      int ok = 1;
+      if (lane == 0) {
+        for (int j = 0; j < ntiles; ++j) {
+          const uint32_t gj = g + j;
+          const int st = (int)(gj % kStages), pb = (int)(gj & 1);
+          if (!mbar_wait(&p_full[pb], (gj >> 1) & 1) ||
+              (j == 0 && !mbar_wait(o_free, (oi & 1) ^ 1))) {   // previous item's O stored
+            ok = 0;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int ks = 0; ks < kTile / 16; ++ks)
+              mma_bf16(tmem + ((uint32_t)(16 * hh) << 16) + kColO, desc_add(pd0, pb * kPBytes + ks * 32),
+                       desc_add(od0, st * kCBytes + 4 * hh * kCChunk + ks * 2048), idO,
+                       (j > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&t_done[st]);
+        }
+      }
+      ok = __shfl_sync(kFull, ok, 0);
+      if (!ok) {
+        if (lane == 0) *abort_flag = 1;
+        break;
+      }
       ++oi;
       g += ntiles;
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue (warps 12-15)
+    // ------------------------------------------------------------ softmax + epilogue (warps 13-16)
     const int sub = warp & 3;                  // TMEM lane quarter of this warp
     const int hrow = 16 * sub + (lane & 15);   // head row (within the group)
     const int half = lane >> 4;                // S: entries 16 half .. + 15 of a tile; O: channels 256 half ..
     const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
+    uint8_t* ostage = o_stage + (warp - 13) * (32 * 128);   // this warp's 32 staging rows
     uint32_t g = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x) {
       if (warp_aborted(abort_flag)) break;
@@ -278,27 +315,30 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       row_entries(a.rm, row, base, avail);
       const int* ir = a.idx + (long long)row * a.topk;
       const int ntiles = mqa_ntiles(ir, a.topk, avail);
-      __nv_bfloat16* orow = a.O + (long long)row * a.ld_O + (long long)(hg * kHeads + hrow) * kC + half * 256;
       if (ntiles == 0) {   // nothing visible: the attention output is zero
+        __nv_bfloat16* orow = a.O + (long long)row * a.ld_O + (long long)(hg * kHeads + hrow) * kC + half * 256;
         const uint4 z = make_uint4(0, 0, 0, 0);
         for (int i = 0; i < 32; ++i) reinterpret_cast<uint4*>(orow)[i] = z;
         continue;
       }
       float m_run = -INFINITY, l_run = 0.f;    // l_run: this lane's half of the normaliser
       bool ok = true;
+      int sidx = lane < a.topk ? __ldg(ir + lane) : -1;   // slot of this lane in tile 0
       for (int j = 0; j < ntiles; ++j) {
         const uint32_t gj = g + j;
-        const int sb = (int)(gj & 1);
-        // validity of this tile's 32 slots, from the index row itself
-        const int e = j * kTile + lane;
-        const int sidx = e < a.topk ? ir[e] : -1;
+        const int sb = (int)(gj % kSBufs), pb = (int)(gj & 1);
+        // validity of this tile's 32 slots; the next tile's slot is fetched meanwhile
         const uint32_t vmask = __ballot_sync(kFull, sidx >= 0 && sidx < avail);
-        if (!warp_wait(&s_full[sb], (gj >> 1) & 1)) { ok = false; break; }
+        {
+          const int e = (j + 1) * kTile + lane;
+          sidx = (j + 1 < ntiles && e < a.topk) ? __ldg(ir + e) : -1;
+        }
+        if (!warp_wait(&s_full[sb], (gj / kSBufs) & 1)) { ok = false; break; }
         tc_fence_after();
         // partials of issuers `half` (x) and `half + 2` (y) for all 32 entries of head hrow
         float x[kTile], y[kTile];
-        tmem_ld_32x32b_x32(tmem + lane_base + kColS + 64u * (uint32_t)sb, x);
-        tmem_ld_32x32b_x32(tmem + lane_base + kColS + 64u * (uint32_t)sb + 32u, y);
+        tmem_ld_32x32b_x32_pair(tmem + lane_base + kColS + 64u * (uint32_t)sb,
+                                tmem + lane_base + kColS + 64u * (uint32_t)sb + 32u, x, y);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
@@ -309,20 +349,37 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
         for (int k = 0; k < 16; ++k) {
           const float mine = half ? x[16 + k] + y[16 + k] : x[k] + y[k];
           const float other = half ? x[k] + y[k] : x[16 + k] + y[16 + k];
-          const float s = mine + __shfl_xor_sync(kFull, other, 16);
-          sv[k] = ((vmask >> (16 * half + k)) & 1u) ? s * a.scale_log2 : -INFINITY;
+          const float sk = mine + __shfl_xor_sync(kFull, other, 16);
+          sv[k] = ((vmask >> (16 * half + k)) & 1u) ? sk * a.scale_log2 : -INFINITY;
           tmax = fmaxf(tmax, sv[k]);
         }
         tmax = fmaxf(tmax, __shfl_xor_sync(kFull, tmax, 16));
         const float m_new = fmaxf(m_run, tmax);
         const bool grow = m_new > m_run + 8.f;   // also true on the first finite tile
         const float m_use = grow ? m_new : m_run;
+        // P of this lane's 16 entries (bf16) and their sum
+        float sum = 0.f;
+        uint4 pk[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float x0 = sv[8 * u + 2 * q], x1 = sv[8 * u + 2 * q + 1];
+            const float p0 = x0 == -INFINITY ? 0.f : ex2_approx(x0 - m_use);
+            const float p1 = x1 == -INFINITY ? 0.f : ex2_approx(x1 - m_use);
+            sum += p0 + p1;
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            w[q] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          pk[u] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
         if (__any_sync(kFull, grow && j > 0)) {
           // rescale O: the O products of the earlier tiles must have completed
           const uint32_t gp = gj - 1;
           if (!warp_wait(&t_done[gp % kStages], (gp / kStages) & 1)) { ok = false; break; }
           tc_fence_after();
-          const float alpha = grow ? exp2f(m_run - m_new) : 1.f;   // exp2(-inf) = 0 when nothing was seen
+          const float alpha = grow ? ex2_approx(m_run - m_new) : 1.f;   // 2^-inf = 0 when nothing was seen
 #pragma unroll 1
           for (int ch = 0; ch < 8; ++ch) {
             float v[32];
@@ -336,35 +393,27 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
           l_run *= alpha;
         }
         m_run = m_use;
+        l_run += sum;
         // P rows, once the P buffer's previous reader (tile gj - 2) is done
         if (gj >= 2) {
           const uint32_t gp = gj - 2;
           if (!warp_wait(&t_done[gp % kStages], (gp / kStages) & 1)) { ok = false; break; }
         }
-        uint8_t* prow = p_s + sb * kPBytes;
-        float sum = 0.f;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          Vec16<__nv_bfloat16> pk;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float xv = sv[8 * u + q];
-            const float p = (xv == -INFINITY) ? 0.f : exp2f(xv - m_use);
-            sum += p;
-            pk.e[q] = __float2bfloat16_rn(p);
-          }
-          *reinterpret_cast<uint4*>(prow + sw128(hrow, 2 * half + u)) = pk.u;
-        }
-        l_run += sum;
+        uint8_t* prow = p_s + pb * kPBytes;
+        *reinterpret_cast<uint4*>(prow + sw128(hrow, 2 * half)) = pk[0];
+        *reinterpret_cast<uint4*>(prow + sw128(hrow, 2 * half + 1)) = pk[1];
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[sb]);
+        if (lane == 0) mbar_arrive(&p_full[pb]);
       }
       if (!ok) {
         if (lane == 0) *abort_flag = 1;
         break;
       }
-      // epilogue: O / l for this lane's head and channel half
+      // epilogue: O / l in four passes of 64 channels per lane (channels
+      // 64 p .. for the lanes of half 0, 256 + 64 p .. for half 1).  Each
+      // pass goes through this warp's 32 staging rows (row = lane) and leaves
+      // as whole 128-byte rows: 4 rows per warp store instead of 32 pieces.
       const float l = l_run + __shfl_xor_sync(kFull, l_run, 16);
       const uint32_t glast = g + ntiles - 1;
       if (!warp_wait(&t_done[glast % kStages], (glast / kStages) & 1)) {
@@ -373,21 +422,35 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       }
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* obase = a.O + (long long)row * a.ld_O + (long long)(hg * kHeads + 16 * sub) * kC;
 #pragma unroll 1
-      for (int ch = 0; ch < 8; ++ch) {
-        float v[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + kColO + ch * 32, v);
-#pragma unroll
-        for (int qd = 0; qd < 4; ++qd) {
-          Vec16<__nv_bfloat16> pk;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) pk.e[q] = __float2bfloat16_rn(v[8 * qd + q] * inv);
-          reinterpret_cast<uint4*>(orow + ch * 32)[qd] = pk.u;
+      for (int p = 0; p < 4; ++p) {
+        float v0[32], v1[32];
+        tmem_ld_32x32b_x32_pair(tmem + lane_base + kColO + 64u * (uint32_t)p,
+                                tmem + lane_base + kColO + 64u * (uint32_t)p + 32u, v0, v1);
+        if (p == 3) {   // O is in registers: the next item's O products may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float* vv = u < 4 ? v0 : v1;
+          Vec16<__nv_bfloat16> pkv;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) pkv.e[q] = __float2bfloat16_rn(vv[8 * (u & 3) + q] * inv);
+          *reinterpret_cast<uint4*>(ostage + sw128(lane, u)) = pkv.u;
+        }
+        __syncwarp();
+        // staging row r holds head 16 sub + r % 16, channels 256 (r / 16) + 64 p ..
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 4 * i + (lane >> 3), u = lane & 7;
+          const uint4 val = *reinterpret_cast<const uint4*>(ostage + sw128(r, u));
+          *reinterpret_cast<uint4*>(obase + (r & 15) * kC + 256 * (r >> 4) + 64 * p + 8 * u) = val;
+        }
+        __syncwarp();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(o_free);
       g += ntiles;
     }
   }
