@@ -90,7 +90,8 @@ class ClockSampler:
         self.proc = None
         self.lines = []
 
-    def start(self):
+    def start(self, wait_s=5.0):
+        """Starts sampling every 50 ms and waits (at most wait_s) for the first sample."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -99,12 +100,17 @@ class ClockSampler:
             self.t.start()
         except OSError:
             self.proc = None
+            return
+        t_end = time.monotonic() + wait_s
+        while not self.lines and time.monotonic() < t_end:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
+        """Summary of the samples taken in [t0, t1] (monotonic seconds; all when not given)."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -115,7 +121,11 @@ class ClockSampler:
         self.t.join(timeout=2)
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = [ln for t, ln in self.lines if (t0 is None or t >= t0) and (t1 is None or t <= t1)]
+        if not lines and self.lines and t0 is not None:   # none inside a short window: the next one after it
+            later = [ln for t, ln in self.lines if t >= t0]
+            lines = later[:1]
+        for ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -134,6 +144,16 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ timing helpers
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# a stage's kernel, from one ncu capture of the current kernel version on the
+# named workload (profiles/<kernel>_<workload>.md).  A kernel change makes the
+# figure stale: it is then removed until the next capture.
+MEASURED_TRAFFIC = {
+    ("prefill", "A5_sparse_mqa"): 557_040_896 + 492_750_080,
+    ("prefill", "A4_indexer_topk"): 102_903_808 + 7_520_000,
+}
+
+
 def timed_steps(fn, steps, flush, stream):
     """Per-step CUDA-event durations (ms) of fn(), with an L2 flush before each step."""
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
@@ -260,29 +280,48 @@ class DecodeRunner:
 
 
 # ------------------------------------------------------------------ oracle baseline
+class OracleSampler:
+    """Times the fp64 oracle on bounded samples of a workload, extrapolated to
+    tokens/s.  The per-token part (projections of every token and the
+    compression) is timed once in full by `base()`; each `sample()` then runs
+    one oracle forward with eqs. 5-11 on `rows_sample` seeded query rows and
+    extrapolates its per-row cost to every row."""
+
+    def __init__(self, w, rows_sample):
+        from oracle import csa_oracle as orc
+        self.orc, self.w = orc, w
+        d = w.dims
+        self.W = {k: v.double().numpy() for k, v in synth.make_weights(d, w.seed).items()}
+        self.T = sum(w.seqlens)
+        self.H = synth.make_hidden(self.T, d, w.seed).double().numpy()
+        self.od = dict(m=d.m, topk=d.topk, nh=d.nh, nhI=d.nhI, c=d.c, cI=d.cI)
+        self.store = "bf16" if d.dtype == csa.CSA_BF16 else "f32"
+        self.rows_sample = min(rows_sample, self.T)
+        self.base_s = None
+
+    def _forward(self, rows):
+        t0 = time.perf_counter()
+        self.orc.csa_forward(self.H, self.W, self.od, list(self.w.seqlens), store=self.store, rows=rows)
+        return time.perf_counter() - t0
+
+    def base(self):
+        self.base_s = self._forward(np.zeros(0, dtype=np.int64))
+        return self.base_s
+
+    def sample(self, seed):
+        if self.base_s is None:
+            self.base()
+        rows = np.sort(np.random.default_rng(seed).choice(self.T, size=self.rows_sample, replace=False))
+        t = self._forward(rows)
+        per_row = max(t - self.base_s, 0.0) / len(rows)
+        return self.T / (self.base_s + per_row * self.T), dict(base_s=self.base_s, per_row_s=per_row,
+                                                               rows=len(rows), wall_s=t)
+
+
 def oracle_sample(w, rows_sample, seed=0):
-    """Time the fp64 oracle on a bounded sample of the workload and extrapolate
-    to tokens/s: the per-token part (projections of every token and the
-    compression) is run in full, the per-query part (eqs. 5-11) on
-    `rows_sample` seeded query rows."""
-    from oracle import csa_oracle as orc
-    d = w.dims
-    W = {k: v.double().numpy() for k, v in synth.make_weights(d, w.seed).items()}
-    T = sum(w.seqlens)
-    H = synth.make_hidden(T, d, w.seed).double().numpy()
-    od = dict(m=d.m, topk=d.topk, nh=d.nh, nhI=d.nhI, c=d.c, cI=d.cI)
-    store = "bf16" if d.dtype == csa.CSA_BF16 else "f32"
-    rng = np.random.default_rng(seed)
-    rows = np.sort(rng.choice(T, size=min(rows_sample, T), replace=False))
-    t0 = time.perf_counter()
-    orc.csa_forward(H, W, od, list(w.seqlens), store=store, rows=np.zeros(0, dtype=np.int64))
-    t1 = time.perf_counter()
-    orc.csa_forward(H, W, od, list(w.seqlens), store=store, rows=rows)
-    t2 = time.perf_counter()
-    base = t1 - t0
-    per_row = max((t2 - t1) - base, 0.0) / len(rows)
-    est = base + per_row * T
-    return T / est, dict(base_s=base, per_row_s=per_row, rows=len(rows), wall_s=t2 - t0)
+    """One bounded oracle sample of the workload (base part timed in full,
+    eqs. 5-11 on `rows_sample` rows), extrapolated to tokens/s."""
+    return OracleSampler(w, rows_sample).sample(seed)
 
 
 def blas_threads():
@@ -296,20 +335,37 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
+def max_over_ranks(ms, dev, world):
+    """The slowest rank's device time (every rank takes part; world 1: ms itself)."""
+    if world == 1:
+        return ms
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step, steps, world, max_ms):
+    """Whole-job tokens/s: the tokens every rank processed over the slowest rank's time."""
+    return tokens_per_rank_step * steps * world / (max_ms / 1000.0)
+
+
 # ------------------------------------------------------------------ arms
 def run_reference(args, rank, world):
     if rank != 0:
         return
     w = synth.workloads()[args.workload]
+    sampler = OracleSampler(w, args.ref_rows)
+    sampler.base()                      # the token-parallel part, timed in full once
     times = []
     info = None
     for i in range(args.warmup + args.steps):
-        tps, info = oracle_sample(w, rows_sample=args.ref_rows, seed=i)
+        tps, info = sampler.sample(seed=i)
         if i >= args.warmup:
             times.append(tps)
     value = statistics.mean(times)
-    sample = (f"oracle forward: projections + compression of all {sum(w.seqlens)} tokens in full, "
-              f"eqs. 5-11 on {info['rows']} seeded query rows per step, extrapolated to every row")
+    sample = (f"oracle forward per step with eqs. 5-11 on {info['rows']} seeded query rows, extrapolated "
+              f"to all {sum(w.seqlens)} rows; projections + compression of every token timed in full "
+              f"({info['base_s']:.2f} s) before the steps")
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000.0 * sum(w.seqlens) / value, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
@@ -342,34 +398,34 @@ def run_ours(args, rank, world, local_rank):
     def flush():
         flush_buf.fill_(1)
 
+    # clock sampling starts before the warm-up: nvidia-smi's first sample takes a while
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    sampler.start()
     for _ in range(args.warmup):
         runner.forward()
     torch.cuda.synchronize()
     st = csa.csa_get_device_status()
     if st != 0:
+        sampler.stop()
         raise RuntimeError(f"device status after warm-up: {csa.status_string(st)}")
 
-    # ---- timed region: exactly K steps
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    # ---- timed region: exactly K steps (clock samples kept from inside it only)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    sampler.start()
+    t_sample0 = time.monotonic()
     n0 = csa.csa_launch_count()
     step_ms = timed_steps(runner.forward, args.steps, flush, stream)
     launches = csa.csa_launch_count() - n0
     torch.cuda.synchronize()
+    t_sample1 = time.monotonic()
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop()
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    clocks = sampler.stop(t_sample0, t_sample1)
+    total_ms = max_over_ranks(sum(step_ms), dev, world)
     tokens = runner.T * args.steps * world
-    value = tokens / (total_ms / 1000.0)
+    value = job_throughput(runner.T, args.steps, world, total_ms)
     ms_per_step = total_ms / args.steps
 
     # ---- end to end through host buffers (H2D of H, forward, D2H of O)
@@ -377,11 +433,7 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_e2e:
         for _ in range(2):
             runner.forward_e2e()
-        e2e_ms = sum(timed_steps(runner.forward_e2e, args.steps, flush, stream))
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(sum(timed_steps(runner.forward_e2e, args.steps, flush, stream)), dev, world)
         e2e = {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": runner.H.numel() * runner.H.element_size(),
                "d2h_bytes_per_step": runner.O.numel() * runner.O.element_size()}
@@ -414,7 +466,7 @@ def run_ours(args, rank, world, local_rank):
         top = max(stages, key=lambda k: stages[k]["ms"])
         s = stages[top]
         roofline = {"kernel": top, "bound": s["bound"], "achieved": s["achieved"], "peak": s["peak"],
-                    "unit": s["unit"], "frac": s["frac"], "traffic": None,
+                    "unit": s["unit"], "frac": s["frac"], "traffic": MEASURED_TRAFFIC.get((args.workload, top)),
                     "peak_source": f"{peaks['source']} ({'hbm_gbs' if s['bound'] == 'hbm' else 'bf16_tflops'})"}
 
     # ---- decode workload, same build
@@ -483,7 +535,7 @@ def runner_T(w):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["prefill", "tiny", "long", "ragged"], default="prefill")
