@@ -150,7 +150,6 @@ class ClockSampler:
 # figure stale: it is then removed until the next capture.
 MEASURED_TRAFFIC = {
     ("prefill", "A5_sparse_mqa"): 557_040_896 + 492_750_080,
-    ("prefill", "A4_indexer_topk"): 102_903_808 + 7_520_000,
 }
 
 

@@ -290,12 +290,12 @@ csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int
   t.topk = d->topk; t.nhI = d->nhI; t.cI = d->cI;
   t.cu_seqlens = a.rm.cu_seqlens; t.cu_blocks = a.rm.cu_blocks; t.nseq = a.rm.nseq; t.total_blocks = NB;
   t.total_tokens = T;
-  if (cudaFuncSetAttribute(indexer_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)idxtc::kSmem) !=
-      cudaSuccess)
+  auto kern = d->nhI == 64 ? indexer_tc_kernel<64> : indexer_tc_kernel<32>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)idxtc::kSmem) != cudaSuccess)
     return CSA_ERR_CUDA;
   const long long items = (long long)NB + a.rm.nseq;
   const int grid = items < sm_count() ? (int)items : sm_count();
-  indexer_tc_kernel<<<grid, idxtc::kThreads, idxtc::kSmem, st>>>(tk, tq, t);
+  kern<<<grid, idxtc::kThreads, idxtc::kSmem, st>>>(tk, tq, t);
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }

@@ -44,12 +44,14 @@ constexpr int kM = 128;                 // blocks per tile
 constexpr int kStages = 3;
 constexpr int kQChunk = 256 * 128;      // [4 x nhI <= 256 rows x 64 bf16]
 constexpr int kKChunk = kM * 128;       // [128 rows x 64 bf16]
+constexpr int kSelChunk = 1536;         // scores staged in shared memory per selection warp
+constexpr int kHistBins = 2048;         // radix histogram per selection warp (11-bit digits)
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + 2 * kQChunk;
 constexpr int kOffW = kOffK + kStages * 2 * kKChunk;   // 4 warps x [4 x 64] floats
-constexpr int kOffH = kOffW + 4 * 256 * 4;             // 4 warps x 256 bins
-constexpr int kOffS = kOffH + 4 * 256 * 4;             // 4 warps x kSelChunk staged scores
-constexpr int kOffB = kOffS + 4 * 2048 * 4;
+constexpr int kOffH = kOffW + 4 * 256 * 4;             // 4 warps x kHistBins counts
+constexpr int kOffS = kOffH + 4 * kHistBins * 4;       // 4 warps x kSelChunk staged scores
+constexpr int kOffB = kOffS + 4 * kSelChunk * 4;
 constexpr size_t kSmem = 1024 + kOffB + 256;
 constexpr int kThreads = 320;
 }  // namespace idxtc
@@ -82,103 +84,171 @@ __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, 
 }
 
 // Exact top-k of sc[0..n) (n > k) by one warp, written to out[0..k) as
-// ascending indices; equal scores are taken lowest index first.  The row is
-// read through `buf` (kSelChunk floats of shared memory) a chunk at a time
-// with 16-byte loads, all in flight together; a row that fits in one chunk
-// is read once and every pass runs on shared memory.  Radix select on the
-// order-preserving 32-bit keys: 4 passes of 8-bit histograms find the k-th
-// largest key and how many keys equal to it are taken, then an ordered pass
-// writes the winners.
-constexpr int kSelChunk = 2048;
-
+// ascending indices; equal scores are taken lowest index first.
+//
+// Radix select on the order-preserving 32-bit keys, most significant digit
+// first, in three passes of 11, 11 and 10 bits: each pass histograms the
+// digit of the keys that share the digits found so far and picks the digit
+// holding the kk-th largest of them; the last pass leaves the k-th largest
+// key `thr` itself and how many keys equal to it are taken.  An ordered pass
+// then writes every key > thr and the first `need_eq` keys == thr.
+//
+// The row is read through `buf` (kSelChunk floats of shared memory) a chunk
+// at a time, eight 16-byte loads per lane in flight; a row that fits in one
+// chunk is read from global memory once and every pass runs on shared
+// memory.  Each lane takes four consecutive scores per step, so that
+// four independent key/histogram chains are in flight per lane.
 __device__ __forceinline__ void warp_stage_chunk(const float* src, int n, float* buf) {
+  constexpr int kBatch = 8;   // 16-byte loads in flight per lane
   const int lane = threadIdx.x & 31;
-  // n <= kSelChunk; 16-byte loads where the whole vector is in range
-  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
-  if (vec) {
+  if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
     const int n4 = n >> 2;
-#pragma unroll 4
-    for (int i = lane; i < n4; i += 32) reinterpret_cast<float4*>(buf)[i] = __ldcg(reinterpret_cast<const float4*>(src) + i);
+    for (int i0 = 0; i0 < n4; i0 += 32 * kBatch) {
+      float4 r[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + lane + 32 * u;
+        if (i < n4) r[u] = __ldcg(reinterpret_cast<const float4*>(src) + i);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + lane + 32 * u;
+        if (i < n4) reinterpret_cast<float4*>(buf)[i] = r[u];
+      }
+    }
     for (int i = (n4 << 2) + lane; i < n; i += 32) buf[i] = __ldcg(src + i);
   } else {
-#pragma unroll 4
+#pragma unroll 8
     for (int i = lane; i < n; i += 32) buf[i] = __ldcg(src + i);
   }
   __syncwarp();
 }
 
-__device__ void warp_topk_ascending(const float* sc, int n, int k, int* out, int* hist, float* buf) {
+// One radix pass over the keys k of sc[0..n) with (k & mask) == prefix:
+// returns the WIDTH-bit digit at `shift` that holds the kk-th largest of
+// them (kk >= 1, at most their number) and, in *above, how many of them have
+// a larger digit.  hist holds 2^WIDTH ints of shared memory.
+template <int WIDTH>
+__device__ __noinline__ uint32_t warp_radix_pass(const float* sc, int n, bool resident, float* buf, int* hist,
+                                                 int shift, uint32_t mask, uint32_t prefix, int kk, int* above) {
+  constexpr int NB = 1 << WIDTH, PER = NB / 32, SUB = PER / 32;
+  constexpr unsigned kFull = 0xffffffffu;
   const int lane = threadIdx.x & 31;
-  const bool resident = n <= kSelChunk;
-  if (resident) warp_stage_chunk(sc, n, buf);
-  uint32_t prefix = 0, mask = 0;
-  int kk = k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = lane; i < 256; i += 32) hist[i] = 0;
-    __syncwarp();
-    for (int c0 = 0; c0 < n; c0 += kSelChunk) {
-      const int cn = min(kSelChunk, n - c0);
-      if (!resident) warp_stage_chunk(sc + c0, cn, buf);
-      for (int s = lane; s < cn; s += 32) {
-        const uint32_t key = ordered_key(buf[s]);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-      }
-      __syncwarp();
-    }
-    // lane L owns bins 255-8L .. 248-8L (descending); find the digit holding the kk-th largest
-    int cnt[8], tot = 0;
+#pragma unroll 4
+  for (int i = lane; i < NB / 4; i += 32) reinterpret_cast<int4*>(hist)[i] = make_int4(0, 0, 0, 0);
+  __syncwarp();
+  for (int c0 = 0; c0 < n; c0 += idxtc::kSelChunk) {
+    const int cn = min(idxtc::kSelChunk, n - c0);
+    if (!resident) warp_stage_chunk(sc + c0, cn, buf);
+    // buf holds kSelChunk floats, a multiple of 4: the last vector may run
+    // past cn but not past the buffer; its extra elements are masked
+    const int nv = (cn + 3) >> 2;
+#pragma unroll 2
+    for (int i = lane; i < nv; i += 32) {
+      const float4 v = reinterpret_cast<const float4*>(buf)[i];
+      const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) { cnt[j] = hist[255 - 8 * lane - j]; tot += cnt[j]; }
-    int incl = tot;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    const int excl = incl - tot;
-    const unsigned hit = __ballot_sync(0xffffffffu, excl < kk && incl >= kk);
-    const int src = __ffs(hit) - 1;
-    int digit = 0, before = 0;
-    if (lane == src) {
-      int c = excl;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (c + cnt[j] >= kk) { digit = 255 - 8 * lane - j; before = c; break; }
-        c += cnt[j];
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t key = ordered_key(e[u]);
+        if (4 * i + u < cn && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint32_t)(NB - 1)], 1);
       }
     }
-    digit = __shfl_sync(0xffffffffu, digit, src);
-    before = __shfl_sync(0xffffffffu, before, src);
-    prefix |= (uint32_t)digit << shift;
-    mask |= 255u << shift;
-    kk -= before;
     __syncwarp();
   }
+  // Position p = NB - 1 - digit (p = 0 is the largest digit).  Lane L sums
+  // positions [PER L, PER L + PER), visiting them in a lane-rotated order so
+  // that the 32 lanes read 32 different banks.
+  int tot = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) tot += hist[NB - 1 - (PER * lane + ((j + lane) & (PER - 1)))];
+  int incl = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(kFull, incl, off);
+    if (lane >= off) incl += v;
+  }
+  const int excl = incl - tot;
+  const int src = __ffs(__ballot_sync(kFull, excl < kk && incl >= kk)) - 1;
+  const int excl_src = __shfl_sync(kFull, excl, src);
+  const int kk2 = kk - excl_src;
+  // within the range of lane `src`: SUB positions per lane
+  const int p0 = PER * src + SUB * lane;
+  int c2 = 0;
+#pragma unroll
+  for (int u = 0; u < SUB; ++u) c2 += hist[NB - 1 - (p0 + u)];
+  int incl2 = c2;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(kFull, incl2, off);
+    if (lane >= off) incl2 += v;
+  }
+  const int excl2 = incl2 - c2;
+  const int src2 = __ffs(__ballot_sync(kFull, excl2 < kk2 && incl2 >= kk2)) - 1;
+  int pos = 0, before = 0;
+  if (lane == src2) {
+    int c = excl2;
+#pragma unroll
+    for (int u = 0; u < SUB; ++u) {
+      const int v = hist[NB - 1 - (p0 + u)];
+      if (c + v >= kk2) { pos = p0 + u; before = c; break; }
+      c += v;
+    }
+  }
+  pos = __shfl_sync(kFull, pos, src2);
+  before = __shfl_sync(kFull, before, src2);
+  __syncwarp();
+  *above = excl_src + before;
+  return (uint32_t)(NB - 1 - pos);
+}
+
+__device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, int* out, int* hist, float* buf) {
+  constexpr unsigned kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const bool resident = n <= idxtc::kSelChunk;
+  if (resident) warp_stage_chunk(sc, n, buf);
+  int kk = k, above;
+  uint32_t prefix = warp_radix_pass<11>(sc, n, resident, buf, hist, 21, 0u, 0u, kk, &above) << 21;
+  kk -= above;
+  prefix |= warp_radix_pass<11>(sc, n, resident, buf, hist, 10, 0xFFE00000u, prefix, kk, &above) << 10;
+  kk -= above;
+  prefix |= warp_radix_pass<10>(sc, n, resident, buf, hist, 0, 0xFFFFFC00u, prefix, kk, &above);
+  kk -= above;
   const uint32_t thr = prefix;
   const int need_eq = kk;
   int out_off = 0, eq_seen = 0;
   const unsigned lt = (1u << lane) - 1u;
-  for (int c0 = 0; c0 < n; c0 += kSelChunk) {
-    const int cn = min(kSelChunk, n - c0);
+  for (int c0 = 0; c0 < n; c0 += idxtc::kSelChunk) {
+    const int cn = min(idxtc::kSelChunk, n - c0);
     if (!resident) warp_stage_chunk(sc + c0, cn, buf);
-    for (int base = 0; base < cn; base += 32) {
-      const int s = base + lane;
-      const uint32_t key = s < cn ? ordered_key(buf[s]) : 0u;
-      const bool gt = s < cn && key > thr;
-      const bool eq = s < cn && key == thr;
-      const unsigned beq = __ballot_sync(0xffffffffu, eq);
-      const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
-      const unsigned btk = __ballot_sync(0xffffffffu, take);
-      const int p = out_off + __popc(btk & lt);
-      if (take && p < k) out[p] = c0 + s;
-      out_off += __popc(btk);
-      eq_seen += __popc(beq);
+    for (int base = 0; base < cn; base += 128) {
+      // four 32-score groups: keys first (independent loads), then the
+      // ordered compaction group by group
+      uint32_t key[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int s = base + 32 * u + lane;
+        key[u] = s < cn ? ordered_key(buf[s]) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int s = base + 32 * u + lane;
+        const bool gt = s < cn && key[u] > thr;
+        const bool eq = s < cn && key[u] == thr;
+        const unsigned beq = __ballot_sync(kFull, eq);
+        const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
+        const unsigned btk = __ballot_sync(kFull, take);
+        const int p = out_off + __popc(btk & lt);
+        if (take && p < k) out[p] = c0 + s;
+        out_off += __popc(btk);
+        eq_seen += __popc(beq);
+      }
     }
     __syncwarp();
   }
 }
 
+// NHI = n_h^I (32 or 64; a.nhI must equal it).
+template <int NHI>
 __global__ void __launch_bounds__(idxtc::kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IdxTcArgs a) {
   using namespace sm100;
@@ -203,9 +273,9 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = 4 * a.nhI;                      // MMA N: (query, head) pairs
+  constexpr int N = 4 * NHI;                    // MMA N: (query, head) pairs
   const int kchunks = a.cI / 64;
-  const uint32_t tmem_cols = N <= 128 ? 256 : 512;
+  constexpr uint32_t tmem_cols = N <= 128 ? 256 : 512;
   const int items = a.total_blocks + a.nseq;
 
   if (threadIdx.x == 0) {
@@ -247,6 +317,19 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
         mbar_arrive_expect_tx(q_full, (uint32_t)(kchunks * N * 128));
         for (int c = 0; c < kchunks; ++c) tma_load_3d(&tmQ, q_full, q_s + c * kQChunk, 64 * c, 0, tok0);
         ++qi;
+        {
+          // the next item's q^I and w^I rows go to L2 while this item runs,
+          // so that its q^I load (issued only once this item's MMAs are
+          // done) and its head weights come from L2
+          int tok1, nq1, av1;
+          long long kb1;
+          const int nx = it + (int)gridDim.x;
+          if (nx < items && idx_item(a, nx, tok1, nq1, av1, kb1) && av1 > a.topk) {
+            for (int c = 0; c < kchunks; ++c) tma_prefetch_3d(&tmQ, 64 * c, 0, tok1);
+            for (int q = 0; q < nq1; ++q)
+              for (int h = 0; h < NHI; h += 32) prefetch_l2(a.wI + (long long)(tok1 + q) * a.ld_wI + h);
+          }
+        }
         bool ok = true;
         for (int j = 0; j < ntiles; ++j, ++g) {
           const int st = g % kStages;
@@ -306,8 +389,8 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
       const int ntiles = (avail + kM - 1) / kM;
       const int buf = wi & 1;
       float* scr = a.scratch + ((size_t)blockIdx.x * 2 + buf) * 4 * a.sc_cap;
-      for (int e = lane; e < 4 * a.nhI; e += 32) {
-        const int q = e / a.nhI, h = e - q * a.nhI;
+      for (int e = lane; e < 4 * NHI; e += 32) {
+        const int q = e / NHI, h = e - q * NHI;
         w_my[q * 64 + h] = q < nq ? a.wI[(long long)(tok0 + q) * a.ld_wI + h] : 0.f;
       }
       __syncwarp();
@@ -319,22 +402,27 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
         if (!warp_wait(&t_full[acc], (acc_it >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const int s = j * kM + 32 * sub + lane;
+        // eight independent partial sums per query keep the FMA chains short
         for (int q = 0; q < nq; ++q) {
-          float acc_s = 0.f;
-          for (int hc = 0; hc < a.nhI; hc += 32) {
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) p[e] = 0.f;
+#pragma unroll 1
+          for (int hc = 0; hc < NHI; hc += 32) {
             float v[32];
-            tmem_ld_32x32b_x32(tmem + lane_base + (uint32_t)(acc * N + q * a.nhI + hc), v);
+            tmem_ld_32x32b_x32(tmem + lane_base + (uint32_t)(acc * N + q * NHI + hc), v);
             const float4* w4 = reinterpret_cast<const float4*>(w_my + q * 64 + hc);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float4 w = w4[e];
-              acc_s = fmaf(w.x, fmaxf(v[4 * e + 0], 0.f), acc_s);
-              acc_s = fmaf(w.y, fmaxf(v[4 * e + 1], 0.f), acc_s);
-              acc_s = fmaf(w.z, fmaxf(v[4 * e + 2], 0.f), acc_s);
-              acc_s = fmaf(w.w, fmaxf(v[4 * e + 3], 0.f), acc_s);
+              p[(4 * e + 0) & 7] = fmaf(w.x, fmaxf(v[4 * e + 0], 0.f), p[(4 * e + 0) & 7]);
+              p[(4 * e + 1) & 7] = fmaf(w.y, fmaxf(v[4 * e + 1], 0.f), p[(4 * e + 1) & 7]);
+              p[(4 * e + 2) & 7] = fmaf(w.z, fmaxf(v[4 * e + 2], 0.f), p[(4 * e + 2) & 7]);
+              p[(4 * e + 3) & 7] = fmaf(w.w, fmaxf(v[4 * e + 3], 0.f), p[(4 * e + 3) & 7]);
             }
           }
-          if (s < avail) __stcg(scr + (size_t)q * a.sc_cap + s, acc_s);
+          const float sc = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+          if (s < avail) __stcg(scr + (size_t)q * a.sc_cap + s, sc);
         }
         tc_fence_before();
         __syncwarp();
@@ -348,7 +436,7 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
   } else {
     // ------------------------------------------------------------ selection (warps 6-9): one query each
     const int q = warp - 6;
-    int* hist = h_s + q * 256;
+    int* hist = h_s + q * kHistBins;
     uint32_t wi = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x) {
       if (warp_aborted(abort_flag)) break;
