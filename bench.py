@@ -175,8 +175,6 @@ class PrefillRunner:
         W = synth.make_weights(d, w.seed)
         self.packed = torch.empty(csa.csa_packed_weights_bytes(d), dtype=torch.uint8, device=dev)
         csa.csa_pack_weights(d, {k: v.to(dev) for k, v in W.items()}, self.packed)
-        # fp32 position biases for the stand-alone compression stage
-        self.bias = {k: W[k].float().to(dev) for k in ("B_a", "B_b", "B_a_I", "B_b_I")}
         del W
         self.H_host = synth.make_hidden(self.T, d, w.seed).pin_memory()
         self.H = self.H_host.to(dev)
@@ -220,12 +218,8 @@ class PrefillRunner:
         def col(j):
             return Y1.data_ptr() + j * es
 
-        def a3():
-            csa.csa_compress(d, col(0), col(c), col(2 * c), col(3 * c), N1b, self.bias["B_a"], self.bias["B_b"], c,
-                             self.cu, self.cb, self.nseq, T, self.NB, self.Cc)
-            o = 4 * c
-            csa.csa_compress(d, col(o), col(o + cI), col(o + 2 * cI), col(o + 3 * cI), N1b, self.bias["B_a_I"],
-                             self.bias["B_b_I"], cI, self.cu, self.cb, self.nseq, T, self.NB, self.KI)
+        def a3():   # both key sets in one launch, as csa_forward runs the stage
+            csa.csa_compress_kv(d, self.packed, self.Y1, T, self.cu, self.cb, self.nseq, self.NB, self.Cc, self.KI)
         return {
             "A1_project_hidden": lambda: csa.csa_project_hidden(d, self.packed, self.H, T, self.Y1, self.wI),
             "A2_project_query": lambda: csa.csa_project_query(d, self.packed, col(4 * c + 4 * cI), N1b, T, self.Y2),

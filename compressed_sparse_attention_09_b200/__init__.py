@@ -10,5 +10,5 @@ from .capi import (CSA_BF16, CSA_F32, CsaError, Dims, csa_cache_append, csa_comp
                    csa_ring_row_elems, csa_sparse_mqa, lib, status_string,
                    csa_hidden_row_elems, csa_query_row_elems, csa_project_hidden, csa_project_query,
                    csa_launch_count, csa_indexer_workspace_bytes,
-                   csa_indexer_topk_noalloc)
+                   csa_indexer_topk_noalloc, csa_compress_kv)
 from .meta import cu_from_lengths  # noqa: F401

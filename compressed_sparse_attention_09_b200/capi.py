@@ -22,7 +22,7 @@ STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "C
 
 # every symbol include/csa.h declares
 EXPORTS = (
-    "csa_packed_weights_bytes", "csa_pack_weights", "csa_compress", "csa_indexer_topk",
+    "csa_packed_weights_bytes", "csa_pack_weights", "csa_compress", "csa_compress_kv", "csa_indexer_topk",
     "csa_sparse_mqa", "csa_forward_workspace_bytes", "csa_forward", "csa_ring_row_elems",
     "csa_cache_append", "csa_decode_workspace_bytes", "csa_decode", "csa_get_device_status",
     "csa_status_string", "csa_hidden_row_elems", "csa_query_row_elems", "csa_project_hidden",
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "csa_packed_weights_bytes": (sz, [D]),
             "csa_pack_weights": (i, [D, ctypes.POINTER(csa_weights), vp, sz, vp]),
             "csa_compress": (i, [D, vp, vp, vp, vp, i, vp, vp, i, vp, vp, i, i, i, vp, vp]),
+            "csa_compress_kv": (i, [D, vp, vp, i, vp, vp, i, i, vp, vp, vp]),
             "csa_indexer_topk": (i, [D, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp, vp, sz, vp]),
             "csa_indexer_workspace_bytes": (sz, [D, i, i, i]),
             "csa_indexer_topk_noalloc": (i, [D, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp, vp]),
@@ -154,6 +155,12 @@ def csa_compress(dims: Dims, Ca, Cb, Za, Zb, ld, Ba, Bb, width, cu_seqlens, cu_b
     _check(lib().csa_compress(_d(dims), _p(Ca), _p(Cb), _p(Za), _p(Zb), ld, _p(Ba), _p(Bb), width,
                               _p(cu_seqlens), _p(cu_blocks), nseq, total_tokens, total_blocks, _p(out),
                               _stream(stream)), "csa_compress")
+
+
+def csa_compress_kv(dims: Dims, packed, Y1, T, cu_seqlens, cu_blocks, nseq, total_blocks, Ccomp, KIcomp,
+                    stream=None):
+    _check(lib().csa_compress_kv(_d(dims), _p(packed), _p(Y1), T, _p(cu_seqlens), _p(cu_blocks), nseq,
+                                 total_blocks, _p(Ccomp), _p(KIcomp), _stream(stream)), "csa_compress_kv")
 
 
 def csa_indexer_workspace_bytes(dims: Dims, total_tokens: int, nseq: int, max_seqlen: int) -> int:

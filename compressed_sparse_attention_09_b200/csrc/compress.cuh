@@ -4,13 +4,15 @@
 // Z^b + B^b) weighting the matching C^a / C^b rows.
 //
 // The work is a pure stream: each C/Z element is read once and each entry
-// written once, so the kernel is HBM-bound.  One thread owns 4 channels of
-// one entry: its 4m row loads are 4-element vector loads (8 bytes for bf16,
-// 16 for fp32), coalesced across the warp (neighbouring threads own
-// neighbouring channels of the same rows), and the 2m-wide softmax and the
-// weighted sum run in fp32 registers.  Four channels per thread keep the
-// live registers low enough for many resident warps, which is what keeps
-// enough loads in flight to stream at HBM rate.
+// written once, so the kernel is HBM-bound.  One thread owns V consecutive
+// channels of one entry (V = 8 for bf16 with 16-byte rows, else 4): its 4m
+// row loads are V-element vector loads, coalesced across the warp
+// (neighbouring threads own neighbouring channels of the same rows), all
+// issued before any arithmetic, and the 2m-wide softmax and the weighted sum
+// run in fp32 registers.  One launch covers both entry widths (C^Comp and
+// K^IComp): the grid is the concatenation of each segment's blocks, and each
+// thread takes exactly one (entry, channel group), so no thread waits on a
+// second round of loads.
 #pragma once
 #include "common.cuh"
 
@@ -57,13 +59,13 @@ struct CompressSeg {
   const float* Bb;     // [m, width]
   int width;
   void* out;           // [total_blocks, width]
+  int groups;          // channel groups per entry: width / V
+  int blk0;            // first CTA of this segment in the grid
 };
 
 struct CompressArgs {
   CompressSeg seg[2];
   int nseg;
-  int vecs0;           // 4-channel groups per entry row of segment 0
-  int vecs_total;      // 4-channel groups per entry over all segments
   const int* cu_seqlens;
   const int* cu_blocks;
   int nseq;
@@ -71,93 +73,122 @@ struct CompressArgs {
   int total_blocks;
 };
 
-// 4 consecutive elements as fp32 (one 8-byte or 16-byte load)
-template <typename T> __device__ __forceinline__ void load4(const T* p, float* o);
-template <> __device__ __forceinline__ void load4<float>(const float* p, float* o) {
-  const float4 v = *reinterpret_cast<const float4*>(p);
-  o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
-}
-template <> __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float* o) {
-  const uint2 v = *reinterpret_cast<const uint2*>(p);
-  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
-  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
-  const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-  o[0] = fa.x; o[1] = fa.y; o[2] = fb.x; o[3] = fb.y;
-}
-template <typename T> __device__ __forceinline__ void store4(T* p, const float* v);
-template <> __device__ __forceinline__ void store4<float>(float* p, const float* v) {
-  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-}
-template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, const float* v) {
-  const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
-  const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+// V consecutive elements of T as one vector load (8 or 16 bytes)
+template <typename T, int V> struct RawVec;
+template <> struct RawVec<__nv_bfloat16, 8> {
+  uint4 u;
+  __device__ __forceinline__ float at(int e) const {
+    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+    return __bfloat162float(h[e]);
+  }
+};
+template <> struct RawVec<__nv_bfloat16, 4> {
   uint2 u;
-  u.x = *reinterpret_cast<const uint32_t*>(&a);
-  u.y = *reinterpret_cast<const uint32_t*>(&b);
-  *reinterpret_cast<uint2*>(p) = u;
+  __device__ __forceinline__ float at(int e) const {
+    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+    return __bfloat162float(h[e]);
+  }
+};
+template <> struct RawVec<float, 4> {
+  float4 u;
+  __device__ __forceinline__ float at(int e) const { return reinterpret_cast<const float*>(&u)[e]; }
+};
+
+template <typename T, int V>
+__device__ __forceinline__ RawVec<T, V> load_raw(const T* p) {
+  RawVec<T, V> r;
+  r.u = __ldcs(reinterpret_cast<const decltype(r.u)*>(p));   // streamed: read once
+  return r;
 }
 
-// grid-stride over (entry, 4-channel group) pairs of all segments
-template <typename T, int M>
+template <typename T, int V>
+__device__ __forceinline__ void store_raw(T* p, const float* v) {
+  if constexpr (sizeof(T) == 2 && V == 8) {
+    Vec16<__nv_bfloat16> o;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o.e[e] = __float2bfloat16_rn(v[e]);
+    *reinterpret_cast<uint4*>(p) = o.u;
+  } else if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&a);
+    u.y = *reinterpret_cast<const uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = u;
+  } else {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+// One thread per (segment, entry, channel group); see the header.
+template <typename T, int M, int V>
 __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
-  constexpr int V = 4;
-  const long long n_items = (long long)a.total_blocks * a.vecs_total;
-  for (long long it = (long long)blockIdx.x * blockDim.x + threadIdx.x; it < n_items;
-       it += (long long)gridDim.x * blockDim.x) {
-    const int g = (int)(it / a.vecs_total);
-    int v = (int)(it - (long long)g * a.vecs_total);
-    const int s = v < a.vecs0 ? 0 : 1;
-    if (s) v -= a.vecs0;
-    const CompressSeg& sg = a.seg[s];
-    // the sequence owning entry g
-    int lo = 0, hi = a.nseq;
-    while (hi - lo > 1) {
-      int mid = (lo + hi) >> 1;
-      if (a.cu_blocks[mid] <= g) lo = mid; else hi = mid;
-    }
-    const int i = g - a.cu_blocks[lo];
-    const long long tok = (long long)a.cu_seqlens[lo] + (long long)M * i;
-    if (i < 0 || tok + M > a.cu_seqlens[lo + 1] || tok + M > a.total_tokens) {
-      flag_status(kStatusMetadata);
-      continue;
-    }
-    const bool has_prev = i > 0;
-    const int col = v * V;
-    float la[M][V], lb[M][V], ca[M][V], cb[M][V];
+  const int s = (a.nseg > 1 && (int)blockIdx.x >= a.seg[1].blk0) ? 1 : 0;
+  const CompressSeg& sg = a.seg[s];
+  const int l = ((int)blockIdx.x - sg.blk0) * (int)blockDim.x + (int)threadIdx.x;
+  const int g = l / sg.groups;
+  if (g >= a.total_blocks) return;
+  const int col = (l - g * sg.groups) * V;
+  // the sequence owning entry g
+  int lo = 0, hi = a.nseq;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (a.cu_blocks[mid] <= g) lo = mid; else hi = mid;
+  }
+  const int i = g - a.cu_blocks[lo];
+  const int tok = a.cu_seqlens[lo] + M * i;
+  if (i < 0 || tok + M > a.cu_seqlens[lo + 1] || tok + M > a.total_tokens) {
+    flag_status(kStatusMetadata);
+    return;
+  }
+  const bool has_prev = i > 0;
+  const T* Za = static_cast<const T*>(sg.Za) + col;
+  const T* Ca = static_cast<const T*>(sg.Ca) + col;
+  const T* Zb = static_cast<const T*>(sg.Zb) + col;
+  const T* Cb = static_cast<const T*>(sg.Cb) + col;
+  RawVec<T, V> za[M], ca[M], zb[M], cb[M];
+#pragma unroll
+  for (int r = 0; r < M; ++r) {
+    const long long ra = (long long)(tok + r) * sg.ld;
+    za[r] = load_raw<T, V>(Za + ra);
+    ca[r] = load_raw<T, V>(Ca + ra);
+  }
+  if (has_prev) {
 #pragma unroll
     for (int r = 0; r < M; ++r) {
-      const long long ra = (tok + r) * sg.ld + col;
-      load4<T>(static_cast<const T*>(sg.Za) + ra, la[r]);
-      load4<T>(static_cast<const T*>(sg.Ca) + ra, ca[r]);
-      if (has_prev) {
-        const long long rb = (tok - M + r) * sg.ld + col;
-        load4<T>(static_cast<const T*>(sg.Zb) + rb, lb[r]);
-        load4<T>(static_cast<const T*>(sg.Cb) + rb, cb[r]);
-      }
+      const long long rb = (long long)(tok - M + r) * sg.ld;
+      zb[r] = load_raw<T, V>(Zb + rb);
+      cb[r] = load_raw<T, V>(Cb + rb);
     }
+  }
+  float res[V];
+#pragma unroll
+  for (int q = 0; q < V / 4; ++q) {
+    // position biases of these four channels, every row of both halves
+    float4 ba[M], bb[M];
 #pragma unroll
     for (int r = 0; r < M; ++r) {
-      const float4 ba = *reinterpret_cast<const float4*>(sg.Ba + (long long)r * sg.width + col);
-      la[r][0] += ba.x; la[r][1] += ba.y; la[r][2] += ba.z; la[r][3] += ba.w;
-      if (has_prev) {
-        const float4 bb = *reinterpret_cast<const float4*>(sg.Bb + (long long)r * sg.width + col);
-        lb[r][0] += bb.x; lb[r][1] += bb.y; lb[r][2] += bb.z; lb[r][3] += bb.w;
-      }
+      ba[r] = __ldg(reinterpret_cast<const float4*>(sg.Ba + r * sg.width + col + 4 * q));
+      bb[r] = has_prev ? __ldg(reinterpret_cast<const float4*>(sg.Bb + r * sg.width + col + 4 * q))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    float res[V];
 #pragma unroll
-    for (int e = 0; e < V; ++e) {
-      float l_a[M], l_b[M], c_a[M], c_b[M];
+    for (int e4 = 0; e4 < 4; ++e4) {
+      const int e = 4 * q + e4;
+      float la[M], lb[M], c_a[M], c_b[M];
 #pragma unroll
       for (int r = 0; r < M; ++r) {
-        l_a[r] = la[r][e]; c_a[r] = ca[r][e];
-        l_b[r] = has_prev ? lb[r][e] : 0.f;
-        c_b[r] = has_prev ? cb[r][e] : 0.f;
+        const float bav = reinterpret_cast<const float*>(&ba[r])[e4];
+        const float bbv = reinterpret_cast<const float*>(&bb[r])[e4];
+        la[r] = za[r].at(e) + bav;
+        c_a[r] = ca[r].at(e);
+        lb[r] = has_prev ? zb[r].at(e) + bbv : 0.f;
+        c_b[r] = has_prev ? cb[r].at(e) : 0.f;
       }
-      res[e] = compress_channel<M>(l_a, l_b, c_a, c_b, has_prev);
+      res[e] = compress_channel<M>(la, lb, c_a, c_b, has_prev);
     }
-    store4<T>(static_cast<T*>(sg.out) + (long long)g * sg.width + col, res);
   }
+  store_raw<T, V>(static_cast<T*>(sg.out) + (long long)g * sg.width + col, res);
 }
 
 // ---------------------------------------------------------------- decode append

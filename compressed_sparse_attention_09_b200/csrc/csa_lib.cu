@@ -224,22 +224,37 @@ csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const vo
   return CSA_OK;
 }
 
-template <typename T, int M>
-void compress_launch(const CompressArgs& a, long long items, cudaStream_t st) {
-  long long blocks = (items + 255) / 256;
-  const long long cap = (long long)sm_count() * 8;   // grid-stride beyond 8 CTAs per SM
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  compress_kernel<T, M><<<(unsigned)blocks, 256, 0, st>>>(a);
+template <typename T, int M, int V>
+void compress_launch(CompressArgs a, cudaStream_t st) {
+  // one thread per (entry, group of V channels); each segment's CTAs in turn
+  int blocks = 0;
+  for (int s = 0; s < a.nseg; ++s) {
+    a.seg[s].groups = a.seg[s].width / V;
+    a.seg[s].blk0 = blocks;
+    blocks += (int)(((long long)a.total_blocks * a.seg[s].groups + 255) / 256);
+  }
+  compress_kernel<T, M, V><<<(unsigned)blocks, 256, 0, st>>>(a);
+}
+
+// 16-byte channel groups for bf16 where every row and pointer allows them
+bool compress_wide_ok(const CompressArgs& a) {
+  for (int s = 0; s < a.nseg; ++s) {
+    const CompressSeg& g = a.seg[s];
+    if (g.width % 8 || g.ld % 8) return false;
+    for (const void* p : {g.Ca, g.Cb, g.Za, g.Zb, (const void*)g.out})
+      if (reinterpret_cast<uintptr_t>(p) % 16) return false;
+  }
+  return true;
 }
 
 csa_status launch_compress(const csa_dims* d, const CompressArgs& a, cudaStream_t st) {
-  const long long items = (long long)a.total_blocks * a.vecs_total;
-  if (items == 0) return CSA_OK;
-#define CSA_COMPRESS_CASE(MM)                                              \
-  case MM:                                                                 \
-    if (d->dtype == CSA_BF16) compress_launch<bf16, MM>(a, items, st);     \
-    else compress_launch<float, MM>(a, items, st);                         \
+  if ((long long)a.total_blocks * (a.seg[0].width + (a.nseg > 1 ? a.seg[1].width : 0)) == 0) return CSA_OK;
+  const bool wide = d->dtype == CSA_BF16 && compress_wide_ok(a);
+#define CSA_COMPRESS_CASE(MM)                                                         \
+  case MM:                                                                            \
+    if (d->dtype != CSA_BF16) compress_launch<float, MM, 4>(a, st);                   \
+    else if (wide) compress_launch<bf16, MM, 8>(a, st);                               \
+    else compress_launch<bf16, MM, 4>(a, st);                                         \
     break;
   switch (d->m) {
     CSA_COMPRESS_CASE(1)
@@ -394,6 +409,25 @@ CompressArgs make_compress_args(const csa_dims* d, const int* cu_seqlens, const 
   return a;
 }
 
+// A3 as the forward runs it: both key sets from the Y1 projection rows.
+csa_status compress_kv(const csa_dims* d, const void* packed, const void* Y1, int T, const int* cu_seqlens,
+                       const int* cu_blocks, int nseq, int NB, void* Cc, void* KIc, cudaStream_t st) {
+  const PackLayout P = pack_layout(d);
+  const size_t es = elem_size(d);
+  const int c = d->c, cI = d->cI;
+  const char* y1 = static_cast<const char*>(Y1);
+  CompressArgs ca = make_compress_args(d, cu_seqlens, cu_blocks, nseq, T, NB);
+  ca.seg[0] = {y1, y1 + (size_t)c * es, y1 + (size_t)2 * c * es, y1 + (size_t)3 * c * es, P.N1b,
+               reinterpret_cast<const float*>(at((void*)packed, P.ba)),
+               reinterpret_cast<const float*>(at((void*)packed, P.bb)), c, Cc, 0, 0};
+  const char* yI = y1 + (size_t)4 * c * es;
+  ca.seg[1] = {yI, yI + (size_t)cI * es, yI + (size_t)2 * cI * es, yI + (size_t)3 * cI * es, P.N1b,
+               reinterpret_cast<const float*>(at((void*)packed, P.baI)),
+               reinterpret_cast<const float*>(at((void*)packed, P.bbI)), cI, KIc, 0, 0};
+  ca.nseg = 2;
+  return launch_compress(d, ca, st);
+}
+
 }  // namespace
 
 // ====================================================================== ABI
@@ -533,11 +567,24 @@ csa_status csa_compress(const csa_dims* d, const void* Ca, const void* Cb, const
     if (reinterpret_cast<uintptr_t>(p) % va) return CSA_ERR_UNSUPPORTED;
   if (reinterpret_cast<uintptr_t>(Ba) % 16 || reinterpret_cast<uintptr_t>(Bb) % 16) return CSA_ERR_UNSUPPORTED;
   CompressArgs a = make_compress_args(d, cu_seqlens, cu_blocks, nseq, total_tokens, total_blocks);
-  a.seg[0] = {Ca, Cb, Za, Zb, ld, Ba, Bb, width, out};
+  a.seg[0] = {Ca, Cb, Za, Zb, ld, Ba, Bb, width, out, 0, 0};
   a.nseg = 1;
-  a.vecs0 = width / 4;
-  a.vecs_total = a.vecs0;
   return launch_compress(d, a, (cudaStream_t)stream);
+}
+
+csa_status csa_compress_kv(const csa_dims* d, const void* packed, const void* Y1, int T, const int* cu_seqlens,
+                           const int* cu_blocks, int nseq, int total_blocks, void* Ccomp, void* KIcomp,
+                           void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!packed || !Y1 || !cu_seqlens || !cu_blocks || !Ccomp || !KIcomp) return CSA_ERR_INVALID_ARG;
+  if (nseq <= 0 || T < 0 || total_blocks < 0 || total_blocks > T / d->m) return CSA_ERR_INVALID_ARG;
+  const uintptr_t va = 4 * elem_size(d);
+  for (const void* p : {Y1, (const void*)Ccomp, (const void*)KIcomp})
+    if (reinterpret_cast<uintptr_t>(p) % va) return CSA_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(packed) % kPtrAlign) return CSA_ERR_UNSUPPORTED;
+  return compress_kv(d, packed, Y1, T, cu_seqlens, cu_blocks, nseq, total_blocks, Ccomp, KIcomp,
+                     (cudaStream_t)stream);
 }
 
 size_t csa_indexer_workspace_bytes(const csa_dims* d, int total_tokens, int nseq, int max_seqlen) {
@@ -680,18 +727,7 @@ csa_status csa_forward(const csa_dims* d, const void* packed, const void* H, con
   s = project_query(d, packed, y1 + (size_t)(4 * c + 4 * cI) * es, P.N1b, T, y2, st);
   if (s != CSA_OK) return s;
   // A3: eqs. (3), (4) for C^Comp and K^IComp in one launch
-  CompressArgs ca = make_compress_args(d, cu_seqlens, cu_blocks, nseq, T, NB);
-  ca.seg[0] = {y1, y1 + (size_t)c * es, y1 + (size_t)2 * c * es, y1 + (size_t)3 * c * es, P.N1b,
-               reinterpret_cast<const float*>(at((void*)packed, P.ba)),
-               reinterpret_cast<const float*>(at((void*)packed, P.bb)), c, Cc};
-  char* yI = y1 + (size_t)4 * c * es;
-  ca.seg[1] = {yI, yI + (size_t)cI * es, yI + (size_t)2 * cI * es, yI + (size_t)3 * cI * es, P.N1b,
-               reinterpret_cast<const float*>(at((void*)packed, P.baI)),
-               reinterpret_cast<const float*>(at((void*)packed, P.bbI)), cI, KIc};
-  ca.nseg = 2;
-  ca.vecs0 = c / 4;
-  ca.vecs_total = (c + cI) / 4;
-  s = launch_compress(d, ca, st);
+  s = compress_kv(d, packed, y1, T, cu_seqlens, cu_blocks, nseq, NB, Cc, KIc, st);
   if (s != CSA_OK) return s;
   // A4: eqs. (8), (9)
   IndexerArgs ia;

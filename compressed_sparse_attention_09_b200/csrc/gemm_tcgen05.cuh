@@ -10,7 +10,9 @@
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M = 128,
 //               N = BN, K = 16) and commits stage releases / tile completions;
 //   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, conversion, and
-//               vectorised stores routed to the output segments.
+//               stores routed to the output segments: bf16 columns go through
+//               a per-warp shared-memory transpose and leave as whole 128-byte
+//               rows (four rows per warp store).
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap
 // the main loop of tile i+1.  Tiles are visited M-fastest so that the CTAs
 // running at one time share the same few B (weight) column blocks in L2.
@@ -35,8 +37,14 @@ struct TcGemmCfg {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;       // two accumulators
-  static constexpr size_t SMEM = 1024 /*align slack*/ + (size_t)kStages * STAGE_BYTES + 256 /*barriers*/;
+  static constexpr int OUT_STAGE = 4 * 32 * 128;  // epilogue staging: 32 rows x 128 B per epilogue warp
+  static constexpr size_t SMEM =
+      1024 /*align slack*/ + (size_t)kStages * STAGE_BYTES + OUT_STAGE + 256 /*barriers*/;
 };
+
+// byte offset of 16-byte piece u (0..7) of row r in 128-byte rows, XOR-swizzled
+// so that a warp writing one piece of 32 rows spreads over the banks
+__device__ __forceinline__ uint32_t r_sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
 template <typename T>
 __device__ __forceinline__ void store_chunk32(const GemmOut& o, long long row, int col0, int N, const float* v) {
@@ -64,8 +72,25 @@ __device__ __forceinline__ void store_chunk32(const GemmOut& o, long long row, i
       return;
     }
   }
+#pragma unroll
   for (int j = 0; j < 32; ++j)
     if (col0 + j < N) store_out<T>(o, row, col0 + j, v[j]);
+}
+
+// The bf16 segment that holds output columns [c0, c0 + 64) in full, with
+// 16-byte aligned rows there (or -1): those columns can leave through the
+// staged, coalesced path.
+__device__ __forceinline__ int staged_segment(const GemmOut& o, int c0, int N) {
+  if (c0 + 64 > N) return -1;
+#pragma unroll
+  for (int s = 0; s < kMaxSeg; ++s) {
+    if (s >= o.nseg) break;
+    const OutSeg& sg = o.seg[s];
+    if (sg.f32 || c0 < sg.col0 || c0 + 64 > sg.col0 + sg.ncols) continue;
+    const bool aligned = (reinterpret_cast<uintptr_t>(sg.ptr) % 16) == 0 && sg.ld % 8 == 0 && (c0 - sg.col0) % 8 == 0;
+    return aligned ? s : -1;
+  }
+  return -1;
 }
 
 template <int BN, int kStages>
@@ -77,7 +102,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* smA = smem;
   uint8_t* smB = smem + kStages * Cfg::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * Cfg::STAGE_BYTES);
+  uint8_t* smOut = smem + kStages * Cfg::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smOut + Cfg::OUT_STAGE);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -152,7 +178,13 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {  // ---------------- epilogue warps 2..5
+    // 64 columns per TMEM wait.  Where the 64 columns go to one bf16 segment,
+    // each thread converts its row into this warp's 32 staging rows (row =
+    // lane) and the warp writes them out as whole 128-byte rows, four rows
+    // per store instruction; other columns (fp32 w^I, ragged edges, the
+    // transposed decode form) are stored per thread.
     const int sub = warp & 3;   // TMEM lane quarter this warp may access
+    uint8_t* stage_out = smOut + (warp - 2) * (32 * 128);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
@@ -161,16 +193,67 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int r = mt * Cfg::BM + sub * 32 + lane;
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
-        float v[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN + ch * 32), v);
-        const int c0 = nt * BN + ch * 32;
-        if (!g.transpose_out) {
-          if (r < g.M && c0 < g.N) store_chunk32<__nv_bfloat16>(g.out, r, c0, g.N, v);
-        } else if (r < g.M) {
-          for (int j = 0; j < 32; ++j)
-            if (c0 + j < g.N) store_out<__nv_bfloat16>(g.out, c0 + j, r, v[j]);
+      for (int ch = 0; ch < BN / 64; ++ch) {
+        float v0[32], v1[32];
+        const uint32_t ta = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN + ch * 64);
+        tmem_ld_32x32b_x32_pair(ta, ta + 32u, v0, v1);
+        const int c0 = nt * BN + ch * 64;
+        if (g.transpose_out) {
+          // D[r][c0 + j] goes to output row c0 + j, column r: one segment
+          // per thread (its column), consecutive lanes write consecutive
+          // columns of the same output row
+          if (r < g.M) {
+            int sidx = -1;
+#pragma unroll
+            for (int s = 0; s < kMaxSeg; ++s)
+              if (s < g.out.nseg && r >= g.out.seg[s].col0 && r < g.out.seg[s].col0 + g.out.seg[s].ncols) sidx = s;
+            if (sidx >= 0) {
+              const OutSeg& sg = g.out.seg[sidx];
+              const long long col = r - sg.col0;
+              if (sg.f32) {
+                float* dst = static_cast<float*>(sg.ptr) + col;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  if (c0 + j < g.N) dst[(long long)(c0 + j) * sg.ld] = v0[j];
+                  if (c0 + 32 + j < g.N) dst[(long long)(c0 + 32 + j) * sg.ld] = v1[j];
+                }
+              } else {
+                __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(sg.ptr) + col;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  if (c0 + j < g.N) dst[(long long)(c0 + j) * sg.ld] = __float2bfloat16_rn(v0[j]);
+                  if (c0 + 32 + j < g.N) dst[(long long)(c0 + 32 + j) * sg.ld] = __float2bfloat16_rn(v1[j]);
+                }
+              }
+            }
+          }
+          continue;
         }
+        const int sidx = staged_segment(g.out, c0, g.N);
+        if (sidx < 0) {
+          if (r < g.M && c0 < g.N) store_chunk32<__nv_bfloat16>(g.out, r, c0, g.N, v0);
+          if (r < g.M && c0 + 32 < g.N) store_chunk32<__nv_bfloat16>(g.out, r, c0 + 32, g.N, v1);
+          continue;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float* vv = u < 4 ? v0 : v1;
+          Vec16<__nv_bfloat16> pk;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pk.e[e] = __float2bfloat16_rn(vv[8 * (u & 3) + e]);
+          *reinterpret_cast<uint4*>(stage_out + r_sw128(lane, u)) = pk.u;
+        }
+        __syncwarp();
+        const OutSeg& sg = g.out.seg[sidx];
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(sg.ptr) + (c0 - sg.col0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3), u = lane & 7;
+          const long long row = (long long)mt * Cfg::BM + sub * 32 + rr;
+          const uint4 val = *reinterpret_cast<const uint4*>(stage_out + r_sw128(rr, u));
+          if (row < g.M) *reinterpret_cast<uint4*>(dst + row * sg.ld + 8 * u) = val;
+        }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();

@@ -147,6 +147,20 @@ csa_status csa_compress(const csa_dims* dims, const void* Ca, const void* Cb, co
                         const int* cu_seqlens, const int* cu_blocks, int nseq, int total_tokens,
                         int total_blocks, void* out, void* stream);
 
+/* Compression of both key sets as the forward pass runs it, eqs. (3)-(4)
+ * and the indexer-key copy of the same operation: C^Comp [total_blocks, c]
+ * and K^IComp [total_blocks, cI] from the H-side projection rows, in one
+ * launch.
+ * Y1 [dev]     : [T, csa_hidden_row_elems] as csa_project_hidden writes it
+ *                (its C^a, C^b, Z^a, Z^b and indexer column blocks are read).
+ * packed [dev] : the packed weights (their fp32 position biases are read).
+ * Ccomp, KIcomp [dev] : outputs, row strides c and cI.
+ * Same entry rule as csa_compress; returns CSA_ERR_INVALID_ARG for null
+ * pointers or inconsistent sizes before any launch. */
+csa_status csa_compress_kv(const csa_dims* dims, const void* packed, const void* Y1, int T,
+                           const int* cu_seqlens, const int* cu_blocks, int nseq, int total_blocks,
+                           void* Ccomp, void* KIcomp, void* stream);
+
 /* Lightning indexer (eq. 8) and top-k selector (eq. 9), prefill.
  * qI [dev]  : [total_tokens, nhI*cI] (row stride ld_qI), heads concatenated.
  * wI [dev]  : [total_tokens, nhI] fp32 (row stride ld_wI).

@@ -109,6 +109,36 @@ def test_stage_compress(dtype, m):
     compare_dense(f64(out.cpu()), want, dtype, "compress")
 
 
+@pytest.mark.parametrize("dtype", [csa.CSA_F32, csa.CSA_BF16])
+def test_stage_compress_kv_from_projection_rows(dtype):
+    """csa_compress_kv (A3 as the forward runs it: both key sets, one launch)
+    on seeded projection rows laid out as csa_project_hidden writes them."""
+    dims = csa.Dims(d=64, c=128, m=4, cI=64, nhI=4, nh=2, dc=64, topk=4, dtype=dtype)
+    lens = [4 * 9 + 3, 2, 4, 4 * 33]
+    T = sum(lens)
+    W = synth.make_weights(dims, 41)
+    packed = gpu_pack(dims, W)
+    N1b = csa.csa_hidden_row_elems(dims)
+    Y = synth.make_normal((T, N1b), dims, 42)
+    cu, cb = csa.cu_from_lengths(lens, dims.m)
+    NB = int(cb[-1])
+    dt = Y.dtype
+    Cc = torch.empty(NB, dims.c, dtype=dt, device=DEV)
+    KI = torch.empty(NB, dims.cI, dtype=dt, device=DEV)
+    csa.csa_compress_kv(dims, packed, Y.to(DEV), T, cu.to(DEV), cb.to(DEV), len(lens), NB, Cc, KI)
+    assert csa.csa_get_device_status() == 0
+    Y64, c, cI = f64(Y), dims.c, dims.cI
+    for width, off, ba, bb, got, name in ((c, 0, "B_a", "B_b", Cc, "C_comp"),
+                                          (cI, 4 * c, "B_a_I", "B_b_I", KI, "K_icomp")):
+        want = []
+        for b in range(len(lens)):
+            s = slice(int(cu[b]), int(cu[b + 1]))
+            cols = [Y64[s, off + j * width:off + (j + 1) * width] for j in range(4)]
+            want.append(orc.compress(*cols, f64(W[ba]), f64(W[bb]), dims.m))
+        want = orc.storage_round(np.concatenate(want), store_mode(dims))
+        compare_dense(f64(got.cpu()), want, dtype, name)
+
+
 def _indexer_case(dims, lens, seed, zero_w=False):
     T = sum(lens)
     cu, cb = csa.cu_from_lengths(lens, dims.m)
