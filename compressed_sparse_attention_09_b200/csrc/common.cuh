@@ -59,6 +59,14 @@ __device__ __forceinline__ void store_vec_f32(T* p, const float* in) {
   *reinterpret_cast<uint4*>(p) = v.u;
 }
 
+// 2^x by the hardware approximation (ex2.approx.ftz.f32: relative error of
+// about 2^-22, 2^-inf = +0).
+__device__ __forceinline__ float ex2_approx_f32(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Map an fp32 score to an unsigned key whose unsigned order is the float
 // order (-0 is folded onto +0 first so that equal scores get equal keys).
 __device__ __forceinline__ uint32_t ordered_key(float f) {

@@ -4,9 +4,10 @@
 // Z^b + B^b) weighting the matching C^a / C^b rows.
 //
 // The work is a pure stream: each C/Z element is read once and each entry
-// written once, so the kernel is HBM-bound.  One thread owns V consecutive
-// channels of one entry (V = 8 for bf16 with 16-byte rows, else 4): its 4m
-// row loads are V-element vector loads, coalesced across the warp
+// written once, so the kernel is HBM-bound.  One thread owns 4 consecutive
+// channels of one entry (8-byte loads for bf16, 16-byte for fp32: more
+// resident threads measured faster than 16-byte bf16 groups): its 4m row
+// loads are 4-element vector loads, coalesced across the warp
 // (neighbouring threads own neighbouring channels of the same rows), all
 // issued before any arithmetic, and the 2m-wide softmax and the weighted sum
 // run in fp32 registers.  One launch covers both entry widths (C^Comp and
@@ -20,33 +21,43 @@ namespace csa {
 
 // One compressed channel value.  la/lb: the m logits of the block and of the
 // block before (already biased); ca/cb: the matching C^a / C^b values.
-// has_prev = false is the i = 0 padding (Z^b = -inf, C^b = 0).
+// has_prev = false is the i = 0 padding (Z^b = -inf, C^b = 0).  The softmax
+// runs in base 2 (logits scaled by log2 e once, exponentials by the hardware
+// 2^x), and the weighted sum is divided by the normaliser (in [1, 2m]) with
+// the fast approximate division.
 template <int M>
 __device__ __forceinline__ float compress_channel(const float* la, const float* lb, const float* ca,
                                                   const float* cb, bool has_prev) {
-  float mx = la[0];
+  constexpr float kLog2e = 1.4426950408889634f;
+  float a2[M], b2[M];
 #pragma unroll
-  for (int r = 1; r < M; ++r) mx = fmaxf(mx, la[r]);
+  for (int r = 0; r < M; ++r) {
+    a2[r] = la[r] * kLog2e;
+    b2[r] = lb[r] * kLog2e;
+  }
+  float mx = a2[0];
+#pragma unroll
+  for (int r = 1; r < M; ++r) mx = fmaxf(mx, a2[r]);
   if (has_prev) {
 #pragma unroll
-    for (int r = 0; r < M; ++r) mx = fmaxf(mx, lb[r]);
+    for (int r = 0; r < M; ++r) mx = fmaxf(mx, b2[r]);
   }
   float den = 0.f, num = 0.f;
 #pragma unroll
   for (int r = 0; r < M; ++r) {
-    float e = expf(la[r] - mx);
+    const float e = ex2_approx_f32(a2[r] - mx);
     den += e;
     num = fmaf(e, ca[r], num);
   }
   if (has_prev) {
 #pragma unroll
     for (int r = 0; r < M; ++r) {
-      float e = expf(lb[r] - mx);
+      const float e = ex2_approx_f32(b2[r] - mx);
       den += e;
       num = fmaf(e, cb[r], num);
     }
   }
-  return num / den;
+  return __fdividef(num, den);
 }
 
 struct CompressSeg {
@@ -73,20 +84,16 @@ struct CompressArgs {
   int total_blocks;
 };
 
-// V consecutive elements of T as one vector load (8 or 16 bytes)
+// V = 4 consecutive elements of T as one vector load (8 or 16 bytes)
 template <typename T, int V> struct RawVec;
-template <> struct RawVec<__nv_bfloat16, 8> {
-  uint4 u;
-  __device__ __forceinline__ float at(int e) const {
-    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
-    return __bfloat162float(h[e]);
-  }
-};
+// a bf16 is the upper half of the fp32 with the same value
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 template <> struct RawVec<__nv_bfloat16, 4> {
   uint2 u;
   __device__ __forceinline__ float at(int e) const {
-    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
-    return __bfloat162float(h[e]);
+    const uint32_t w = e < 2 ? u.x : u.y;
+    return (e & 1) ? bf16_hi(w) : bf16_lo(w);
   }
 };
 template <> struct RawVec<float, 4> {
@@ -103,12 +110,7 @@ __device__ __forceinline__ RawVec<T, V> load_raw(const T* p) {
 
 template <typename T, int V>
 __device__ __forceinline__ void store_raw(T* p, const float* v) {
-  if constexpr (sizeof(T) == 2 && V == 8) {
-    Vec16<__nv_bfloat16> o;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) o.e[e] = __float2bfloat16_rn(v[e]);
-    *reinterpret_cast<uint4*>(p) = o.u;
-  } else if constexpr (sizeof(T) == 2) {
+  if constexpr (sizeof(T) == 2) {
     const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
     const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
     uint2 u;

@@ -236,24 +236,11 @@ void compress_launch(CompressArgs a, cudaStream_t st) {
   compress_kernel<T, M, V><<<(unsigned)blocks, 256, 0, st>>>(a);
 }
 
-// 16-byte channel groups for bf16 where every row and pointer allows them
-bool compress_wide_ok(const CompressArgs& a) {
-  for (int s = 0; s < a.nseg; ++s) {
-    const CompressSeg& g = a.seg[s];
-    if (g.width % 8 || g.ld % 8) return false;
-    for (const void* p : {g.Ca, g.Cb, g.Za, g.Zb, (const void*)g.out})
-      if (reinterpret_cast<uintptr_t>(p) % 16) return false;
-  }
-  return true;
-}
-
 csa_status launch_compress(const csa_dims* d, const CompressArgs& a, cudaStream_t st) {
   if ((long long)a.total_blocks * (a.seg[0].width + (a.nseg > 1 ? a.seg[1].width : 0)) == 0) return CSA_OK;
-  const bool wide = d->dtype == CSA_BF16 && compress_wide_ok(a);
 #define CSA_COMPRESS_CASE(MM)                                                         \
   case MM:                                                                            \
     if (d->dtype != CSA_BF16) compress_launch<float, MM, 4>(a, st);                   \
-    else if (wide) compress_launch<bf16, MM, 8>(a, st);                               \
     else compress_launch<bf16, MM, 4>(a, st);                                         \
     break;
   switch (d->m) {
