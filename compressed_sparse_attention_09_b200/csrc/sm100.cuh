@@ -32,27 +32,42 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Number of try_wait polls before a wait gives up (each poll may itself
-// suspend briefly): a bounded wait of the order of a second.
-constexpr uint32_t kWaitLimit = 1u << 22;
+// Bounded waits.  Each poll is a try_wait with a suspend-time hint, so a
+// waiting thread sleeps in hardware until the phase completes (or the hint
+// runs out) instead of spinning and taking issue slots from the working
+// warps of its SM sub-partition.  A wait gives up after kWaitNs of global
+// time (read from %globaltimer), i.e. of the order of a second.
+constexpr uint32_t kSuspendHintNs = 1000000;        // 1 ms per poll at most
+constexpr uint64_t kWaitNs = 1500000000ull;         // 1.5 s per wait at most
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
 
 // Waits for the phase of parity `parity` to complete.  Returns false (and
-// records kStatusTimeout) if it did not complete within kWaitLimit polls.
+// records kStatusTimeout) if it did not complete within kWaitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t addr = smem_u32(bar);
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; ++i) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(addr), "r"(parity)
+        : "r"(addr), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     if (done) return true;
+    if (i == 0) {
+      t0 = global_ns();
+    } else if (global_ns() - t0 > kWaitNs) {
+      flag_status(kStatusTimeout);
+      return false;
+    }
   }
-  flag_status(kStatusTimeout);
-  return false;
 }
 
 // Warp-uniform bounded wait: every lane polls, and the warp proceeds only if
