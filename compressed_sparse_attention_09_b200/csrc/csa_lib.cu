@@ -6,6 +6,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 
 #include "../../include/csa.h"
@@ -201,12 +202,24 @@ csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const vo
     TcGemmArgs g;
     g.K = K;
     g.out = out;
-    if (M >= 128) {  // activations as the M operand, 128 x 256 tiles
+    if (M >= 128) {  // activations as the M operand, 128 x BN tiles
+      // BN = 192 where it fills the last wave and the padded columns better
+      // (the packed weights are padded to 256 rows, so both widths stay in range)
+      auto wave_eff = [&](int bn) {
+        const long long nt = (N + bn - 1) / bn, tiles = nt * ((M + 127) / 128), sms = sm_count();
+        return (double)N / (double)(nt * bn) * (double)tiles / (double)(((tiles + sms - 1) / sms) * sms);
+      };
+      const int BN = wave_eff(192) > 1.03 * wave_eff(256) ? 192 : 256;
       const uint64_t nrows_b = (uint64_t)round_up_int(N, 256);
-      if (!make_tmap_bf16(&ta, A, K, M, lda * 2, 64, 128) || !make_tmap_bf16(&tb, B, K, nrows_b, ldb * 2, 64, 256))
+      if (!make_tmap_bf16(&ta, A, K, M, lda * 2, 64, 128) || !make_tmap_bf16(&tb, B, K, nrows_b, ldb * 2, 64, BN))
         return CSA_ERR_UNSUPPORTED;
       g.M = M; g.N = N; g.transpose_out = 0;
-      return launch_tc_gemm<256, 4>(ta, tb, g, st);
+      // A too large to stay in L2 across the column bands: visit groups of
+      // row tiles (about one wave each) so that B stays in L2 instead
+      const int m_tiles = (M + 127) / 128, n_tiles = (N + BN - 1) / BN;
+      g.group_m = (size_t)M * K * 2 > ((size_t)32 << 20) ? std::max(1, (sm_count() + n_tiles - 1) / n_tiles) : m_tiles;
+      if (g.group_m > m_tiles) g.group_m = m_tiles;
+      return BN == 192 ? launch_tc_gemm<192, 4>(ta, tb, g, st) : launch_tc_gemm<256, 4>(ta, tb, g, st);
     }
     // few rows (decode): swap A and B so the weights fill the 128-row MMA
     // operand and the tokens are the N = 64 operand; the epilogue transposes.
@@ -214,6 +227,7 @@ csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const vo
     if (!make_tmap_bf16(&ta, B, K, nrows_w, ldb * 2, 64, 128) || !make_tmap_bf16(&tb, A, K, M, lda * 2, 64, 64))
       return CSA_ERR_UNSUPPORTED;
     g.M = N; g.N = M; g.transpose_out = 1;
+    g.group_m = (N + 127) / 128;
     if (M <= 64) return launch_tc_gemm<64, 8>(ta, tb, g, st);
     return CSA_ERR_UNSUPPORTED;
   }

@@ -28,7 +28,22 @@ struct TcGemmArgs {
   int M, N, K;
   GemmOut out;
   int transpose_out;   // 1: D[i][j] is stored at output row j, column i (swap-AB use)
+  int group_m;         // tile order: groups of group_m row tiles, each group's tiles column by column
 };
+
+// Tile `tile` of the visiting order -> (row tile, column tile).  Within a
+// group of group_m row tiles the row tile runs fastest, so the CTAs running
+// at one time share a few column blocks of B; with group_m = m_tiles this is
+// plain row-fastest order.  Smaller groups keep the A rows of a group and
+// all of B resident in L2 when A is too large to stay there.
+__device__ __forceinline__ void gemm_tile_coords(int tile, int m_tiles, int n_tiles, int group_m, int& mt, int& nt) {
+  const int per_group = group_m * n_tiles;
+  const int grp = tile / per_group;
+  const int r = tile - grp * per_group;
+  const int gm = min(group_m, m_tiles - grp * group_m);
+  mt = grp * group_m + r % gm;
+  nt = r / gm;
+}
 
 template <int BN, int kStages>
 struct TcGemmCfg {
@@ -36,7 +51,7 @@ struct TcGemmCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN;       // two accumulators
+  static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;   // two accumulators (power of two)
   static constexpr int OUT_STAGE = 4 * 32 * 128;  // epilogue staging: 32 rows x 128 B per epilogue warp
   static constexpr size_t SMEM =
       1024 /*align slack*/ + (size_t)kStages * STAGE_BYTES + OUT_STAGE + 256 /*barriers*/;
@@ -141,7 +156,8 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-        const int mt = tile % m_tiles, nt = tile / m_tiles;
+        int mt, nt;
+        gemm_tile_coords(tile, m_tiles, n_tiles, g.group_m, mt, nt);
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
           mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
@@ -188,7 +204,8 @@ __global__ void __launch_bounds__(192, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
-      const int mt = tile % m_tiles, nt = tile / m_tiles;
+      int mt, nt;
+      gemm_tile_coords(tile, m_tiles, n_tiles, g.group_m, mt, nt);
       if (!mbar_wait(&tfull[acc], acc_phase)) { *abort_flag = 1; break; }
       tc_fence_after();
       const int r = mt * Cfg::BM + sub * 32 + lane;
