@@ -177,15 +177,24 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
         }
       }
       ++qw;
+      // slots of this thread's rows, one tile ahead: the index loads of tile
+      // j + 1 are in flight while tile j waits for its stage
+      int sn[kTile / 4];
+#pragma unroll
+      for (int i = 0; i < kTile / 4; ++i) {
+        const int e = r0 + 4 * i;
+        sn[i] = e < a.topk ? __ldg(ir + e) : -1;
+      }
       for (int j = 0; j < ntiles; ++j, ++g) {
         const int st = (int)(g % kStages);
-        if (!warp_wait(&t_done[st], ((g / kStages) & 1) ^ 1)) { ok = false; break; }
         int s[kTile / 4];
 #pragma unroll
         for (int i = 0; i < kTile / 4; ++i) {
-          const int e = j * kTile + r0 + 4 * i;
-          s[i] = e < a.topk ? ir[e] : -1;
+          s[i] = sn[i];
+          const int e = (j + 1) * kTile + r0 + 4 * i;
+          sn[i] = (j + 1 < ntiles && e < a.topk) ? __ldg(ir + e) : -1;
         }
+        if (!warp_wait(&t_done[st], ((g / kStages) & 1) ^ 1)) { ok = false; break; }
         uint8_t* cst = c_s + st * kCBytes + (c16 >> 3) * kCChunk;
 #pragma unroll
         for (int i = 0; i < kTile / 4; ++i) {
