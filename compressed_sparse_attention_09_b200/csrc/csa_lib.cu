@@ -824,12 +824,10 @@ csa_status launch_indexer_decode_tc(const csa_dims* d, const IndexerArgs& a, int
   const int grid = items < sm_count() ? (int)items : sm_count();
   indexer_decode_tc_kernel<<<grid, idxdec::kThreads, idxdec::kSmem, st>>>(tk, tq, t);
   CSA_CHECK_LAUNCH();
-  const size_t smem = (size_t)cap * 4 + 256 * 4 + 40 * 4;
-  if (smem > kMaxSmem) return CSA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+  if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsel::kSmem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
-  decode_select_kernel<<<B, 512, smem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
+  decode_select_kernel<<<B, 512, dsel::kSmem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }

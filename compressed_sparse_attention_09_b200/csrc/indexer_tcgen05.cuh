@@ -626,26 +626,161 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
   }
 }
 
-// Exact top-k of each decode row's score row (one CTA per sequence; the row
-// is staged in shared memory).
+// Exact top-k of each decode row's score row, one CTA of 16 warps per
+// sequence, same selection rule as warp_topk_ascending (the k largest
+// scores, equal scores lowest index first, ascending indices).  Radix select
+// on the order-preserving keys in three passes of 11, 11 and 10 bits; every
+// warp builds its own histogram of its share of the row (so increments only
+// collide within a warp), the 16 are summed, and warp 0 picks the digit.
+// The ordered output splits the row into 16 contiguous segments: a counting
+// pass, a prefix over the warps, and a writing pass.  The row is read from
+// global memory (L2) on every pass; shared memory holds only histograms.
+namespace dsel {
+constexpr int kWarps = 16, kBins = 2048;
+constexpr size_t kSmem = (size_t)(kWarps + 1) * kBins * 4 + 64 * 4;
+}  // namespace dsel
+
+// Warp 0: the digit of the combined histogram hist[0..NB) holding the kk-th
+// largest key, the count above it and the count in it (to ws[0..2]).
+template <int NB>
+__device__ __forceinline__ void dsel_pick(const int* hist, int kk, int* ws) {
+  constexpr int PER = NB / 32, SUB = PER / 32 > 0 ? PER / 32 : 1;
+  constexpr unsigned kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  int tot = 0;
+#pragma unroll 8
+  for (int j = 0; j < PER; ++j) tot += hist[NB - 1 - (PER * lane + ((j + lane) & (PER - 1)))];
+  int incl = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(kFull, incl, off);
+    if (lane >= off) incl += v;
+  }
+  const int excl = incl - tot;
+  const int src = __ffs(__ballot_sync(kFull, excl < kk && incl >= kk)) - 1;
+  const int excl_src = __shfl_sync(kFull, excl, src);
+  const int kk2 = kk - excl_src;
+  const int p0 = PER * src + SUB * lane;
+  int c2 = 0;
+  for (int u = 0; u < SUB; ++u) c2 += hist[NB - 1 - (p0 + u)];
+  int incl2 = c2;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(kFull, incl2, off);
+    if (lane >= off) incl2 += v;
+  }
+  const int excl2 = incl2 - c2;
+  const int src2 = __ffs(__ballot_sync(kFull, excl2 < kk2 && incl2 >= kk2)) - 1;
+  if (lane == src2) {
+    int c = excl2;
+    for (int u = 0; u < SUB; ++u) {
+      const int v = hist[NB - 1 - (p0 + u)];
+      if (c + v >= kk2) {
+        ws[0] = NB - 1 - (p0 + u);
+        ws[1] = excl_src + c;
+        ws[2] = v;
+        break;
+      }
+      c += v;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch, const int* pos, int cap, int m,
                                                             int topk, int* idx) {
-  extern __shared__ __align__(16) float sc_s[];   // [cap] then hist[256], ws[40]
-  unsigned* hist = reinterpret_cast<unsigned*>(sc_s + cap);
-  int* ws = reinterpret_cast<int*>(hist + 256);
+  using namespace dsel;
+  constexpr unsigned kFull = 0xffffffffu;
+  extern __shared__ __align__(16) int dsm[];
+  int* whist = dsm;                         // [kWarps][kBins] per-warp histograms
+  int* hist = dsm + kWarps * kBins;         // [kBins] combined
+  int* ws = hist + kBins;                   // [64] scratch words
   const int b = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = pos[b];
   int avail = t >= 0 ? t / m : 0;
   if (avail > cap) avail = cap;
   int* out = idx + (long long)b * topk;
   if (avail <= topk) {
-    for (int j = threadIdx.x; j < topk; j += blockDim.x) out[j] = j < avail ? j : -1;
+    for (int j = tid; j < topk; j += blockDim.x) out[j] = j < avail ? j : -1;
     return;
   }
   const float* row = scratch + (long long)b * cap;
-  for (int s = threadIdx.x; s < avail; s += blockDim.x) sc_s[s] = __ldcg(row + s);
+  int* myh = whist + warp * kBins;
+  uint32_t prefix = 0, mask = 0;
+  int kk = topk;
+#pragma unroll 1
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 21 : pass == 1 ? 10 : 0;
+    const int width = pass == 2 ? 10 : 11;
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int i = lane; i < kBins / 4; i += 32) reinterpret_cast<int4*>(myh)[i] = make_int4(0, 0, 0, 0);
+    __syncthreads();
+    // this thread's scores: 4 consecutive per step, the CTA covering 2048 per step
+    for (int i0 = 4 * tid; i0 < avail; i0 += 4 * 512) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u;
+        if (i < avail) {
+          const uint32_t key = ordered_key(__ldcg(row + i));
+          if ((key & mask) == prefix) atomicAdd(&myh[(key >> shift) & dmask], 1);
+        }
+      }
+    }
+    __syncthreads();
+    for (int bin = tid; bin < kBins; bin += 512) {
+      int c = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) c += whist[w * kBins + bin];
+      hist[bin] = c;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      if (width == 11) dsel_pick<2048>(hist, kk, ws);
+      else dsel_pick<1024>(hist, kk, ws);
+    }
+    __syncthreads();
+    prefix |= (uint32_t)ws[0] << shift;
+    mask |= dmask << shift;
+    kk -= ws[1];
+    __syncthreads();
+  }
+  const uint32_t thr = prefix;
+  const int need_eq = kk;
+  // ordered output over 16 contiguous segments
+  const int seg = (((avail + kWarps - 1) / kWarps) + 31) & ~31;
+  const int s0 = min(avail, warp * seg), s1 = min(avail, s0 + seg);
+  int n_gt = 0, n_eq = 0;
+  for (int base = s0; base < s1; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < s1 ? ordered_key(__ldcg(row + i)) : 0u;
+    n_gt += __popc(__ballot_sync(kFull, i < s1 && key > thr));
+    n_eq += __popc(__ballot_sync(kFull, i < s1 && key == thr));
+  }
+  if (lane == 0) {
+    ws[8 + warp] = n_gt;
+    ws[8 + kWarps + warp] = n_eq;
+  }
   __syncthreads();
-  cta_topk_ascending(sc_s, avail, topk, out, hist, ws);
+  int gt_before = 0, eq_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    gt_before += ws[8 + w];
+    eq_before += ws[8 + kWarps + w];
+  }
+  int out_off = gt_before + min(eq_before, need_eq), eq_seen = eq_before;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = s0; base < s1; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < s1 ? ordered_key(__ldcg(row + i)) : 0u;
+    const bool gt = i < s1 && key > thr;
+    const bool eq = i < s1 && key == thr;
+    const unsigned beq = __ballot_sync(kFull, eq);
+    const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
+    const unsigned btk = __ballot_sync(kFull, take);
+    const int p = out_off + __popc(btk & lt);
+    if (take && p < topk) out[p] = i;
+    out_off += __popc(btk);
+    eq_seen += __popc(beq);
+  }
 }
 
 }  // namespace csa
