@@ -402,11 +402,12 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
         if (!warp_wait(&t_full[acc], (acc_it >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const int s = j * kM + 32 * sub + lane;
-        // eight independent partial sums per query keep the FMA chains short
+        // four independent packed (fp32x2) partial sums per query keep the
+        // FMA chains short and fold two heads per FMA instruction
         for (int q = 0; q < nq; ++q) {
-          float p[8];
+          float2 p[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) p[e] = 0.f;
+          for (int e = 0; e < 4; ++e) p[e] = make_float2(0.f, 0.f);
 #pragma unroll 1
           for (int hc = 0; hc < NHI; hc += 32) {
             float v[32];
@@ -415,13 +416,15 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float4 w = w4[e];
-              p[(4 * e + 0) & 7] = fmaf(w.x, fmaxf(v[4 * e + 0], 0.f), p[(4 * e + 0) & 7]);
-              p[(4 * e + 1) & 7] = fmaf(w.y, fmaxf(v[4 * e + 1], 0.f), p[(4 * e + 1) & 7]);
-              p[(4 * e + 2) & 7] = fmaf(w.z, fmaxf(v[4 * e + 2], 0.f), p[(4 * e + 2) & 7]);
-              p[(4 * e + 3) & 7] = fmaf(w.w, fmaxf(v[4 * e + 3], 0.f), p[(4 * e + 3) & 7]);
+              p[(2 * e) & 3] = __ffma2_rn(make_float2(w.x, w.y),
+                                          make_float2(fmaxf(v[4 * e + 0], 0.f), fmaxf(v[4 * e + 1], 0.f)),
+                                          p[(2 * e) & 3]);
+              p[(2 * e + 1) & 3] = __ffma2_rn(make_float2(w.z, w.w),
+                                              make_float2(fmaxf(v[4 * e + 2], 0.f), fmaxf(v[4 * e + 3], 0.f)),
+                                              p[(2 * e + 1) & 3]);
             }
           }
-          const float sc = ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+          const float sc = ((p[0].x + p[0].y) + (p[1].x + p[1].y)) + ((p[2].x + p[2].y) + (p[3].x + p[3].y));
           if (s < avail) __stcg(scr + (size_t)q * a.sc_cap + s, sc);
         }
         tc_fence_before();
