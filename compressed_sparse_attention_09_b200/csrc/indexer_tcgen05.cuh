@@ -6,7 +6,8 @@
 // 128-block tile the MMA computes
 //     D[s, (q, h)] = K^IComp_s . q^I_{t_q, h}      M = 128 blocks, N = 4 x n_h^I, K = c^I
 // into one of two TMEM accumulators, and the epilogue warps (one TMEM lane =
-// one block s per thread) fold it straight into the index score
+// one block s per thread) fold it straight into the index score (stored as
+// its order-preserving 32-bit key)
 //     I[t_q, s] = sum_h w_{t_q, h} ReLU(D[s, (q, h)])
 // so the per-head products never leave the SM.  The four score rows of the
 // item go to one of two per-CTA scratch buffers (written and read back
@@ -83,8 +84,12 @@ __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, 
   return nq > 0;
 }
 
-// Exact top-k of sc[0..n) (n > k) by one warp, written to out[0..k) as
-// ascending indices; equal scores are taken lowest index first.
+// Exact top-k of a score row by one warp, written to out[0..k) as ascending
+// indices; equal scores are taken lowest index first.  The row sc[0..n)
+// holds the scores' order-preserving 32-bit keys (ordered_key), written by
+// the epilogue in place of the floats, so no pass converts them again (the
+// rows are handled as 32-bit words: float-typed pointers only for the
+// 16-byte copies).
 //
 // Radix select on the order-preserving 32-bit keys, most significant digit
 // first, in three passes of 11, 11 and 10 bits: each pass histograms the
@@ -145,11 +150,11 @@ __device__ __noinline__ uint32_t warp_radix_pass(const float* sc, int n, bool re
     const int nv = (cn + 3) >> 2;
 #pragma unroll 2
     for (int i = lane; i < nv; i += 32) {
-      const float4 v = reinterpret_cast<const float4*>(buf)[i];
-      const float e[4] = {v.x, v.y, v.z, v.w};
+      const uint4 v = reinterpret_cast<const uint4*>(buf)[i];
+      const uint32_t e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const uint32_t key = ordered_key(e[u]);
+        const uint32_t key = e[u];
         if (4 * i + u < cn && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint32_t)(NB - 1)], 1);
       }
     }
@@ -227,7 +232,7 @@ __device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, 
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int s = base + 32 * u + lane;
-        key[u] = s < cn ? ordered_key(buf[s]) : 0u;
+        key[u] = s < cn ? __float_as_uint(buf[s]) : 0u;
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -425,7 +430,7 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
             }
           }
           const float sc = ((p[0].x + p[0].y) + (p[1].x + p[1].y)) + ((p[2].x + p[2].y) + (p[3].x + p[3].y));
-          if (s < avail) __stcg(scr + (size_t)q * a.sc_cap + s, sc);
+          if (s < avail) __stcg(reinterpret_cast<unsigned*>(scr) + (size_t)q * a.sc_cap + s, ordered_key(sc));
         }
         tc_fence_before();
         __syncwarp();
