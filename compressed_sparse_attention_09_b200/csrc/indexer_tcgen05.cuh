@@ -132,10 +132,13 @@ __device__ __forceinline__ void warp_stage_chunk(const float* src, int n, float*
 // One radix pass over the keys k of sc[0..n) with (k & mask) == prefix:
 // returns the WIDTH-bit digit at `shift` that holds the kk-th largest of
 // them (kk >= 1, at most their number) and, in *above, how many of them have
-// a larger digit.  hist holds 2^WIDTH ints of shared memory.
-template <int WIDTH>
+// a larger digit, and in *in_bin how many have the returned digit.  hist
+// holds 2^WIDTH ints of shared memory.  FIRST: the first pass (mask = 0:
+// every key takes part).
+template <int WIDTH, bool FIRST>
 __device__ __noinline__ uint32_t warp_radix_pass(const float* sc, int n, bool resident, float* buf, int* hist,
-                                                 int shift, uint32_t mask, uint32_t prefix, int kk, int* above) {
+                                                 int shift, uint32_t mask, uint32_t prefix, int kk, int* above,
+                                                 int* in_bin) {
   constexpr int NB = 1 << WIDTH, PER = NB / 32, SUB = PER / 32;
   constexpr unsigned kFull = 0xffffffffu;
   const int lane = threadIdx.x & 31;
@@ -145,18 +148,19 @@ __device__ __noinline__ uint32_t warp_radix_pass(const float* sc, int n, bool re
   for (int c0 = 0; c0 < n; c0 += idxtc::kSelChunk) {
     const int cn = min(idxtc::kSelChunk, n - c0);
     if (!resident) warp_stage_chunk(sc + c0, cn, buf);
-    // buf holds kSelChunk floats, a multiple of 4: the last vector may run
-    // past cn but not past the buffer; its extra elements are masked
-    const int nv = (cn + 3) >> 2;
+    // whole 16-byte vectors first, then the last cn % 4 keys one per lane
+    const int nv = cn >> 2;
 #pragma unroll 2
     for (int i = lane; i < nv; i += 32) {
       const uint4 v = reinterpret_cast<const uint4*>(buf)[i];
       const uint32_t e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t key = e[u];
-        if (4 * i + u < cn && (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint32_t)(NB - 1)], 1);
-      }
+      for (int u = 0; u < 4; ++u)
+        if (FIRST || (e[u] & mask) == prefix) atomicAdd(&hist[(e[u] >> shift) & (uint32_t)(NB - 1)], 1);
+    }
+    if (lane < cn - 4 * nv) {
+      const uint32_t key = __float_as_uint(buf[4 * nv + lane]);
+      if (FIRST || (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint32_t)(NB - 1)], 1);
     }
     __syncwarp();
   }
@@ -189,20 +193,22 @@ __device__ __noinline__ uint32_t warp_radix_pass(const float* sc, int n, bool re
   }
   const int excl2 = incl2 - c2;
   const int src2 = __ffs(__ballot_sync(kFull, excl2 < kk2 && incl2 >= kk2)) - 1;
-  int pos = 0, before = 0;
+  int pos = 0, before = 0, cnt = 0;
   if (lane == src2) {
     int c = excl2;
 #pragma unroll
     for (int u = 0; u < SUB; ++u) {
       const int v = hist[NB - 1 - (p0 + u)];
-      if (c + v >= kk2) { pos = p0 + u; before = c; break; }
+      if (c + v >= kk2) { pos = p0 + u; before = c; cnt = v; break; }
       c += v;
     }
   }
   pos = __shfl_sync(kFull, pos, src2);
   before = __shfl_sync(kFull, before, src2);
+  cnt = __shfl_sync(kFull, cnt, src2);
   __syncwarp();
   *above = excl_src + before;
+  *in_bin = cnt;
   return (uint32_t)(NB - 1 - pos);
 }
 
@@ -211,15 +217,19 @@ __device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, 
   const int lane = threadIdx.x & 31;
   const bool resident = n <= idxtc::kSelChunk;
   if (resident) warp_stage_chunk(sc, n, buf);
-  int kk = k, above;
-  uint32_t prefix = warp_radix_pass<11>(sc, n, resident, buf, hist, 21, 0u, 0u, kk, &above) << 21;
+  int kk = k, above, in_bin;
+  uint32_t prefix = warp_radix_pass<11, true>(sc, n, resident, buf, hist, 21, 0u, 0u, kk, &above, &in_bin) << 21;
   kk -= above;
-  prefix |= warp_radix_pass<11>(sc, n, resident, buf, hist, 10, 0xFFE00000u, prefix, kk, &above) << 10;
+  prefix |= warp_radix_pass<11, false>(sc, n, resident, buf, hist, 10, 0xFFE00000u, prefix, kk, &above, &in_bin)
+            << 10;
   kk -= above;
-  prefix |= warp_radix_pass<10>(sc, n, resident, buf, hist, 0, 0xFFFFFC00u, prefix, kk, &above);
+  prefix |= warp_radix_pass<10, false>(sc, n, resident, buf, hist, 0, 0xFFFFFC00u, prefix, kk, &above, &in_bin);
   kk -= above;
   const uint32_t thr = prefix;
   const int need_eq = kk;
+  // in_bin = the number of keys equal to thr: when all of them are taken
+  // (the usual case) the choice is simply key >= thr
+  const bool all_eq = need_eq == in_bin;
   int out_off = 0, eq_seen = 0;
   const unsigned lt = (1u << lane) - 1u;
   for (int c0 = 0; c0 < n; c0 += idxtc::kSelChunk) {
@@ -234,18 +244,30 @@ __device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, 
         const int s = base + 32 * u + lane;
         key[u] = s < cn ? __float_as_uint(buf[s]) : 0u;
       }
+      if (all_eq) {
+        unsigned btk[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int s = base + 32 * u + lane;
-        const bool gt = s < cn && key[u] > thr;
-        const bool eq = s < cn && key[u] == thr;
-        const unsigned beq = __ballot_sync(kFull, eq);
-        const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
-        const unsigned btk = __ballot_sync(kFull, take);
-        const int p = out_off + __popc(btk & lt);
-        if (take && p < k) out[p] = c0 + s;
-        out_off += __popc(btk);
-        eq_seen += __popc(beq);
+        for (int u = 0; u < 4; ++u) btk[u] = __ballot_sync(kFull, base + 32 * u + lane < cn && key[u] >= thr);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int p = out_off + __popc(btk[u] & lt);
+          if (((btk[u] >> lane) & 1u) && p < k) out[p] = c0 + base + 32 * u + lane;
+          out_off += __popc(btk[u]);
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int s = base + 32 * u + lane;
+          const bool gt = s < cn && key[u] > thr;
+          const bool eq = s < cn && key[u] == thr;
+          const unsigned beq = __ballot_sync(kFull, eq);
+          const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
+          const unsigned btk = __ballot_sync(kFull, take);
+          const int p = out_off + __popc(btk & lt);
+          if (take && p < k) out[p] = c0 + s;
+          out_off += __popc(btk);
+          eq_seen += __popc(beq);
+        }
       }
     }
     __syncwarp();
