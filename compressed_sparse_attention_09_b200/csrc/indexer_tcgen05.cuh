@@ -98,10 +98,10 @@ __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, 
 // key `thr` itself and how many keys equal to it are taken.  An ordered pass
 // then writes every key > thr and the first `need_eq` keys == thr.
 //
-// The row is read through `buf` (kSelChunk floats of shared memory) a chunk
-// at a time, eight 16-byte loads per lane in flight; a row that fits in one
-// chunk is read from global memory once and every pass runs on shared
-// memory.  Each lane takes four consecutive scores per step, so that
+// A row that fits in `buf` (kSelChunk words of shared memory) is read from
+// global memory once and every pass runs on shared memory; a longer row is
+// read straight into registers on every pass, kStreamVecs 16-byte loads per
+// lane in flight.  Each lane takes four consecutive scores per step, so that
 // four independent key/histogram chains are in flight per lane.
 __device__ __forceinline__ void warp_stage_chunk(const float* src, int n, float* buf) {
   constexpr int kBatch = 8;   // 16-byte loads in flight per lane
@@ -129,6 +129,19 @@ __device__ __forceinline__ void warp_stage_chunk(const float* src, int n, float*
   __syncwarp();
 }
 
+// 16-byte loads per lane in flight when a row is read straight from global memory
+constexpr int kStreamVecs = 8;
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += t;
+  }
+  return v;
+}
+
 // One radix pass over the keys k of sc[0..n) with (k & mask) == prefix:
 // returns the WIDTH-bit digit at `shift` that holds the kk-th largest of
 // them (kk >= 1, at most their number) and, in *above, how many of them have
@@ -145,11 +158,9 @@ __device__ __noinline__ uint32_t warp_radix_pass(const float* sc, int n, bool re
 #pragma unroll 4
   for (int i = lane; i < NB / 4; i += 32) reinterpret_cast<int4*>(hist)[i] = make_int4(0, 0, 0, 0);
   __syncwarp();
-  for (int c0 = 0; c0 < n; c0 += idxtc::kSelChunk) {
-    const int cn = min(idxtc::kSelChunk, n - c0);
-    if (!resident) warp_stage_chunk(sc + c0, cn, buf);
-    // whole 16-byte vectors first, then the last cn % 4 keys one per lane
-    const int nv = cn >> 2;
+  if (resident) {
+    // whole 16-byte vectors first, then the last n % 4 keys one per lane
+    const int nv = n >> 2;
 #pragma unroll 2
     for (int i = lane; i < nv; i += 32) {
       const uint4 v = reinterpret_cast<const uint4*>(buf)[i];
@@ -158,12 +169,38 @@ __device__ __noinline__ uint32_t warp_radix_pass(const float* sc, int n, bool re
       for (int u = 0; u < 4; ++u)
         if (FIRST || (e[u] & mask) == prefix) atomicAdd(&hist[(e[u] >> shift) & (uint32_t)(NB - 1)], 1);
     }
-    if (lane < cn - 4 * nv) {
+    if (lane < n - 4 * nv) {
       const uint32_t key = __float_as_uint(buf[4 * nv + lane]);
       if (FIRST || (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint32_t)(NB - 1)], 1);
     }
-    __syncwarp();
+  } else {
+    // a row longer than the staging buffer is read straight into registers,
+    // kStreamVecs 16-byte loads per lane in flight
+    const uint4* src4 = reinterpret_cast<const uint4*>(sc);
+    const int nv = n >> 2;
+    for (int i0 = 0; i0 < nv; i0 += 32 * kStreamVecs) {
+      uint4 v[kStreamVecs];
+#pragma unroll
+      for (int u = 0; u < kStreamVecs; ++u) {
+        const int i = i0 + lane + 32 * u;
+        v[u] = i < nv ? __ldcg(src4 + i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kStreamVecs; ++u) {
+        if (i0 + lane + 32 * u < nv) {
+          const uint32_t e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (FIRST || (e[j] & mask) == prefix) atomicAdd(&hist[(e[j] >> shift) & (uint32_t)(NB - 1)], 1);
+        }
+      }
+    }
+    if (lane < n - 4 * nv) {
+      const uint32_t key = __ldcg(reinterpret_cast<const unsigned*>(sc) + 4 * nv + lane);
+      if (FIRST || (key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (uint32_t)(NB - 1)], 1);
+    }
   }
+  __syncwarp();
   // Position p = NB - 1 - digit (p = 0 is the largest digit).  Lane L sums
   // positions [PER L, PER L + PER), visiting them in a lane-rotated order so
   // that the 32 lanes read 32 different banks.
@@ -232,9 +269,73 @@ __device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, 
   const bool all_eq = need_eq == in_bin;
   int out_off = 0, eq_seen = 0;
   const unsigned lt = (1u << lane) - 1u;
+  if (!resident) {
+    // long row, straight from global memory: lane l takes the four keys
+    // 4 (i0 + l) .. + 3 of each 128-key step, and the positions follow from a
+    // prefix over the lanes' take counts (ascending index order)
+    const uint4* src4 = reinterpret_cast<const uint4*>(sc);
+    const int nv = n >> 2;
+    for (int i0 = 0; i0 < nv; i0 += 32 * kStreamVecs) {
+      uint4 v[kStreamVecs];
+#pragma unroll
+      for (int u = 0; u < kStreamVecs; ++u) {
+        const int i = i0 + lane + 32 * u;
+        v[u] = i < nv ? __ldcg(src4 + i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kStreamVecs; ++u) {
+        const int i = i0 + lane + 32 * u;
+        const bool valid = i < nv;
+        const uint32_t e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        bool take[4];
+        if (all_eq) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) take[j] = valid && e[j] >= thr;
+        } else {
+          int ceq = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) ceq += (valid && e[j] == thr) ? 1 : 0;
+          const int incl_eq = warp_incl_scan(ceq);
+          int eqr = eq_seen + incl_eq - ceq;   // equal keys before this lane's four
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const bool eq = valid && e[j] == thr;
+            take[j] = (valid && e[j] > thr) || (eq && eqr < need_eq);
+            eqr += eq ? 1 : 0;
+          }
+          eq_seen += __shfl_sync(kFull, incl_eq, 31);
+        }
+        int cnt = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cnt += take[j] ? 1 : 0;
+        const int incl = warp_incl_scan(cnt);
+        int p = out_off + incl - cnt;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (take[j]) {
+            if (p < k) out[p] = 4 * i + j;
+            ++p;
+          }
+        out_off += __shfl_sync(kFull, incl, 31);
+      }
+    }
+    // the last n % 4 keys, one per lane
+    {
+      const int s = 4 * nv + lane;
+      const bool in = s < n;
+      const uint32_t key = in ? __ldcg(reinterpret_cast<const unsigned*>(sc) + s) : 0u;
+      const bool gt = in && key > thr;
+      const bool eq = in && key == thr;
+      const unsigned beq = __ballot_sync(kFull, eq);
+      const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
+      const unsigned btk = __ballot_sync(kFull, take);
+      const int p = out_off + __popc(btk & lt);
+      if (take && p < k) out[p] = s;
+    }
+    return;
+  }
   for (int c0 = 0; c0 < n; c0 += idxtc::kSelChunk) {
     const int cn = min(idxtc::kSelChunk, n - c0);
-    if (!resident) warp_stage_chunk(sc + c0, cn, buf);
     for (int base = 0; base < cn; base += 128) {
       // four 32-score groups: keys first (independent loads), then the
       // ordered compaction group by group
