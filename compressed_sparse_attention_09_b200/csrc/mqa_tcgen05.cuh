@@ -31,10 +31,11 @@
 // the lower 16 lanes of every lane quarter, 256-511 in the upper 16); four S
 // buffers of 64 columns, each holding the four partials (issuer i at column
 // offset 32 (i / 2) and lane offset 16 (i % 2)).  A softmax thread owns one
-// head and half of a tile (16 entries).  O is rescaled (TMEM load, multiply,
-// store) only when a head's running maximum grows by more than 8 in log2
-// units; otherwise the stale maximum is kept, which is exact because O and
-// the normaliser l share it.
+// head and half of a tile (16 entries) and writes its piece of the P row into
+// one of four P buffers (64-byte rows in the 64-byte swizzle).  O is rescaled
+// (TMEM load, multiply, store) only when a head's running maximum grows by
+// more than 8 in log2 units; otherwise the stale maximum is kept, which is
+// exact because O and the normaliser l share it.
 //
 // Warp roles (544 threads): warps 0-7 gather the entry tiles (thread 0 also
 // loads q with a 3-D TMA); warps 8-11 issue the S products and warp 12 the O
@@ -61,7 +62,8 @@ constexpr int kQChunk = 64 * 128;           // [64 heads x 64 bf16], 128-byte ro
 constexpr int kCChunk = kTile * 128;        // [32 entries x 64 bf16]
 constexpr int kQBytes = 8 * kQChunk;        // 64 x 512
 constexpr int kCBytes = 8 * kCChunk;        // one tile: 32 entries x 512
-constexpr int kPBytes = 64 * 128;           // 64 heads x 32 entries (rows padded to 128 B), swizzled
+constexpr int kPBytes = 64 * 64;            // 64 heads x 32 entries, 64-byte rows, swizzled
+constexpr int kPBufs = 4;                   // P buffers
 constexpr int kProducers = 256;             // threads of warps 0-7
 constexpr int kIssuers = 4;                 // S issuers: warps 8-11
 constexpr int kSBufs = 4;                   // S buffers in TMEM
@@ -69,7 +71,7 @@ constexpr int kOffQ = 0;
 constexpr int kOffC = kOffQ + kQBytes;
 constexpr int kOffP = kOffC + kStages * kCBytes;
 constexpr int kStageBytes = 4 * 32 * 128;     // O staging: 32 rows of 128 B per softmax warp
-constexpr int kOffStage = kOffP + 2 * kPBytes;
+constexpr int kOffStage = kOffP + kPBufs * kPBytes;
 constexpr int kOffMisc = kOffStage + kStageBytes;
 constexpr int kMiscBytes = 256;
 constexpr size_t kSmem = 1024 + kOffMisc + kMiscBytes;
@@ -80,6 +82,8 @@ constexpr uint32_t kColO = 0, kColS = 256;
 
 // byte offset of 16-byte unit u (0..7) of row r in a 128-byte-swizzled chunk
 __device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
+// byte offset of 16-byte unit u (0..3) of row r in a 64-byte-swizzled block
+__device__ __forceinline__ uint32_t sw64(int r, int u) { return (uint32_t)(r * 64 + ((u ^ ((r >> 1) & 3)) << 4)); }
 
 // Number of kTile-entry tiles a query row needs: up to its last valid slot
 // (0 <= s < avail).  Called by a whole warp; every warp role derives it on
@@ -121,8 +125,8 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
   uint64_t* t_done = c_full + kStages;         // [kStages] O product of the stage's tile done (frees it)
   uint64_t* s_full = t_done + kStages;         // [kSBufs] all four S partials written
   uint64_t* s_free = s_full + kSBufs;          // [kSBufs]
-  uint64_t* p_full = s_free + kSBufs;          // [2]
-  uint64_t* o_free = p_full + 2;
+  uint64_t* p_full = s_free + kSBufs;          // [kPBufs]
+  uint64_t* o_free = p_full + kPBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_free + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -141,7 +145,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       mbar_init(&s_full[s], kIssuers);
       mbar_init(&s_free[s], 4);
     }
-    for (int s = 0; s < 2; ++s) mbar_init(&p_full[s], 4);
+    for (int s = 0; s < kPBufs; ++s) mbar_init(&p_full[s], 4);
     mbar_init(o_free, 4);
     *abort_flag = 0;
     fence_barrier_init();
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
     // only once P is written, i.e. after all four S partials have completed.
     constexpr uint32_t idO = idesc_bf16_f32_bmn(64, 256);
     const uint64_t od0 = sdesc_mn_sw128(smem_u32(c_s), kCChunk, 1024);  // stages as MN-major operands
-    const uint64_t pd0 = sdesc_k_sw128(smem_u32(p_s));
+    const uint64_t pd0 = sdesc_k_sw64(smem_u32(p_s));
     uint32_t g = 0, oi = 0;
     for (int it = blockIdx.x; it < items; it += gridDim.x) {
       if (warp_aborted(abort_flag)) break;
@@ -283,8 +287,8 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       if (lane == 0) {
         for (int j = 0; j < ntiles; ++j) {
           const uint32_t gj = g + j;
-          const int st = (int)(gj % kStages), pb = (int)(gj & 1);
-          if (!mbar_wait(&p_full[pb], (gj >> 1) & 1) ||
+          const int st = (int)(gj % kStages), pb = (int)(gj % kPBufs);
+          if (!mbar_wait(&p_full[pb], (gj / kPBufs) & 1) ||
               (j == 0 && !mbar_wait(o_free, (oi & 1) ^ 1))) {   // previous item's O stored
             ok = 0;
             break;
@@ -335,7 +339,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       int sidx = lane < a.topk ? __ldg(ir + lane) : -1;   // slot of this lane in tile 0
       for (int j = 0; j < ntiles; ++j) {
         const uint32_t gj = g + j;
-        const int sb = (int)(gj % kSBufs), pb = (int)(gj & 1);
+        const int sb = (int)(gj % kSBufs), pb = (int)(gj % kPBufs);
         // validity of this tile's 32 slots; the next tile's slot is fetched meanwhile
         const uint32_t vmask = __ballot_sync(kFull, sidx >= 0 && sidx < avail);
         {
@@ -403,14 +407,14 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
         }
         m_run = m_use;
         l_run += sum;
-        // P rows, once the P buffer's previous reader (tile gj - 2) is done
-        if (gj >= 2) {
-          const uint32_t gp = gj - 2;
+        // P rows, once the P buffer's previous reader (tile gj - kPBufs) is done
+        if (gj >= (uint32_t)kPBufs) {
+          const uint32_t gp = gj - kPBufs;
           if (!warp_wait(&t_done[gp % kStages], (gp / kStages) & 1)) { ok = false; break; }
         }
         uint8_t* prow = p_s + pb * kPBytes;
-        *reinterpret_cast<uint4*>(prow + sw128(hrow, 2 * half)) = pk[0];
-        *reinterpret_cast<uint4*>(prow + sw128(hrow, 2 * half + 1)) = pk[1];
+        *reinterpret_cast<uint4*>(prow + sw64(hrow, 2 * half)) = pk[0];
+        *reinterpret_cast<uint4*>(prow + sw64(hrow, 2 * half + 1)) = pk[1];
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[pb]);

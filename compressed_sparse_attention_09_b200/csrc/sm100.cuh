@@ -182,6 +182,16 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t addr) {
 // the start-address field (address / 16, 14 bits) cannot overflow because
 // shared memory addresses stay below 256 KB.  With constant offsets this is
 // one add, instead of rebuilding the descriptor before every MMA.
+// Shared-memory descriptor of a K-major operand in 64-byte-swizzled storage:
+// 64-byte rows (32 bf16 of K), 8-row atoms of 512 B stacked along M/N.
+__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu)     // start address / 16
+         | ((uint64_t)1 << 16)                  // leading-dimension byte offset (unused for swizzled K-major)
+         | ((uint64_t)(512 >> 4) << 32)         // stride byte offset: 8 rows x 64 B
+         | ((uint64_t)1 << 46)                  // descriptor version (sm_100)
+         | ((uint64_t)4 << 61);                 // swizzle mode: 64 B
+}
+
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t byte_off) { return d + (uint64_t)(byte_off >> 4); }
 
 // 32 consecutive fp32 TMEM columns of this thread's lane.
