@@ -768,7 +768,8 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
 // global memory (L2) on every pass; shared memory holds only histograms.
 namespace dsel {
 constexpr int kWarps = 16, kBins = 2048;
-constexpr size_t kSmem = (size_t)(kWarps + 1) * kBins * 4 + 64 * 4;
+constexpr int kResident = 16384;   // rows of up to this many scores are selected from shared memory
+constexpr size_t kSmem = (size_t)(kWarps + 1) * kBins * 4 + 64 * 4 + (size_t)kResident * 4;
 }  // namespace dsel
 
 // Warp 0: the digit of the combined histogram hist[0..NB) holding the kk-th
@@ -825,6 +826,7 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
   int* whist = dsm;                         // [kWarps][kBins] per-warp histograms
   int* hist = dsm + kWarps * kBins;         // [kBins] combined
   int* ws = hist + kBins;                   // [64] scratch words
+  uint32_t* keys = reinterpret_cast<uint32_t*>(ws + 64);   // [kResident] the row's keys, when it fits
   const int b = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = pos[b];
@@ -836,6 +838,26 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
     return;
   }
   const float* row = scratch + (long long)b * cap;
+  // A row that fits is read from L2 once, with every thread's loads in
+  // flight together, and kept as keys; the passes below then read shared
+  // memory.  Longer rows are read from L2 on every pass.
+  const bool resident = avail <= kResident;
+  if (resident) {
+    for (int i0 = tid; i0 < avail; i0 += 512 * 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + 512 * u;
+        v[u] = i < avail ? __ldcg(row + i) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + 512 * u;
+        if (i < avail) keys[i] = ordered_key(v[u]);
+      }
+    }
+  }
+  auto key_at = [&](int i) -> uint32_t { return resident ? keys[i] : ordered_key(__ldcg(row + i)); };
   int* myh = whist + warp * kBins;
   uint32_t prefix = 0, mask = 0;
   int kk = topk;
@@ -852,7 +874,7 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
       for (int u = 0; u < 4; ++u) {
         const int i = i0 + u;
         if (i < avail) {
-          const uint32_t key = ordered_key(__ldcg(row + i));
+          const uint32_t key = key_at(i);
           if ((key & mask) == prefix) atomicAdd(&myh[(key >> shift) & dmask], 1);
         }
       }
@@ -883,7 +905,7 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
   int n_gt = 0, n_eq = 0;
   for (int base = s0; base < s1; base += 32) {
     const int i = base + lane;
-    const uint32_t key = i < s1 ? ordered_key(__ldcg(row + i)) : 0u;
+    const uint32_t key = i < s1 ? key_at(i) : 0u;
     n_gt += __popc(__ballot_sync(kFull, i < s1 && key > thr));
     n_eq += __popc(__ballot_sync(kFull, i < s1 && key == thr));
   }
@@ -901,7 +923,7 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
   const unsigned lt = (1u << lane) - 1u;
   for (int base = s0; base < s1; base += 32) {
     const int i = base + lane;
-    const uint32_t key = i < s1 ? ordered_key(__ldcg(row + i)) : 0u;
+    const uint32_t key = i < s1 ? key_at(i) : 0u;
     const bool gt = i < s1 && key > thr;
     const bool eq = i < s1 && key == thr;
     const unsigned beq = __ballot_sync(kFull, eq);

@@ -406,3 +406,10 @@ def test_decode_tensor_core_indexer(m):
     and the per-sequence selection, across cache appends."""
     dims = csa.Dims(d=256, c=128, m=m, cI=128, nhI=64, nh=4, dc=128, topk=16, dtype=csa.CSA_BF16)
     decode_case(dims, B=5, pos0=301, cap=400, steps=6, seed=63 + m, check=[0, 3, 4])
+
+
+def test_decode_selection_of_rows_longer_than_shared_memory():
+    """Cached rows longer than the 16384 scores the selection keeps in shared
+    memory are selected from L2 instead; both forms must pick the oracle's set."""
+    dims = csa.Dims(d=256, c=128, m=4, cI=128, nhI=64, nh=4, dc=128, topk=64, dtype=csa.CSA_BF16)
+    decode_case(dims, B=2, pos0=4 * 17000 + 1, cap=17100, steps=2, seed=67, check=[0, 1])
