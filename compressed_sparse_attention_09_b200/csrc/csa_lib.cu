@@ -185,23 +185,36 @@ csa_status launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const Tc
   auto k = gemm_tc_kernel<BN, kStages>;
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM) != cudaSuccess)
     return CSA_ERR_CUDA;
-  const int tiles = ((g.M + Cfg::BM - 1) / Cfg::BM) * ((g.N + BN - 1) / BN);
+  const int tiles = ((g.M + Cfg::BM - 1) / Cfg::BM) * ((g.N + BN - 1) / BN) * g.k_split;
   const int grid = tiles < sm_count() ? tiles : sm_count();
   k<<<grid, 192, Cfg::SMEM, st>>>(ta, tb, g);
   CSA_CHECK_LAUNCH();
+  if (g.k_split > 1) {
+    const int m_pad = ((g.M + Cfg::BM - 1) / Cfg::BM) * Cfg::BM;
+    const long long n = (long long)g.N * g.M;
+    gemm_split_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(g.part, g.k_split, g.M, m_pad, g.N, g.out);
+    CSA_CHECK_LAUNCH();
+  }
   return CSA_OK;
 }
+
+// fp32 bytes of the K-split partial sums a swap-AB GEMM with n_out output
+// features and m_rows activation rows may use (four slices).
+size_t gemm_split_bytes(int n_out, int m_rows) { return (size_t)4 * round_up_int(n_out, 128) * m_rows * 4; }
 
 // D[M, N] = A[M, K] . B[N, K]^T routed to `out`.  A: activations (row stride
 // lda), B: packed K-major weights with at least round_up(N, 256) rows.
 csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const void* B, long long ldb,
-                       int M, int N, int K, const GemmOut& out, cudaStream_t st) {
+                       int M, int N, int K, const GemmOut& out, cudaStream_t st, float* split_ws = nullptr,
+                       size_t split_ws_bytes = 0) {
   if (M == 0) return CSA_OK;
   if (d->dtype == CSA_BF16) {
     CUtensorMap ta, tb;
     TcGemmArgs g;
     g.K = K;
     g.out = out;
+    g.k_split = 1;
+    g.part = nullptr;
     if (M >= 128) {  // activations as the M operand, 128 x BN tiles
       // BN = 192 where it fills the last wave and the padded columns better
       // (the packed weights are padded to 256 rows, so both widths stay in range)
@@ -228,6 +241,18 @@ csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const vo
       return CSA_ERR_UNSUPPORTED;
     g.M = N; g.N = M; g.transpose_out = 1;
     g.group_m = (N + 127) / 128;
+    // Few weight tiles (fewer than half the SMs): split K over 4 or 2 work
+    // units per tile so that more SMs stream the weights; the slices' fp32
+    // sums go through split_ws and one reduction kernel.
+    const int w_tiles = (N + 127) / 128, k_blocks = (K + 63) / 64;
+    for (int ks = 4; split_ws && ks >= 2; ks /= 2) {
+      if ((long long)w_tiles * ks <= sm_count() && k_blocks % ks == 0 && k_blocks / ks >= 4 &&
+          (size_t)ks * (size_t)w_tiles * 128 * (size_t)M * 4 <= split_ws_bytes) {
+        g.k_split = ks;
+        g.part = split_ws;
+        break;
+      }
+    }
     if (M <= 64) return launch_tc_gemm<64, 8>(ta, tb, g, st);
     return CSA_ERR_UNSUPPORTED;
   }
@@ -377,14 +402,14 @@ csa_status launch_mqa(const csa_dims* d, const MqaArgs& a, int rows, cudaStream_
 
 // A1: eqs. (1), (2), (5), (7) and the indexer-key projections, one GEMM
 csa_status project_hidden(const csa_dims* d, const void* packed, const void* H, int T, void* Y1, float* wI,
-                          cudaStream_t st) {
+                          cudaStream_t st, float* split_ws = nullptr, size_t split_ws_bytes = 0) {
   const PackLayout P = pack_layout(d);
   GemmOut o;
   memset(&o, 0, sizeof(o));
   o.seg[0] = {0, P.N1b, Y1, P.N1b, 0};
   o.seg[1] = {P.N1b, d->nhI, wI, d->nhI, 1};
   o.nseg = 2;
-  return launch_gemm(d, H, d->d, at((void*)packed, P.w1), d->d, T, P.N1, d->d, o, st);
+  return launch_gemm(d, H, d->d, at((void*)packed, P.w1), d->d, T, P.N1, d->d, o, st, split_ws, split_ws_bytes);
 }
 
 // A2: eqs. (6), (10) from the shared c^Q
@@ -790,7 +815,7 @@ csa_status launch_append(const csa_dims* d, const void* packed, const void* rows
 }
 
 struct DecLayout {
-  size_t y1, wI, y2, idx, scratch, total;
+  size_t y1, wI, y2, idx, scratch, split, total;
 };
 DecLayout dec_layout(const csa_dims* d, int B, int cap) {
   const PackLayout P = pack_layout(d);
@@ -802,6 +827,7 @@ DecLayout dec_layout(const csa_dims* d, int B, int cap) {
   L.y2 = off; off = align_up(off + (size_t)B * P.N2 * es);
   L.idx = off; off = align_up(off + (size_t)B * d->topk * 4);
   L.scratch = off; off = align_up(off + (size_t)B * (size_t)cap * 4);
+  L.split = off; off = align_up(off + gemm_split_bytes(P.N1, B));   // K-split sums of the A1 projection
   L.total = off;
   return L;
 }
@@ -869,7 +895,8 @@ csa_status csa_decode(const csa_dims* d, const void* packed, const void* h, cons
   float* wI = reinterpret_cast<float*>(at(ws, L.wI));
   char* y2 = at(ws, L.y2);
   int* idx = idx_out ? idx_out : reinterpret_cast<int*>(at(ws, L.idx));
-  s = project_hidden(d, packed, h, B, y1, wI, st);
+  s = project_hidden(d, packed, h, B, y1, wI, st, reinterpret_cast<float*>(at(ws, L.split)),
+                     L.total - L.split);
   if (s != CSA_OK) return s;
   s = launch_append(d, packed, y1, P.N1b, pos, ring, Ccache, KIcache, cache_len, cap, B, st);
   if (s != CSA_OK) return s;

@@ -29,6 +29,12 @@ struct TcGemmArgs {
   GemmOut out;
   int transpose_out;   // 1: D[i][j] is stored at output row j, column i (swap-AB use)
   int group_m;         // tile order: groups of group_m row tiles, each group's tiles column by column
+  // Split of K (swap-AB use only): k_split > 1 gives every tile k_split work
+  // units over equal ranges of K blocks; each stores its fp32 sum for rows
+  // r < M at part[(ks * N + j) * Mpad + r] (Mpad = row tiles x 128) instead of
+  // `out`, and gemm_split_reduce_kernel adds the slices in order.
+  int k_split;
+  float* part;
 };
 
 // Tile `tile` of the visiting order -> (row tile, column tile).  Within a
@@ -129,7 +135,8 @@ __global__ void __launch_bounds__(192, 1)
   const int m_tiles = (g.M + Cfg::BM - 1) / Cfg::BM;
   const int n_tiles = (g.N + BN - 1) / BN;
   const int k_blocks = (g.K + Cfg::BK - 1) / Cfg::BK;
-  const int total = m_tiles * n_tiles;
+  const int kbs = (k_blocks + g.k_split - 1) / g.k_split;   // K blocks per work unit
+  const int total = m_tiles * n_tiles * g.k_split;          // work units: (tile, K slice)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -155,10 +162,11 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {  // ---------------- TMA producer
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+      for (int unit = blockIdx.x; unit < total && !*abort_flag; unit += gridDim.x) {
+        const int tile = unit / g.k_split, kb0 = (unit % g.k_split) * kbs, kb1 = min(k_blocks, kb0 + kbs);
         int mt, nt;
         gemm_tile_coords(tile, m_tiles, n_tiles, g.group_m, mt, nt);
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
           mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
           tma_load_2d(&tmA, &full[stage], smA + stage * Cfg::A_BYTES, kb * Cfg::BK, mt * Cfg::BM);
@@ -174,18 +182,19 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+      for (int unit = blockIdx.x; unit < total && !*abort_flag; unit += gridDim.x) {
+        const int kb0 = (unit % g.k_split) * kbs, kb1 = min(k_blocks, kb0 + kbs);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
           tc_fence_after();
           const uint64_t ad = sdesc_k_sw128(smem_u32(smA + stage * Cfg::A_BYTES));
           const uint64_t bd = sdesc_k_sw128(smem_u32(smB + stage * Cfg::B_BYTES));
 #pragma unroll
           for (int k = 0; k < Cfg::BK / 16; ++k)
-            mma_bf16(d_tmem, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc, (kb | k) != 0);
+            mma_bf16(d_tmem, desc_add(ad, k * 32), desc_add(bd, k * 32), idesc, (kb != kb0 || k != 0) ? 1u : 0u);
           mma_commit(&empty[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
@@ -203,7 +212,8 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* stage_out = smOut + (warp - 2) * (32 * 128);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+    for (int unit = blockIdx.x; unit < total && !*abort_flag; unit += gridDim.x) {
+      const int tile = unit / g.k_split, ks = unit % g.k_split;
       int mt, nt;
       gemm_tile_coords(tile, m_tiles, n_tiles, g.group_m, mt, nt);
       if (!mbar_wait(&tfull[acc], acc_phase)) { *abort_flag = 1; break; }
@@ -215,6 +225,18 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t ta = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN + ch * 64);
         tmem_ld_32x32b_x32_pair(ta, ta + 32u, v0, v1);
         const int c0 = nt * BN + ch * 64;
+        if (g.k_split > 1) {   // this K slice's fp32 sum, column c0 + j of row r at part[(ks N + c0 + j) Mpad + r]
+          if (r < g.M) {
+            float* dst = g.part + (size_t)ks * g.N * ((size_t)m_tiles * Cfg::BM) + r;
+            const size_t ld = (size_t)m_tiles * Cfg::BM;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (c0 + j < g.N) dst[(size_t)(c0 + j) * ld] = v0[j];
+              if (c0 + 32 + j < g.N) dst[(size_t)(c0 + 32 + j) * ld] = v1[j];
+            }
+          }
+          continue;
+        }
         if (g.transpose_out) {
           // D[r][c0 + j] goes to output row c0 + j, column r: one segment
           // per thread (its column), consecutive lanes write consecutive
@@ -284,6 +306,18 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
+}
+
+// The K slices of a split swap-AB GEMM added in slice order (the same sum
+// whatever the timing of the slices) and stored as that GEMM stores its
+// output: D[r][j] at output row j, column r, through the segments of `out`.
+__global__ void gemm_split_reduce_kernel(const float* part, int k_split, int M, int Mpad, int N, GemmOut out) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)N * M) return;
+  const int j = (int)(i / M), r = (int)(i % M);
+  float acc = 0.f;
+  for (int q = 0; q < k_split; ++q) acc += part[((size_t)q * N + j) * Mpad + r];
+  store_out<__nv_bfloat16>(out, j, r, acc);
 }
 
 }  // namespace csa

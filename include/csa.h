@@ -267,7 +267,8 @@ csa_status csa_cache_append(const csa_dims* dims, const void* packed, const void
                             int* cache_len, int cap, int B, void* stream);
 
 /* Workspace bytes csa_decode needs for B sequences with caches of capacity
- * cap entries. */
+ * cap entries: the projections, the indexer scores [B, cap] fp32, the
+ * selected indices and the fp32 partial sums of the K-split A1 projection. */
 size_t csa_decode_workspace_bytes(const csa_dims* dims, int B, int cap);
 
 /* One decode step: each of B independent sequences gets one new token h_b

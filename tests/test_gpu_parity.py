@@ -413,3 +413,12 @@ def test_decode_selection_of_rows_longer_than_shared_memory():
     memory are selected from L2 instead; both forms must pick the oracle's set."""
     dims = csa.Dims(d=256, c=128, m=4, cI=128, nhI=64, nh=4, dc=128, topk=64, dtype=csa.CSA_BF16)
     decode_case(dims, B=2, pos0=4 * 17000 + 1, cap=17100, steps=2, seed=67, check=[0, 1])
+
+
+def test_decode_projection_split_over_k():
+    """A decode projection with few output tiles splits K over several CTAs
+    (d = 1024: four slices of four K blocks) and adds the slices in a
+    reduction that also routes the fp32 head weights; the step must still
+    match the oracle."""
+    dims = csa.Dims(d=1024, c=128, m=4, cI=128, nhI=64, nh=4, dc=128, topk=16, dtype=csa.CSA_BF16)
+    decode_case(dims, B=5, pos0=301, cap=400, steps=2, seed=71, check=[0, 2, 4])
