@@ -51,14 +51,6 @@ __device__ __forceinline__ void load_vec_f32(const T* p, float* out) {
   for (int i = 0; i < Vec16<T>::V; ++i) out[i] = to_f32(v.e[i]);
 }
 
-template <typename T>
-__device__ __forceinline__ void store_vec_f32(T* p, const float* in) {
-  Vec16<T> v;
-#pragma unroll
-  for (int i = 0; i < Vec16<T>::V; ++i) v.e[i] = from_f32<T>(in[i]);
-  *reinterpret_cast<uint4*>(p) = v.u;
-}
-
 // 2^x by the hardware approximation (ex2.approx.ftz.f32: relative error of
 // about 2^-22, 2^-inf = +0).
 __device__ __forceinline__ float ex2_approx_f32(float x) {

@@ -379,8 +379,8 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float x0 = sv[8 * u + 2 * q], x1 = sv[8 * u + 2 * q + 1];
-            const float p0 = x0 == -INFINITY ? 0.f : ex2_approx(x0 - m_use);
-            const float p1 = x1 == -INFINITY ? 0.f : ex2_approx(x1 - m_use);
+            const float p0 = x0 == -INFINITY ? 0.f : ex2_approx_f32(x0 - m_use);
+            const float p1 = x1 == -INFINITY ? 0.f : ex2_approx_f32(x1 - m_use);
             sum += p0 + p1;
             __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
             w[q] = *reinterpret_cast<uint32_t*>(&h2);
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
           const uint32_t gp = gj - 1;
           if (!warp_wait(&t_done[gp % kStages], (gp / kStages) & 1)) { ok = false; break; }
           tc_fence_after();
-          const float alpha = grow ? ex2_approx(m_run - m_new) : 1.f;   // 2^-inf = 0 when nothing was seen
+          const float alpha = grow ? ex2_approx_f32(m_run - m_new) : 1.f;   // 2^-inf = 0 when nothing was seen
 #pragma unroll 1
           for (int ch = 0; ch < 8; ++ch) {
             float v[32];
