@@ -120,7 +120,8 @@ def compress(Ca, Cb, Za, Zb, Ba, Bb, m):
         Z^a[m*i + r, j] + B^a[r, j]          (r = 0..m-1, the block itself)
         Z^b[m*(i-1) + r, j] + B^b[r, j]      (r = 0..m-1, the block before)
     Softmax_row normalises these 2m values jointly and independently for each
-    channel j (eq. 3: "normalises the total 2m elements from Z^a and Z^b").
+    channel j (eq. 3 and the paragraph after eq. 4: the row softmax spans the
+    2m logits from Z^a and Z^b together).
     Eq. (4) then sums S^a * C^a over the block and S^b * C^b over the block
     before.  At i = 0 the Z^b logits are -inf and the C^b rows are 0, so the
     softmax runs over the m C^a logits only.  Row r of each bias is added to
@@ -227,8 +228,9 @@ def csa_forward(H, W, dims, seqlens, store="exact", rows=None, keep_scores=False
     W: dict of weights, shapes as on the page ([in, out]):
        W_aKV, W_bKV, W_aZ, W_bZ [d, c]; B_a, B_b [m, c];
        W_aKV_I, W_bKV_I, W_aZ_I, W_bZ_I [d, c^I]; B_a_I, B_b_I [m, c^I]
-       (the indexer keys use "the same compression operation", read as a
-       separate parameter set of the same form with width c^I);
+       (the page builds the indexer keys by the same kind of compression as
+       C^Comp without naming its parameters; read as a separate parameter
+       set of the same form with width c^I);
        W_DQ [d, d_c]; W_IUQ [d_c, n_h^I c^I] (eq. 6); W_UQ [d_c, n_h c]
        (eq. 10 -- the page reuses the symbol W^UQ with a second shape, read as
        a second matrix); W_w [d, n_h^I].
