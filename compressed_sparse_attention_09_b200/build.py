@@ -1,4 +1,9 @@
-"""Builds libcsa.so in-tree with nvcc for sm_100a (no GPU needed to build)."""
+"""Builds libcsa.so in-tree with nvcc for sm_100a (no GPU needed to build).
+
+CSA_NVTX=1 in the environment compiles in NVTX ranges named after the stages
+(host side, around each stage's launches) for profiler timelines; it takes
+effect on a forced rebuild (``python build.py --force``).
+"""
 from __future__ import annotations
 
 import os
@@ -39,7 +44,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not needs_build():
         return LIB
     tmp = LIB + ".tmp"
-    cmd = [NVCC, *FLAGS, *extra, "-o", tmp, os.path.join(CSRC, "csa_lib.cu")]
+    nvtx = ["-DCSA_NVTX"] if os.environ.get("CSA_NVTX") == "1" else []
+    cmd = [NVCC, *FLAGS, *nvtx, *extra, "-o", tmp, os.path.join(CSRC, "csa_lib.cu")]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)

@@ -8,6 +8,9 @@
 
 #include <algorithm>
 #include <atomic>
+#ifdef CSA_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
 
 #include "../../include/csa.h"
 #include "common.cuh"
@@ -38,6 +41,20 @@ std::atomic<uint64_t> g_launches{0};
     g_launches.fetch_add(1, std::memory_order_relaxed);         \
     if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA; \
   } while (0)
+
+// NVTX ranges around each stage's launches (host side), compiled in only
+// with -DCSA_NVTX so that a profiler timeline shows the stages by name.
+#ifdef CSA_NVTX
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define CSA_RANGE(name) NvtxRange csa_nvtx_range(name)
+#else
+#define CSA_RANGE(name) ((void)0)
+#endif
 
 size_t elem_size(const csa_dims* d) { return d->dtype == CSA_BF16 ? 2 : 4; }
 
@@ -318,6 +335,7 @@ bool indexer_tc_ok(const csa_dims* d) {
 
 csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int NB, void* ws, size_t ws_bytes,
                              cudaStream_t st) {
+  CSA_RANGE("A4 indexer_topk");
   const int sc_cap = padded_cap(a.sc_cap > 0 ? a.sc_cap : 1);
   if (!ws || ws_bytes < indexer_scratch_bytes(sc_cap) || reinterpret_cast<uintptr_t>(ws) % 16)
     return CSA_ERR_WORKSPACE;
@@ -342,6 +360,7 @@ csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int
 }
 
 csa_status launch_indexer(const csa_dims* d, const IndexerArgs& a, int rows, cudaStream_t st) {
+  CSA_RANGE("A4 indexer_topk");
   if (rows == 0) return CSA_OK;
   const size_t smem = indexer_smem(d, a.sc_cap);
   if (smem > kMaxSmem) return CSA_ERR_UNSUPPORTED;
@@ -367,6 +386,7 @@ csa_status mqa_launch(const MqaArgs& a, int rows, cudaStream_t st) {
 }
 
 csa_status launch_mqa(const csa_dims* d, const MqaArgs& a, int rows, cudaStream_t st) {
+  CSA_RANGE("A5 sparse_mqa");
   if (rows == 0) return CSA_OK;
   const bool b = d->dtype == CSA_BF16;
   if (b && d->c == mqa::kC && d->nh % mqa::kHeads == 0 && a.topk >= 1 && a.ld_q % 8 == 0 && a.ld_O % 8 == 0 &&
@@ -403,6 +423,7 @@ csa_status launch_mqa(const csa_dims* d, const MqaArgs& a, int rows, cudaStream_
 // A1: eqs. (1), (2), (5), (7) and the indexer-key projections, one GEMM
 csa_status project_hidden(const csa_dims* d, const void* packed, const void* H, int T, void* Y1, float* wI,
                           cudaStream_t st, float* split_ws = nullptr, size_t split_ws_bytes = 0) {
+  CSA_RANGE("A1 project_hidden");
   const PackLayout P = pack_layout(d);
   GemmOut o;
   memset(&o, 0, sizeof(o));
@@ -415,6 +436,7 @@ csa_status project_hidden(const csa_dims* d, const void* packed, const void* H, 
 // A2: eqs. (6), (10) from the shared c^Q
 csa_status project_query(const csa_dims* d, const void* packed, const void* cQ, long long ld_cQ, int T,
                          void* Y2, cudaStream_t st) {
+  CSA_RANGE("A2 project_query");
   const PackLayout P = pack_layout(d);
   GemmOut o;
   memset(&o, 0, sizeof(o));
@@ -438,6 +460,7 @@ CompressArgs make_compress_args(const csa_dims* d, const int* cu_seqlens, const 
 // A3 as the forward runs it: both key sets from the Y1 projection rows.
 csa_status compress_kv(const csa_dims* d, const void* packed, const void* Y1, int T, const int* cu_seqlens,
                        const int* cu_blocks, int nseq, int NB, void* Cc, void* KIc, cudaStream_t st) {
+  CSA_RANGE("A3 compress");
   const PackLayout P = pack_layout(d);
   const size_t es = elem_size(d);
   const int c = d->c, cI = d->cI;
@@ -724,6 +747,7 @@ csa_status csa_forward(const csa_dims* d, const void* packed, const void* H, con
                        const int* cu_blocks, int nseq, int total_tokens, int total_blocks, int max_seqlen,
                        void* O, void* Ccomp_out, void* KI_out, int* idx_out, void* ws, size_t ws_bytes,
                        void* stream) {
+  CSA_RANGE("csa_forward");
   csa_status s = check_dims(d);
   if (s != CSA_OK) return s;
   if (!packed || !H || !cu_seqlens || !cu_blocks || !O || !ws) return CSA_ERR_INVALID_ARG;
@@ -787,6 +811,7 @@ namespace {
 csa_status launch_append(const csa_dims* d, const void* packed, const void* rows, long long ld_rows,
                          const int* pos, void* ring, void* Ccache, void* KIcache, int* cache_len, int cap,
                          int B, cudaStream_t st) {
+  CSA_RANGE("A6 cache_append");
   if (B == 0) return CSA_OK;
   const PackLayout P = pack_layout(d);
   AppendArgs a;
@@ -836,6 +861,7 @@ DecLayout dec_layout(const csa_dims* d, int B, int cap) {
 // workspace, then one selection CTA per sequence.
 csa_status launch_indexer_decode_tc(const csa_dims* d, const IndexerArgs& a, int B, int cap, float* scratch,
                                     cudaStream_t st) {
+  CSA_RANGE("A4 indexer_topk (decode)");
   CUtensorMap tk, tq;
   if (!make_tmap_bf16(&tk, a.KI, d->cI, (uint64_t)B * cap, (uint64_t)d->cI * 2, 64, idxdec::kM) ||
       !make_tmap_bf16_3d(&tq, a.qI, d->cI, d->nhI, B, (uint64_t)d->cI * 2, (uint64_t)a.ld_qI * 2, 64, d->nhI, 1))
@@ -878,6 +904,7 @@ size_t csa_decode_workspace_bytes(const csa_dims* d, int B, int cap) {
 csa_status csa_decode(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
                       void* Ccache, void* KIcache, int* cache_len, int cap, int B, void* O, int* idx_out,
                       void* ws, size_t ws_bytes, void* stream) {
+  CSA_RANGE("csa_decode");
   csa_status s = check_dims(d);
   if (s != CSA_OK) return s;
   if (!packed || !h || !pos || !ring || !Ccache || !KIcache || !cache_len || !O || !ws) return CSA_ERR_INVALID_ARG;
