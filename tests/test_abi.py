@@ -85,3 +85,42 @@ def test_misaligned_workspace_rejected():
     p = ctypes.c_void_p(1 << 20)
     q = ctypes.c_void_p((1 << 20) + 128)
     assert L.csa_forward(d, p, p, p, p, 1, 256, 64, 256, p, None, None, None, q, 1 << 30, None) == 1
+
+
+def test_every_stage_rejects_null_pointers_before_any_launch():
+    """Each stage entry checks its pointers on the host: a null buffer is
+    CSA_ERR_INVALID_ARG and nothing is launched."""
+    L = csa.lib()
+    d = ctypes.byref(TINY.c_struct())
+    n0 = csa.csa_launch_count()
+    assert L.csa_pack_weights(d, None, None, 0, None) == 1
+    assert L.csa_project_hidden(d, None, None, 64, None, None, None) == 1
+    assert L.csa_project_query(d, None, None, 128, 64, None, None) == 1
+    assert L.csa_compress_kv(d, None, None, 64, None, None, 1, 16, None, None, None) == 1
+    assert L.csa_indexer_topk(d, None, 128, None, 4, None, None, None, 1, 256, 64, 256, None, None, 0, None) == 1
+    assert L.csa_indexer_topk_noalloc(d, None, 128, None, 4, None, None, None, 1, 256, 64, 256, None, None) == 1
+    assert L.csa_sparse_mqa(d, None, 512, None, None, None, None, 1, 256, 64, None, None) == 1
+    assert L.csa_cache_append(d, None, None, None, None, None, None, None, 10, 1, None) == 1
+    assert csa.csa_launch_count() == n0
+
+
+def test_decode_workspace_too_small_rejected():
+    L = csa.lib()
+    d = ctypes.byref(TINY.c_struct())
+    p = ctypes.c_void_p(1 << 20)   # 1024-aligned fake address; nothing is launched
+    need = csa.csa_decode_workspace_bytes(TINY, 3, 40)
+    n0 = csa.csa_launch_count()
+    assert L.csa_decode(d, p, p, p, p, p, p, p, 40, 3, p, None, p, need - 1, None) == 7
+    assert csa.csa_launch_count() == n0
+
+
+def test_decode_workspace_holds_scores_and_split_sums():
+    """The decode workspace covers the [B, cap] fp32 scores and the four fp32
+    K-slices of the hidden-side projection ([slice][token][feature], features
+    padded to 128)."""
+    dims = csa.Dims(d=4096, c=512, m=4, cI=128, nhI=64, nh=128, dc=1536, topk=2048, dtype=csa.CSA_BF16)
+    B, cap = 64, 16384
+    n1 = 4 * dims.c + 4 * dims.cI + dims.dc + dims.nhI
+    n1p = (n1 + 127) // 128 * 128
+    assert csa.csa_decode_workspace_bytes(dims, B, cap) >= B * cap * 4 + 4 * n1p * B * 4
+    assert csa.csa_decode_workspace_bytes(dims, 2 * B, cap) > csa.csa_decode_workspace_bytes(dims, B, cap)
