@@ -150,7 +150,6 @@ class ClockSampler:
 # figure stale: it is then removed until the next capture.
 MEASURED_TRAFFIC = {
     ("prefill", "A4_indexer_topk"): 102_976_512 + 7_183_104,
-    ("prefill", "A5_sparse_mqa"): 556_155_904 + 491_758_336,
 }
 
 
