@@ -145,9 +145,9 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ timing helpers
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
-# a stage's kernel, from one ncu capture of the current kernel version on the
-# named workload (profiles/<kernel>_<workload>.md).  A kernel change makes the
-# figure stale: it is then removed until the next capture.
+# a stage's kernel, taken from one ncu capture of the current kernel version
+# on the named workload.  A kernel change makes the figure stale: it is then
+# removed until the kernel is captured again.
 MEASURED_TRAFFIC = {
     ("prefill", "A4_indexer_topk"): 102_976_512 + 7_183_104,
 }
@@ -166,7 +166,7 @@ def timed_steps(fn, steps, flush, stream):
 
 
 class PrefillRunner:
-    def __init__(self, w, dev):
+    def __init__(self, w, dev, stage_buffers=True):
         self.w, self.dims, self.dev = w, w.dims, dev
         d = self.dims
         self.T = sum(w.seqlens)
@@ -183,9 +183,11 @@ class PrefillRunner:
         self.cu, self.cb = cu.to(dev), cb.to(dev)
         dt = self.H.dtype
         self.O = torch.empty(self.T, d.nh * d.c, dtype=dt, device=dev)
-        self.O_host = None   # pinned host copy of O, made on first end-to-end use
+        self.e2e_bufs = None   # second H / O buffers, pinned host O and copy streams, made on first use
         self.ws = torch.empty(csa.csa_forward_workspace_bytes(d, self.T, self.nseq), dtype=torch.uint8,
                               device=dev)
+        if not stage_buffers:
+            return
         # stage buffers (separate from the workspace so stages can be timed one by one)
         self.Y1 = torch.empty(self.T, csa.csa_hidden_row_elems(d), dtype=dt, device=dev)
         self.wI = torch.empty(self.T, d.nhI, dtype=torch.float32, device=dev)
@@ -196,17 +198,56 @@ class PrefillRunner:
         self.iws = torch.empty(csa.csa_indexer_workspace_bytes(d, self.T, self.nseq, self.maxlen), dtype=torch.uint8,
                                device=dev)
 
-    def forward(self):
+    def forward(self, H=None, O=None):
         d = self.dims
-        csa.csa_forward(d, self.packed, self.H, self.cu, self.cb, self.nseq, self.T, self.NB, self.maxlen,
-                        self.O, None, None, None, self.ws)
+        csa.csa_forward(d, self.packed, self.H if H is None else H, self.cu, self.cb, self.nseq, self.T, self.NB,
+                        self.maxlen, self.O if O is None else O, None, None, None, self.ws)
 
-    def forward_e2e(self):
-        if self.O_host is None:
-            self.O_host = torch.empty(self.T, self.dims.nh * self.dims.c, dtype=self.O.dtype).pin_memory()
-        self.H.copy_(self.H_host, non_blocking=True)
-        self.forward()
-        self.O_host.copy_(self.O, non_blocking=True)
+    def forward_staged(self, events):
+        d = self.dims
+        csa.csa_forward_staged(d, self.packed, self.H, self.cu, self.cb, self.nseq, self.T, self.NB, self.maxlen,
+                               self.O, None, None, None, self.ws, events)
+
+    def e2e_pipeline(self, steps, flush):
+        """`steps` end-to-end steps through host buffers; returns the device
+        time in ms from the first step's H2D copy to the last step's D2H copy.
+        Step i copies H from pinned host memory into device buffer i % 2 (copy
+        stream), runs the forward on the compute stream into O buffer i % 2,
+        and copies that O to pinned host memory (second copy stream), so that
+        step i's forward overlaps step i+1's H2D and step i-1's D2H.  The L2
+        is flushed before every forward."""
+        if self.e2e_bufs is None:
+            self.e2e_bufs = {"H": [self.H, torch.empty_like(self.H)], "O": [self.O, torch.empty_like(self.O)],
+                             "O_host": torch.empty(self.O.shape, dtype=self.O.dtype).pin_memory(),
+                             "s_in": torch.cuda.Stream(), "s_out": torch.cuda.Stream()}
+        b = self.e2e_bufs
+        comp, s_in, s_out = torch.cuda.current_stream(), b["s_in"], b["s_out"]
+        ready = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        freed = [torch.cuda.Event() for _ in range(2)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(s_in)
+        for i in range(steps):
+            k = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done[k])        # step i-2's forward has read H[k]
+                b["H"][k].copy_(self.H_host, non_blocking=True)
+                ready[k].record(s_in)
+            comp.wait_event(ready[k])
+            if i >= 2:
+                comp.wait_event(freed[k])           # step i-2's D2H has read O[k]
+            flush()
+            self.forward(b["H"][k], b["O"][k])
+            done[k].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[k])
+                b["O_host"].copy_(b["O"][k], non_blocking=True)
+                freed[k].record(s_out)
+        end.record(s_out)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
 
     def stages(self):
         d, T = self.dims, self.T
@@ -260,6 +301,10 @@ class DecodeRunner:
         csa.csa_decode(self.dims, self.packed, self.h, self.pos, self.ring, self.Cc, self.Kc, self.clen,
                        self.cap, self.B, self.O, None, self.ws)
 
+    def step_staged(self, events):
+        csa.csa_decode_staged(self.dims, self.packed, self.h, self.pos, self.ring, self.Cc, self.Kc, self.clen,
+                              self.cap, self.B, self.O, None, self.ws, events)
+
     def bytes_per_step(self):
         d = self.dims
         N1 = 4 * d.c + 4 * d.cI + d.dc + d.nhI
@@ -274,13 +319,13 @@ class DecodeRunner:
 
 # ------------------------------------------------------------------ oracle baseline
 class OracleSampler:
-    """Times the fp64 oracle on bounded samples of a workload, extrapolated to
-    tokens/s.  The per-token part (projections of every token and the
-    compression) is timed once in full by `base()`; each `sample()` then runs
-    one oracle forward with eqs. 5-11 on `rows_sample` seeded query rows and
-    extrapolates its per-row cost to every row."""
+    """Times the fp64 oracle on bounded samples of a workload.  The
+    token-parallel half (eqs. 1-4: projections and compression of every
+    token) is timed once in full by `base()`; `rows(n, seed)` times the
+    per-query half (eqs. 5-11) on n seeded query rows, on its own.  The
+    whole-workload rate is then T / (base + per-row cost x T)."""
 
-    def __init__(self, w, rows_sample):
+    def __init__(self, w):
         from oracle import csa_oracle as orc
         self.orc, self.w = orc, w
         d = w.dims
@@ -289,32 +334,61 @@ class OracleSampler:
         self.H = synth.make_hidden(self.T, d, w.seed).double().numpy()
         self.od = dict(m=d.m, topk=d.topk, nh=d.nh, nhI=d.nhI, c=d.c, cI=d.cI)
         self.store = "bf16" if d.dtype == csa.CSA_BF16 else "f32"
-        self.rows_sample = min(rows_sample, self.T)
         self.base_s = None
-
-    def _forward(self, rows):
-        t0 = time.perf_counter()
-        self.orc.csa_forward(self.H, self.W, self.od, list(self.w.seqlens), store=self.store, rows=rows)
-        return time.perf_counter() - t0
+        self.entries = None
 
     def base(self):
-        self.base_s = self._forward(np.zeros(0, dtype=np.int64))
+        t0 = time.perf_counter()
+        self.entries = self.orc.compressed_entries(self.H, self.W, self.od, list(self.w.seqlens), self.store)
+        self.base_s = time.perf_counter() - t0
         return self.base_s
 
-    def sample(self, seed):
-        if self.base_s is None:
+    def rows(self, n, seed):
+        """Seconds the per-query half takes on n seeded rows (distinct, sorted)."""
+        if self.entries is None:
             self.base()
-        rows = np.sort(np.random.default_rng(seed).choice(self.T, size=self.rows_sample, replace=False))
-        t = self._forward(rows)
-        per_row = max(t - self.base_s, 0.0) / len(rows)
-        return self.T / (self.base_s + per_row * self.T), dict(base_s=self.base_s, per_row_s=per_row,
-                                                               rows=len(rows), wall_s=t)
+        rows = np.sort(np.random.default_rng(seed).choice(self.T, size=min(n, self.T), replace=False))
+        Cc, Kc, cu, cb = self.entries
+        t0 = time.perf_counter()
+        self.orc.query_rows(self.H, self.W, self.od, Cc, Kc, cu, cb, rows, self.store)
+        return time.perf_counter() - t0, len(rows)
+
+    def tokens_per_s(self, per_row_s):
+        return self.T / (self.base_s + per_row_s * self.T)
 
 
-def oracle_sample(w, rows_sample, seed=0):
-    """One bounded oracle sample of the workload (base part timed in full,
-    eqs. 5-11 on `rows_sample` rows), extrapolated to tokens/s."""
-    return OracleSampler(w, rows_sample).sample(seed)
+def oracle_baseline(w, budget_s=15.0, chunk=16):
+    """cpu_baseline of the default line: the token-parallel half in full, then
+    seeded query rows in chunks until about budget_s of row time (at least
+    two chunks); per-row cost = row time / rows, measured, not differenced."""
+    smp = OracleSampler(w)
+    smp.base()
+    t_rows, n_rows, seed = 0.0, 0, 0
+    while (t_rows < budget_s or seed < 2) and n_rows < smp.T:
+        dt, n = smp.rows(chunk, seed)
+        t_rows += dt
+        n_rows += n
+        seed += 1
+    per_row = t_rows / n_rows
+    return smp.tokens_per_s(per_row), dict(base_s=smp.base_s, per_row_s=per_row, rows=n_rows, rows_s=t_rows)
+
+
+def oracle_tiny_one_thread():
+    """The tiny fp32 workload, whole forward (every row), on one BLAS thread."""
+    from threadpoolctl import threadpool_limits
+    from oracle import csa_oracle as orc
+    w = synth.workloads()["tiny"]
+    d = w.dims
+    W = {k: v.double().numpy() for k, v in synth.make_weights(d, w.seed).items()}
+    T = sum(w.seqlens)
+    H = synth.make_hidden(T, d, w.seed).double().numpy()
+    od = dict(m=d.m, topk=d.topk, nh=d.nh, nhI=d.nhI, c=d.c, cI=d.cI)
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        orc.csa_forward(H, W, od, list(w.seqlens), store="f32")
+        dt = time.perf_counter() - t0
+    return {"value": T / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"tiny fp32 workload ({T} tokens), whole forward, every row, one BLAS thread ({dt:.2f} s)"}
 
 
 def blas_threads():
@@ -347,20 +421,22 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     w = synth.workloads()[args.workload]
-    sampler = OracleSampler(w, args.ref_rows)
-    sampler.base()                      # the token-parallel part, timed in full once
-    times = []
-    info = None
+    smp = OracleSampler(w)
+    smp.base()                      # the token-parallel half, timed in full once, before the steps
+    values, step_s = [], []
     for i in range(args.warmup + args.steps):
-        tps, info = sampler.sample(seed=i)
+        dt, n = smp.rows(args.ref_rows, seed=i)
         if i >= args.warmup:
-            times.append(tps)
-    value = statistics.mean(times)
-    sample = (f"oracle forward per step with eqs. 5-11 on {info['rows']} seeded query rows, extrapolated "
-              f"to all {sum(w.seqlens)} rows; projections + compression of every token timed in full "
-              f"({info['base_s']:.2f} s) before the steps")
+            values.append(smp.tokens_per_s(dt / n))
+            step_s.append(dt)
+    value = statistics.mean(values)
+    T = sum(w.seqlens)
+    sample = (f"each step: the oracle's per-query half (eqs. 5-11) on {args.ref_rows} seeded query rows, timed "
+              f"on its own ({1e3 * statistics.mean(step_s) / args.ref_rows:.1f} ms/row); the token-parallel half "
+              f"(eqs. 1-4, all {T} tokens) timed in full once before the steps ({smp.base_s:.2f} s); value = "
+              f"{T} / (that + per-row cost x {T}); ms_per_step = the measured sampled step")
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1000.0 * sum(w.seqlens) / value, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(step_s), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": workload_config(w, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
@@ -379,13 +455,123 @@ def workload_config(w, world):
             "l2": "flushed before every timed step (512 MiB write)"}
 
 
+def stage_entry(name, ms, work, peaks, peak_key="bf16"):
+    """Roofline record of one stage timed for `ms` milliseconds."""
+    bound, amount = work[name]
+    if bound == "hbm":
+        ach = amount / (ms / 1000.0) / 1e9
+        return {"ms": ms, "bound": "hbm", "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": ach / peaks["hbm"], "algorithmic": amount}
+    ach = amount / (ms / 1000.0) / 1e12
+    return {"ms": ms, "bound": "tensor", "achieved": ach, "peak": peaks[peak_key], "unit": "TFLOP/s",
+            "frac": ach / peaks[peak_key], "algorithmic": amount}
+
+
+STAGES = ("A1_project_hidden", "A2_project_query", "A3_compress", "A4_indexer_topk", "A5_sparse_mqa")
+
+
+def staged_step_ms(step_fn, nstages, steps, flush, stream):
+    """Mean in-step duration of each stage over `steps` steps of step_fn(events)
+    (L2 flushed before each step; events recorded between the stages)."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstages + 1)] for _ in range(steps)]
+    for ev in evs:
+        for e in ev:
+            e.record(stream)   # creates the handles
+    torch.cuda.synchronize()
+    for ev in evs:
+        flush()
+        step_fn(ev)
+    torch.cuda.synchronize()
+    return [statistics.mean(ev[k].elapsed_time(ev[k + 1]) for ev in evs) for k in range(nstages)]
+
+
+def measure_stages(runner, w, args, peaks, flush, stream, reps):
+    """Each stage timed alone (inputs from one pass of the stages), and the
+    same stages timed inside the real step (csa_forward_staged)."""
+    work = stage_work(w.dims, w.seqlens)
+    alone = {}
+    for name, fn in runner.stages().items():
+        for _ in range(2):
+            fn()
+        alone[name] = stage_entry(name, statistics.mean(timed_steps(fn, reps, flush, stream)), work, peaks)
+    in_step_ms = staged_step_ms(runner.forward_staged, len(STAGES), reps, flush, stream)
+    in_step = {n: stage_entry(n, ms, work, peaks, "bf16_sustained") for n, ms in zip(STAGES, in_step_ms)}
+    st = csa.csa_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after stages: {csa.status_string(st)}")
+    return alone, in_step
+
+
+def decode_stage_bytes(w):
+    """Algorithmic HBM bytes of each stage of one decode step."""
+    d = w.dims
+    B, avail = w.decode_batch, w.decode_pos // d.m
+    es = 2
+    N1 = 4 * d.c + 4 * d.cI + d.dc + d.nhI
+    N2 = d.nhI * d.cI + d.nh * d.c
+    ring = 4 * d.c + 4 * d.cI
+    return {
+        "A1_project_hidden": d.d * N1 * es + B * d.d * es + B * N1 * es,
+        "A6_cache_append": B * (2 * d.m * ring * es + (d.c + d.cI) * es),
+        "A2_project_query": d.dc * N2 * es + B * d.dc * es + B * N2 * es,
+        "A4_indexer_scores": B * avail * d.cI * es + B * avail * 4,
+        "A4_topk_select": B * avail * 4 + B * d.topk * 4,
+        "A5_sparse_mqa": B * min(d.topk, avail) * d.c * es + 2 * B * d.nh * d.c * es + B * d.topk * 4,
+    }
+
+
+def run_decode(dev, args, peaks, flush, stream):
+    w = synth.workloads()["decode"]
+    dr = DecodeRunner(w, dev)
+    for _ in range(3):
+        dr.step()
+    dms = statistics.mean(timed_steps(dr.step, args.steps, flush, stream))
+    names = ("A1_project_hidden", "A6_cache_append", "A2_project_query", "A4_indexer_scores", "A4_topk_select",
+             "A5_sparse_mqa")
+    in_step_ms = staged_step_ms(dr.step_staged, len(names), max(3, min(args.steps, 50)), flush, stream)
+    st = csa.csa_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after decode: {csa.status_string(st)}")
+    nbytes = decode_stage_bytes(w)
+    stages = {}
+    for n, ms in zip(names, in_step_ms):
+        gbs = nbytes[n] / (ms / 1000.0) / 1e9
+        stages[n] = {"ms": ms, "bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm"], "algorithmic_bytes": nbytes[n]}
+    gbs = dr.bytes_per_step() / (dms / 1000.0) / 1e9
+    out = {"value": dr.B / (dms / 1000.0), "unit": "tokens/s", "ms_per_step": dms,
+           "workload": "64 sequences x 1 new token over 16384 cached entries (t=65536), nh=128, k=2048",
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                        "frac": gbs / peaks["hbm"], "algorithmic_bytes": dr.bytes_per_step()},
+           "stages_in_step": stages}
+    del dr
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_extra_workload(name, dev, args, peaks, flush, stream):
+    """Step time, throughput and per-stage rooflines of another prefill workload."""
+    w = synth.workloads()[name]
+    runner = PrefillRunner(w, dev, stage_buffers=True)
+    for _ in range(3):
+        runner.forward()
+    steps = max(3, min(args.steps, 5))
+    ms = statistics.mean(timed_steps(runner.forward, steps, flush, stream))
+    alone, in_step = measure_stages(runner, w, args, peaks, flush, stream, 3)
+    out = {"workload": workload_config(w, 1)["workload"], "tokens": runner.T, "steps": steps, "ms_per_step": ms,
+           "value": runner.T / (ms / 1000.0), "unit": "tokens/s", "stages": alone, "stages_in_step": in_step}
+    del runner
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
     peaks = load_peaks()
     w = synth.workloads()[args.workload]
-    runner = PrefillRunner(w, dev)
+    runner = PrefillRunner(w, dev, stage_buffers=not args.no_stages)
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def flush():
@@ -417,43 +603,27 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     clocks = sampler.stop(t_sample0, t_sample1)
     total_ms = max_over_ranks(sum(step_ms), dev, world)
-    tokens = runner.T * args.steps * world
     value = job_throughput(runner.T, args.steps, world, total_ms)
     ms_per_step = total_ms / args.steps
 
-    # ---- end to end through host buffers (H2D of H, forward, D2H of O)
+    # ---- end to end through host buffers: every step copies its H in from
+    # pinned host memory and its O out to pinned host memory; the copies run
+    # on their own streams, overlapped with the neighbouring steps' compute
     e2e = None
     if not args.no_e2e:
-        for _ in range(2):
-            runner.forward_e2e()
-        e2e_ms = max_over_ranks(sum(timed_steps(runner.forward_e2e, args.steps, flush, stream)), dev, world)
-        e2e = {"value": tokens / (e2e_ms / 1000.0), "unit": "tokens/s",
+        runner.e2e_pipeline(2, flush)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(runner.e2e_pipeline(args.steps, flush), dev, world)
+        e2e = {"value": runner.T * args.steps * world / (e2e_ms / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": runner.H.numel() * runner.H.element_size(),
-               "d2h_bytes_per_step": runner.O.numel() * runner.O.element_size()}
+               "d2h_bytes_per_step": runner.O.numel() * runner.O.element_size(),
+               "how": "H2D of step i+1 and D2H of step i-1 on copy streams, overlapped with step i's forward; "
+                      "timed from the first H2D to the last D2H"}
 
-    # ---- stages, each timed alone (per-stage roofline)
-    stages = {}
-    work = stage_work(w.dims, w.seqlens)
+    # ---- stages: each alone (per-stage roofline) and inside the step
+    stages, stages_in_step = {}, {}
     if not args.no_stages:
-        fns = runner.stages()
-        for name, fn in fns.items():
-            for _ in range(2):
-                fn()
-            ms = statistics.mean(timed_steps(fn, max(3, min(args.steps, 10)), flush, stream))
-            bound, amount = work[name]
-            if bound == "hbm":
-                ach = amount / (ms / 1000.0) / 1e9
-                peak = peaks["hbm"]
-                stages[name] = {"ms": ms, "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                                "frac": ach / peak, "algorithmic": amount}
-            else:
-                ach = amount / (ms / 1000.0) / 1e12
-                peak = peaks["bf16"]
-                stages[name] = {"ms": ms, "bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                                "frac": ach / peak, "algorithmic": amount}
-        st = csa.csa_get_device_status()
-        if st != 0:
-            raise RuntimeError(f"device status after stages: {csa.status_string(st)}")
+        stages, stages_in_step = measure_stages(runner, w, args, peaks, flush, stream, max(3, min(args.steps, 10)))
     roofline = None
     if stages:
         top = max(stages, key=lambda k: stages[k]["ms"])
@@ -461,32 +631,28 @@ def run_ours(args, rank, world, local_rank):
         roofline = {"kernel": top, "bound": s["bound"], "achieved": s["achieved"], "peak": s["peak"],
                     "unit": s["unit"], "frac": s["frac"], "traffic": MEASURED_TRAFFIC.get((args.workload, top)),
                     "peak_source": f"{peaks['source']} ({'hbm_gbs' if s['bound'] == 'hbm' else 'bf16_tflops'})"}
+    del runner
+    torch.cuda.empty_cache()
 
     # ---- decode workload, same build
-    decode = None
-    if not args.no_decode:
-        del runner
-        torch.cuda.empty_cache()
-        dr = DecodeRunner(synth.workloads()["decode"], dev)
-        for _ in range(3):
-            dr.step()
-        dms = statistics.mean(timed_steps(dr.step, args.steps, flush, stream))
-        st = csa.csa_get_device_status()
-        if st != 0:
-            raise RuntimeError(f"device status after decode: {csa.status_string(st)}")
-        gbs = dr.bytes_per_step() / (dms / 1000.0) / 1e9
-        decode = {"value": dr.B / (dms / 1000.0), "unit": "tokens/s", "ms_per_step": dms,
-                  "workload": "64 sequences x 1 new token over 16384 cached entries (t=65536), nh=128, k=2048",
-                  "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                               "frac": gbs / peaks["hbm"], "algorithmic_bytes": dr.bytes_per_step()}}
+    decode = None if args.no_decode else run_decode(dev, args, peaks, flush, stream)
+
+    # ---- the long and ragged prefill workloads (step, stages, rooflines)
+    workloads = {}
+    if not args.no_workloads and world == 1:
+        for name in ("long", "ragged"):
+            if name != args.workload:
+                workloads[name] = run_extra_workload(name, dev, args, peaks, flush, stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tps, info = oracle_sample(w, rows_sample=args.ref_rows)
+        tps, info = oracle_baseline(w, budget_s=args.cpu_budget)
         cpu = {"value": tps, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": (f"projections + compression of all {runner_T(w)} tokens in full "
-                          f"({info['base_s']:.1f} s), eqs. 5-11 on {info['rows']} seeded query rows "
-                          f"({info['per_row_s'] * 1e3:.1f} ms/row), extrapolated")}
+               "sample": (f"token-parallel half (eqs. 1-4) of all {runner_T(w)} tokens in full "
+                          f"({info['base_s']:.1f} s), per-query half (eqs. 5-11) timed on its own on "
+                          f"{info['rows']} seeded query rows ({info['per_row_s'] * 1e3:.1f} ms/row), "
+                          f"tokens/s = T / (base + per-row x T)"),
+               "tiny_1thread": oracle_tiny_one_thread()}
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -494,7 +660,8 @@ def run_ours(args, rank, world, local_rank):
                 "vs_baseline": None, "dtype": "bf16" if w.dims.dtype == csa.CSA_BF16 else "f32",
                 "data": "synthetic (seeded normal H, N(0,1/fan_in) weights)", "config": workload_config(w, world),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clocks, "stages": stages, "decode": decode}
+                "clocks": clocks, "stages": stages, "stages_in_step": stages_in_step, "decode": decode,
+                "workloads": workloads}
         print(json.dumps(line), flush=True)
 
 
@@ -532,7 +699,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["prefill", "tiny", "long", "ragged"], default="prefill")
-    ap.add_argument("--ref-rows", type=int, default=64, help="query rows the oracle runs per sample")
+    ap.add_argument("--ref-rows", type=int, default=16, help="query rows the reference arm runs per step")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle row time for cpu_baseline")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the long and ragged workload lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-stages", action="store_true")
     ap.add_argument("--no-decode", action="store_true")

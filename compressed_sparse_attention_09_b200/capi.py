@@ -27,6 +27,7 @@ EXPORTS = (
     "csa_cache_append", "csa_decode_workspace_bytes", "csa_decode", "csa_get_device_status",
     "csa_status_string", "csa_hidden_row_elems", "csa_query_row_elems", "csa_project_hidden",
     "csa_project_query", "csa_launch_count", "csa_indexer_workspace_bytes", "csa_indexer_topk_noalloc",
+    "csa_set_wait_limit_ns", "csa_check_wait_timeout", "csa_forward_staged", "csa_decode_staged",
 )
 
 
@@ -98,6 +99,10 @@ def lib() -> ctypes.CDLL:
             "csa_project_hidden": (i, [D, vp, vp, i, vp, vp, vp]),
             "csa_project_query": (i, [D, vp, vp, i, i, vp, vp]),
             "csa_launch_count": (ctypes.c_uint64, []),
+            "csa_set_wait_limit_ns": (i, [ctypes.c_ulonglong]),
+            "csa_forward_staged": (i, [D, vp, vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp, vp]),
+            "csa_decode_staged": (i, [D, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, sz, vp, vp]),
+            "csa_check_wait_timeout": (i, [vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -247,3 +252,39 @@ def csa_launch_count() -> int:
 def csa_get_device_status(stream=None) -> int:
     """Status code (0 = CSA_OK) of the conditions kernels recorded; syncs the stream."""
     return lib().csa_get_device_status(_stream(stream))
+
+
+def csa_set_wait_limit_ns(ns: int):
+    """Limit of every bounded device wait on the current device (ns)."""
+    _check(lib().csa_set_wait_limit_ns(int(ns)), "csa_set_wait_limit_ns")
+
+
+def csa_check_wait_timeout(out, stream=None):
+    """Enqueues the bounded-wait self-check kernel; out: 3 x int64 on the device."""
+    _check(lib().csa_check_wait_timeout(_p(out), _stream(stream)), "csa_check_wait_timeout")
+
+
+def _event_array(events):
+    """ctypes array of cudaEvent_t handles from torch.cuda.Event objects (each
+    recorded once beforehand, so that its handle exists)."""
+    arr = (ctypes.c_void_p * len(events))()
+    for k, e in enumerate(events):
+        arr[k] = e.cuda_event if hasattr(e, "cuda_event") else int(e)
+    return arr
+
+
+def csa_forward_staged(dims: Dims, packed, H, cu_seqlens, cu_blocks, nseq, total_tokens, total_blocks, max_seqlen,
+                       O, Ccomp_out, KI_out, idx_out, ws, events, stream=None):
+    """csa_forward recording events[0..5] around its five stages."""
+    _check(lib().csa_forward_staged(_d(dims), _p(packed), _p(H), _p(cu_seqlens), _p(cu_blocks), nseq,
+                                    total_tokens, total_blocks, max_seqlen, _p(O), _p(Ccomp_out), _p(KI_out),
+                                    _p(idx_out), _p(ws), ws.numel() * ws.element_size(), _event_array(events),
+                                    _stream(stream)), "csa_forward_staged")
+
+
+def csa_decode_staged(dims: Dims, packed, h, pos, ring, Ccache, KIcache, cache_len, cap, B, O, idx_out, ws, events,
+                      stream=None):
+    """csa_decode recording events[0..6] around its stages."""
+    _check(lib().csa_decode_staged(_d(dims), _p(packed), _p(h), _p(pos), _p(ring), _p(Ccache), _p(KIcache),
+                                   _p(cache_len), cap, B, _p(O), _p(idx_out), _p(ws), ws.numel() * ws.element_size(),
+                                   _event_array(events), _stream(stream)), "csa_decode_staged")

@@ -21,6 +21,11 @@ __device__ unsigned g_status;
 
 __device__ __forceinline__ void flag_status(unsigned bits) { atomicOr(&g_status, bits); }
 
+// Limit of every bounded device wait, in ns of %globaltimer (set per device
+// by csa_set_wait_limit_ns; read by a wait when its first poll fails).
+constexpr unsigned long long kDefaultWaitNs = 1500000000ull;   // 1.5 s
+__device__ unsigned long long g_wait_ns = kDefaultWaitNs;
+
 // ---------------------------------------------------------------- conversions
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }

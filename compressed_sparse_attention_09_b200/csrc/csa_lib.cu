@@ -22,6 +22,7 @@
 #include "mqa_simt.cuh"
 #include "mqa_tcgen05.cuh"
 #include "pack.cuh"
+#include "selfcheck.cuh"
 
 using namespace csa;
 using bf16 = __nv_bfloat16;
@@ -509,6 +510,19 @@ csa_status csa_get_device_status(void* stream) {
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+csa_status csa_set_wait_limit_ns(unsigned long long ns) {
+  if (ns < 1000ull || ns > 60000000000ull) return CSA_ERR_INVALID_ARG;
+  if (cudaMemcpyToSymbol(g_wait_ns, &ns, sizeof(ns)) != cudaSuccess) return CSA_ERR_CUDA;
+  return CSA_OK;
+}
+
+csa_status csa_check_wait_timeout(unsigned long long* out, void* stream) {
+  if (!out || reinterpret_cast<uintptr_t>(out) % 8) return CSA_ERR_INVALID_ARG;
+  wait_selfcheck_kernel<<<1, 64, 0, (cudaStream_t)stream>>>(out);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
 int csa_hidden_row_elems(const csa_dims* d) {
   if (check_dims(d) != CSA_OK) return 0;
   return pack_layout(d).N1b;
@@ -743,10 +757,19 @@ size_t csa_forward_workspace_bytes(const csa_dims* d, int total_tokens, int nseq
   return fwd_layout(d, total_tokens).total;
 }
 
-csa_status csa_forward(const csa_dims* d, const void* packed, const void* H, const int* cu_seqlens,
-                       const int* cu_blocks, int nseq, int total_tokens, int total_blocks, int max_seqlen,
-                       void* O, void* Ccomp_out, void* KI_out, int* idx_out, void* ws, size_t ws_bytes,
-                       void* stream) {
+}  // extern "C"
+
+namespace {
+// Records events[i] on st when a stage-event array was given (staged entries).
+inline csa_status mark(void* const* events, int i, cudaStream_t st) {
+  if (events && cudaEventRecord((cudaEvent_t)events[i], st) != cudaSuccess) return CSA_ERR_CUDA;
+  return CSA_OK;
+}
+
+csa_status forward_impl(const csa_dims* d, const void* packed, const void* H, const int* cu_seqlens,
+                        const int* cu_blocks, int nseq, int total_tokens, int total_blocks, int max_seqlen,
+                        void* O, void* Ccomp_out, void* KI_out, int* idx_out, void* ws, size_t ws_bytes,
+                        void* const* ev, void* stream) {
   CSA_RANGE("csa_forward");
   csa_status s = check_dims(d);
   if (s != CSA_OK) return s;
@@ -772,13 +795,14 @@ csa_status csa_forward(const csa_dims* d, const void* packed, const void* H, con
   void* KIc = KI_out ? KI_out : at(ws, L.kicomp);
   int* idx = idx_out ? idx_out : reinterpret_cast<int*>(at(ws, L.idx));
 
+  if ((s = mark(ev, 0, st)) != CSA_OK) return s;
   s = project_hidden(d, packed, H, T, y1, wI, st);
-  if (s != CSA_OK) return s;
+  if (s != CSA_OK || (s = mark(ev, 1, st)) != CSA_OK) return s;
   s = project_query(d, packed, y1 + (size_t)(4 * c + 4 * cI) * es, P.N1b, T, y2, st);
-  if (s != CSA_OK) return s;
+  if (s != CSA_OK || (s = mark(ev, 2, st)) != CSA_OK) return s;
   // A3: eqs. (3), (4) for C^Comp and K^IComp in one launch
   s = compress_kv(d, packed, y1, T, cu_seqlens, cu_blocks, nseq, NB, Cc, KIc, st);
-  if (s != CSA_OK) return s;
+  if (s != CSA_OK || (s = mark(ev, 3, st)) != CSA_OK) return s;
   // A4: eqs. (8), (9)
   IndexerArgs ia;
   ia.qI = y2; ia.ld_qI = P.N2; ia.wI = wI; ia.ld_wI = d->nhI; ia.KI = KIc; ia.idx = idx;
@@ -791,14 +815,38 @@ csa_status csa_forward(const csa_dims* d, const void* packed, const void* H, con
   } else {
     s = launch_indexer(d, ia, T, st);
   }
-  if (s != CSA_OK) return s;
+  if (s != CSA_OK || (s = mark(ev, 4, st)) != CSA_OK) return s;
   // A5: eq. (11)
   MqaArgs ma;
   ma.q = y2 + (size_t)d->nhI * cI * es; ma.ld_q = P.N2; ma.C = Cc; ma.idx = idx;
   ma.O = O; ma.ld_O = (long long)d->nh * c; ma.topk = d->topk; ma.nh = d->nh;
   ma.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c));
   ma.rm = RowMap{cu_seqlens, cu_blocks, nseq, NB, nullptr, 0, d->m};
-  return launch_mqa(d, ma, T, st);
+  s = launch_mqa(d, ma, T, st);
+  if (s != CSA_OK) return s;
+  return mark(ev, 5, st);
+}
+}  // namespace
+
+extern "C" {
+
+csa_status csa_forward(const csa_dims* d, const void* packed, const void* H, const int* cu_seqlens,
+                       const int* cu_blocks, int nseq, int total_tokens, int total_blocks, int max_seqlen,
+                       void* O, void* Ccomp_out, void* KI_out, int* idx_out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  return forward_impl(d, packed, H, cu_seqlens, cu_blocks, nseq, total_tokens, total_blocks, max_seqlen, O,
+                      Ccomp_out, KI_out, idx_out, ws, ws_bytes, nullptr, stream);
+}
+
+csa_status csa_forward_staged(const csa_dims* d, const void* packed, const void* H, const int* cu_seqlens,
+                              const int* cu_blocks, int nseq, int total_tokens, int total_blocks, int max_seqlen,
+                              void* O, void* Ccomp_out, void* KI_out, int* idx_out, void* ws, size_t ws_bytes,
+                              void* const* events, void* stream) {
+  if (!events) return CSA_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i)
+    if (!events[i]) return CSA_ERR_INVALID_ARG;
+  return forward_impl(d, packed, H, cu_seqlens, cu_blocks, nseq, total_tokens, total_blocks, max_seqlen, O,
+                      Ccomp_out, KI_out, idx_out, ws, ws_bytes, events, stream);
 }
 
 // ------------------------------------------------------------------ decode
@@ -860,7 +908,7 @@ DecLayout dec_layout(const csa_dims* d, int B, int cap) {
 // Decode rows through the tensor-core indexer: split-s scores into the
 // workspace, then one selection CTA per sequence.
 csa_status launch_indexer_decode_tc(const csa_dims* d, const IndexerArgs& a, int B, int cap, float* scratch,
-                                    cudaStream_t st) {
+                                    cudaStream_t st, cudaEvent_t after_scores = nullptr) {
   CSA_RANGE("A4 indexer_topk (decode)");
   CUtensorMap tk, tq;
   if (!make_tmap_bf16(&tk, a.KI, d->cI, (uint64_t)B * cap, (uint64_t)d->cI * 2, 64, idxdec::kM) ||
@@ -876,6 +924,7 @@ csa_status launch_indexer_decode_tc(const csa_dims* d, const IndexerArgs& a, int
   const int grid = items < sm_count() ? (int)items : sm_count();
   indexer_decode_tc_kernel<<<grid, idxdec::kThreads, idxdec::kSmem, st>>>(tk, tq, t);
   CSA_CHECK_LAUNCH();
+  if (after_scores && cudaEventRecord(after_scores, st) != cudaSuccess) return CSA_ERR_CUDA;
   if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsel::kSmem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
@@ -901,9 +950,12 @@ size_t csa_decode_workspace_bytes(const csa_dims* d, int B, int cap) {
   return dec_layout(d, B, cap).total;
 }
 
-csa_status csa_decode(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
-                      void* Ccache, void* KIcache, int* cache_len, int cap, int B, void* O, int* idx_out,
-                      void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+csa_status decode_impl(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
+                       void* Ccache, void* KIcache, int* cache_len, int cap, int B, void* O, int* idx_out,
+                       void* ws, size_t ws_bytes, void* const* ev, void* stream) {
   CSA_RANGE("csa_decode");
   csa_status s = check_dims(d);
   if (s != CSA_OK) return s;
@@ -922,29 +974,55 @@ csa_status csa_decode(const csa_dims* d, const void* packed, const void* h, cons
   float* wI = reinterpret_cast<float*>(at(ws, L.wI));
   char* y2 = at(ws, L.y2);
   int* idx = idx_out ? idx_out : reinterpret_cast<int*>(at(ws, L.idx));
+  if ((s = mark(ev, 0, st)) != CSA_OK) return s;
   s = project_hidden(d, packed, h, B, y1, wI, st, reinterpret_cast<float*>(at(ws, L.split)),
                      L.total - L.split);
-  if (s != CSA_OK) return s;
+  if (s != CSA_OK || (s = mark(ev, 1, st)) != CSA_OK) return s;
   s = launch_append(d, packed, y1, P.N1b, pos, ring, Ccache, KIcache, cache_len, cap, B, st);
-  if (s != CSA_OK) return s;
+  if (s != CSA_OK || (s = mark(ev, 2, st)) != CSA_OK) return s;
   s = project_query(d, packed, y1 + (size_t)(4 * c + 4 * cI) * es, P.N1b, B, y2, st);
-  if (s != CSA_OK) return s;
+  if (s != CSA_OK || (s = mark(ev, 3, st)) != CSA_OK) return s;
   IndexerArgs ia;
   ia.qI = y2; ia.ld_qI = P.N2; ia.wI = wI; ia.ld_wI = d->nhI; ia.KI = KIcache; ia.idx = idx;
   ia.topk = d->topk; ia.nhI = d->nhI; ia.sc_cap = cap;
   ia.rm = RowMap{nullptr, nullptr, 0, 0, pos, cap, d->m};
   if (d->dtype == CSA_BF16 && (d->nhI == 32 || d->nhI == 64) && (d->cI == 64 || d->cI == 128) &&
-      reinterpret_cast<uintptr_t>(KIcache) % 16 == 0)
-    s = launch_indexer_decode_tc(d, ia, B, cap, reinterpret_cast<float*>(at(ws, L.scratch)), st);
-  else
-    s = launch_indexer(d, ia, B, st);
-  if (s != CSA_OK) return s;
+      reinterpret_cast<uintptr_t>(KIcache) % 16 == 0) {
+    s = launch_indexer_decode_tc(d, ia, B, cap, reinterpret_cast<float*>(at(ws, L.scratch)), st,
+                                 ev ? (cudaEvent_t)ev[4] : nullptr);
+  } else {
+    s = launch_indexer(d, ia, B, st);   // scores and selection in one kernel: both events after it
+    if (s == CSA_OK) s = mark(ev, 4, st);
+  }
+  if (s != CSA_OK || (s = mark(ev, 5, st)) != CSA_OK) return s;
   MqaArgs ma;
   ma.q = y2 + (size_t)d->nhI * cI * es; ma.ld_q = P.N2; ma.C = Ccache; ma.idx = idx;
   ma.O = O; ma.ld_O = (long long)d->nh * c; ma.topk = d->topk; ma.nh = d->nh;
   ma.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c));
   ma.rm = RowMap{nullptr, nullptr, 0, 0, pos, cap, d->m};
-  return launch_mqa(d, ma, B, st);
+  s = launch_mqa(d, ma, B, st);
+  if (s != CSA_OK) return s;
+  return mark(ev, 6, st);
+}
+}  // namespace
+
+extern "C" {
+
+csa_status csa_decode(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
+                      void* Ccache, void* KIcache, int* cache_len, int cap, int B, void* O, int* idx_out,
+                      void* ws, size_t ws_bytes, void* stream) {
+  return decode_impl(d, packed, h, pos, ring, Ccache, KIcache, cache_len, cap, B, O, idx_out, ws, ws_bytes,
+                     nullptr, stream);
+}
+
+csa_status csa_decode_staged(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
+                             void* Ccache, void* KIcache, int* cache_len, int cap, int B, void* O, int* idx_out,
+                             void* ws, size_t ws_bytes, void* const* events, void* stream) {
+  if (!events) return CSA_ERR_INVALID_ARG;
+  for (int i = 0; i < 7; ++i)
+    if (!events[i]) return CSA_ERR_INVALID_ARG;
+  return decode_impl(d, packed, h, pos, ring, Ccache, KIcache, cache_len, cap, B, O, idx_out, ws, ws_bytes,
+                     events, stream);
 }
 
 }  // extern "C"

@@ -58,7 +58,12 @@ constexpr int kThreads = 320;
 }  // namespace idxtc
 
 // Item `it` of the work list: compression blocks from the last one down, then
-// one tail item per sequence.  Returns false for an empty tail item.
+// one tail item per sequence.  Returns false for an empty tail item and for
+// an item the metadata cannot place: its score rows would not fit the
+// scratch rows (more visible blocks than sc_cap, i.e. a max_seqlen below the
+// real length), its queries lie outside [0, total_tokens) or its blocks
+// outside [0, total_blocks).  Such an item is skipped by every role alike
+// (each evaluates the same test) and kStatusMetadata is raised.
 __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, int& nq, int& avail,
                                          long long& kbase) {
   if (it < a.total_blocks) {
@@ -73,6 +78,11 @@ __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, 
     nq = 4;
     avail = i;
     kbase = a.cu_blocks[lo];
+    if (i < 0 || tok0 < 0 || tok0 + 4 > a.cu_seqlens[lo + 1] || a.cu_seqlens[lo + 1] > a.total_tokens ||
+        avail >= a.sc_cap) {
+      flag_status(kStatusMetadata);
+      return false;
+    }
     return true;
   }
   const int b = it - a.total_blocks;
@@ -81,6 +91,13 @@ __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, 
   tok0 = a.cu_seqlens[b + 1] - nq;
   avail = L >> 2;
   kbase = a.cu_blocks[b];
+  // every sequence's tail item also checks that cu_blocks gives the sequence
+  // floor(L/4) blocks, so that no block of queries goes unvisited unnoticed
+  if (L < 0 || a.cu_seqlens[b] < 0 || a.cu_seqlens[b + 1] > a.total_tokens || kbase < 0 ||
+      a.cu_blocks[b + 1] - kbase != avail || kbase + avail > a.total_blocks || (nq > 0 && avail >= a.sc_cap)) {
+    flag_status(kStatusMetadata);
+    return false;
+  }
   return nq > 0;
 }
 

@@ -35,10 +35,13 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // Bounded waits.  Each poll is a try_wait with a suspend-time hint, so a
 // waiting thread sleeps in hardware until the phase completes (or the hint
 // runs out) instead of spinning and taking issue slots from the working
-// warps of its SM sub-partition.  A wait gives up after kWaitNs of global
-// time (read from %globaltimer), i.e. of the order of a second.
+// warps of its SM sub-partition.  A wait gives up after g_wait_ns of global
+// time (read from %globaltimer; 1.5 s unless csa_set_wait_limit_ns changed
+// it), and in any case after kMaxPolls polls, a backstop that does not
+// depend on the timer (at least ~20 s of polling even if every poll returned
+// at once, so it never ends a wait the time limit would have kept).
 constexpr uint32_t kSuspendHintNs = 1000000;        // 1 ms per poll at most
-constexpr uint64_t kWaitNs = 1500000000ull;         // 1.5 s per wait at most
+constexpr uint32_t kMaxPolls = 1u << 30;
 
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
@@ -47,10 +50,10 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Waits for the phase of parity `parity` to complete.  Returns false (and
-// records kStatusTimeout) if it did not complete within kWaitNs.
+// records kStatusTimeout) if it did not complete within the wait limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint32_t addr = smem_u32(bar);
-  uint64_t t0 = 0;
+  uint64_t t0 = 0, limit = 0;
   for (uint32_t i = 0;; ++i) {
     uint32_t done;
     asm volatile(
@@ -63,7 +66,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (done) return true;
     if (i == 0) {
       t0 = global_ns();
-    } else if (global_ns() - t0 > kWaitNs) {
+      limit = *reinterpret_cast<volatile unsigned long long*>(&g_wait_ns);
+    } else if (global_ns() - t0 > limit || i >= kMaxPolls) {
       flag_status(kStatusTimeout);
       return false;
     }

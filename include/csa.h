@@ -169,8 +169,13 @@ csa_status csa_compress_kv(const csa_dims* dims, const void* packed, const void*
  *             local block indices s < floor(t/m) in ascending order, then -1.
  *             k is clamped to floor(t/m); ties are broken by the lower s.
  * max_seqlen [host] : an upper bound of every sequence length (it sizes the
- *             per-query candidate storage; a longer sequence is clamped and
- *             flags CSA_ERR_BAD_METADATA).
+ *             per-query candidate storage).  A query of a longer sequence
+ *             is not computed in full: the CUDA-core path clamps its
+ *             candidates, the tensor-core path skips its block of queries
+ *             (their idx rows keep their old contents); either way nothing
+ *             is written outside the workspace and CSA_ERR_BAD_METADATA is
+ *             flagged.  The same holds for cu_seqlens / cu_blocks that
+ *             place a query or block outside total_tokens / total_blocks.
  * ws [dev]  : workspace of ws_bytes >= csa_indexer_workspace_bytes(), 256-byte
  *             aligned, no initialisation needed.
  * The score matrix is never written to memory. */
@@ -194,8 +199,8 @@ size_t csa_indexer_workspace_bytes(const csa_dims* dims, int total_tokens, int n
  * every GPU that loads the library, held until the process exits).
  * Limits: the tensor-core indexer's shapes only (bf16, m = 4, nhI in {32, 64},
  * cI in {64, 128}, qI and KI 16-byte aligned, ld_qI a multiple of 8) and
- * max_seqlen / m + 1 <= 4096 (max_seqlen <= 16380 for m = 4); anything else
- * returns CSA_ERR_UNSUPPORTED before any launch.  It calls no allocating
+ * floor(max_seqlen / m) + 1 <= 4096 (max_seqlen <= 16383 for m = 4); anything
+ * else returns CSA_ERR_UNSUPPORTED before any launch.  It calls no allocating
  * routine.  The first call on a device looks up the scratch array's device
  * address (cudaGetSymbolAddress) with that device current; make that first
  * call before any stream capture.  Every call shares the one array: calls
@@ -244,6 +249,19 @@ csa_status csa_forward(const csa_dims* dims, const void* packed, const void* H,
                        int total_blocks, int max_seqlen, void* O, void* Ccomp_out, void* KI_out, int* idx_out,
                        void* ws, size_t ws_bytes, void* stream);
 
+/* csa_forward with stage timing: the same launches and results, plus a
+ * CUDA event recorded on `stream` before the first stage and after each
+ * stage: events[0] before A1, then after A1 (eqs. 1, 2, 5, 7 projection),
+ * A2 (eqs. 6, 10), A3 (eqs. 3-4 compression), A4 (eqs. 8-9 indexer +
+ * top-k) and A5 (eq. 11 MQA), i.e. events[1..5].
+ * events [host] : 6 cudaEvent_t handles (passed as void*), created by the
+ *                 caller; a NULL array or handle returns CSA_ERR_INVALID_ARG
+ *                 before any launch.  Recording adds no kernel. */
+csa_status csa_forward_staged(const csa_dims* dims, const void* packed, const void* H,
+                              const int* cu_seqlens, const int* cu_blocks, int nseq, int total_tokens,
+                              int total_blocks, int max_seqlen, void* O, void* Ccomp_out, void* KI_out,
+                              int* idx_out, void* ws, size_t ws_bytes, void* const* events, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Decode over a compressed cache                                          */
 /* ---------------------------------------------------------------------- */
@@ -279,6 +297,19 @@ csa_status csa_decode(const csa_dims* dims, const void* packed, const void* h, c
                       void* ring, void* Ccache, void* KIcache, int* cache_len, int cap, int B,
                       void* O, int* idx_out, void* ws, size_t ws_bytes, void* stream);
 
+/* csa_decode with stage timing: the same launches and results, plus a CUDA
+ * event recorded on `stream` before the first stage (events[0]) and after
+ * each stage: the H-side projection with its K-split reduction (1), the
+ * cache append (2), the c^Q-side projection (3), the indexer scores (4),
+ * the top-k selection (5) and the MQA (6).
+ * events [host] : 7 cudaEvent_t handles (passed as void*), created by the
+ *                 caller; a NULL array or handle returns CSA_ERR_INVALID_ARG
+ *                 before any launch.  Recording adds no kernel. */
+csa_status csa_decode_staged(const csa_dims* dims, const void* packed, const void* h, const int* pos,
+                             void* ring, void* Ccache, void* KIcache, int* cache_len, int cap, int B,
+                             void* O, int* idx_out, void* ws, size_t ws_bytes, void* const* events,
+                             void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Status                                                                  */
 /* ---------------------------------------------------------------------- */
@@ -294,6 +325,34 @@ const char* csa_status_string(csa_status s);
 /* Number of kernels this library has enqueued in this process so far (all
  * devices, all streams).  A monotone counter for accounting; never reset. */
 uint64_t csa_launch_count(void);
+
+/* ---------------------------------------------------------------------- */
+/* Failure detection                                                       */
+/* ---------------------------------------------------------------------- */
+/* Not steps of the method (the page describes no runtime): every wait
+ * inside a kernel of this library is bounded, and one that runs out records
+ * CSA_ERR_DEVICE_TIMEOUT in the status word and ends its kernel instead of
+ * hanging the GPU. */
+
+/* Sets the limit of every bounded device wait on the current device, in ns
+ * of the GPU's global timer (default 1.5 s; accepted range 1 us .. 60 s,
+ * else CSA_ERR_INVALID_ARG).  Each wait also ends after 2^30 polls whatever
+ * the timer says.  Takes effect for kernels launched after the call
+ * returns; call it while no kernel of this library is running.  Meant for
+ * tests and diagnostics: a too-short limit turns slow but healthy waits
+ * into timeouts. */
+csa_status csa_set_wait_limit_ns(unsigned long long ns);
+
+/* Self-check of the bounded waits: enqueues one small kernel whose first
+ * warp waits on a barrier that nothing arrives on (the wait must run out at
+ * the limit, return to its caller and record CSA_ERR_DEVICE_TIMEOUT) and
+ * whose second warp waits on a barrier it completes itself.
+ * out [dev] : 3 x uint64, 8-byte aligned: out[0] = 1 if the first wait
+ *             claimed completion (it must not), out[1] = ns the first wait
+ *             took, out[2] = 1 if the second wait completed.
+ * Read the result with csa_get_device_status (CSA_ERR_DEVICE_TIMEOUT is the
+ * expected answer). */
+csa_status csa_check_wait_timeout(unsigned long long* out, void* stream);
 
 #ifdef __cplusplus
 }

@@ -41,6 +41,8 @@ __all__ = [
     "topk_select",
     "core_attn",
     "num_blocks",
+    "compressed_entries",
+    "query_rows",
     "csa_forward",
     "csa_forward_sampled",
     "csa_decode_step",
@@ -221,6 +223,73 @@ def core_attn(q_t, C_sel):
 _HSIDE = ("W_aKV", "W_bKV", "W_aZ", "W_bZ", "W_aKV_I", "W_bKV_I", "W_aZ_I", "W_bZ_I")
 
 
+def compressed_entries(H, W, dims, seqlens, store="exact"):
+    """The token-parallel half of the forward pass: eqs. (1), (2), the
+    indexer-key projections, and eqs. (3), (4) per sequence.
+
+    Returns (C_comp [NB, c], K_icomp [NB, c^I], cu [nseq+1], cu_blocks [nseq+1]).
+    Arguments as for ``csa_forward``.
+    """
+    H = np.asarray(H, dtype=np.float64)
+    m, c, cI = dims["m"], dims["c"], dims["cI"]
+    assert sum(seqlens) == H.shape[0]
+    rnd = lambda x: storage_round(x, store)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int64)
+    cu_blocks = np.concatenate([[0], np.cumsum([num_blocks(L, m) for L in seqlens])]).astype(np.int64)
+    proj = {name: rnd(project(H, W[name])) for name in _HSIDE}
+    C_comp_parts, K_icomp_parts = [], []
+    for b, L in enumerate(seqlens):
+        sl = slice(cu[b], cu[b] + L)
+        C_comp_parts.append(compress(proj["W_aKV"][sl], proj["W_bKV"][sl], proj["W_aZ"][sl],
+                                     proj["W_bZ"][sl], W["B_a"], W["B_b"], m))
+        K_icomp_parts.append(compress(proj["W_aKV_I"][sl], proj["W_bKV_I"][sl], proj["W_aZ_I"][sl],
+                                      proj["W_bZ_I"][sl], W["B_a_I"], W["B_b_I"], m))
+    C_comp = rnd(np.concatenate(C_comp_parts, axis=0)) if C_comp_parts else np.zeros((0, c))
+    K_icomp = rnd(np.concatenate(K_icomp_parts, axis=0)) if K_icomp_parts else np.zeros((0, cI))
+    return C_comp, K_icomp, cu, cu_blocks
+
+
+def query_rows(H, W, dims, C_comp, K_icomp, cu, cu_blocks, rows, store="exact", keep_scores=False):
+    """The per-query half of the forward pass for the global rows ``rows``:
+    eqs. (5), (6), (7), (10), then eq. (8) over the visible blocks, eq. (9)
+    and eq. (11), given the compressed entries of ``compressed_entries``.
+
+    Returns a dict with, per row, idx [R, topk], O [R, n_h, c], cQ, wI, qI,
+    q and, if keep_scores, the list of score rows.
+    """
+    H = np.asarray(H, dtype=np.float64)
+    m, k = dims["m"], dims["topk"]
+    nh, nhI, c, cI = dims["nh"], dims["nhI"], dims["c"], dims["cI"]
+    rnd = lambda x: storage_round(x, store)
+    rnd_w = (lambda x: round_f32(x)) if store == "bf16" else rnd
+    rows = np.asarray(rows, dtype=np.int64)
+    seq_of = np.searchsorted(cu, rows, side="right") - 1
+
+    cQ = rnd(project(H[rows], W["W_DQ"]))                    # [R, d_c]
+    wI = rnd_w(project(H[rows], W["W_w"]))                   # [R, n_h^I]
+    qI = rnd(project(cQ, W["W_IUQ"])).reshape(len(rows), nhI, cI)
+    q = rnd(project(cQ, W["W_UQ"])).reshape(len(rows), nh, c)
+
+    idx = np.full((len(rows), k), -1, dtype=np.int64)
+    O = np.zeros((len(rows), nh, c))
+    scores = []
+    for r, (tg, b) in enumerate(zip(rows, seq_of)):
+        t = int(tg - cu[b])                                  # local token index
+        avail = t // m                                       # blocks s < floor(t/m)
+        base = int(cu_blocks[b])
+        I_t = indexer_scores(qI[r], wI[r], K_icomp[base:base + avail])      # eq. (8)
+        sel = topk_select(I_t, k)                                           # eq. (9)
+        idx[r] = sel
+        chosen = sel[sel >= 0]
+        O[r] = core_attn(q[r], C_comp[base + chosen])                       # eq. (11)
+        if keep_scores:
+            scores.append(I_t)
+    out = {"rows": rows, "idx": idx, "O": O, "cQ": cQ, "wI": wI, "qI": qI, "q": q}
+    if keep_scores:
+        out["scores"] = scores
+    return out
+
+
 def csa_forward(H, W, dims, seqlens, store="exact", rows=None, keep_scores=False):
     """CSA forward pass, eqs. (1)-(11), over packed sequences.
 
@@ -243,59 +312,15 @@ def csa_forward(H, W, dims, seqlens, store="exact", rows=None, keep_scores=False
     Returns a dict with C_comp [NB, c], K_icomp [NB, c^I], cu_blocks, and per
     evaluated row: idx [R, topk] (local block indices, -1 padded), O [R, n_h, c]
     and, if keep_scores, the list of score rows.
+    The work is the two halves ``compressed_entries`` (eqs. 1-4) and
+    ``query_rows`` (eqs. 5-11), in that order.
     """
     H = np.asarray(H, dtype=np.float64)
-    m, k = dims["m"], dims["topk"]
-    nh, nhI, c, cI = dims["nh"], dims["nhI"], dims["c"], dims["cI"]
-    T = H.shape[0]
-    assert sum(seqlens) == T
-    rnd = lambda x: storage_round(x, store)
-    rnd_w = (lambda x: round_f32(x)) if store == "bf16" else rnd
-
-    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int64)
-    cu_blocks = np.concatenate([[0], np.cumsum([num_blocks(L, m) for L in seqlens])]).astype(np.int64)
-
-    # Eqs. (1), (2) and the indexer copies, then eqs. (3), (4) per sequence.
-    proj = {name: rnd(project(H, W[name])) for name in _HSIDE}
-    C_comp_parts, K_icomp_parts = [], []
-    for b, L in enumerate(seqlens):
-        sl = slice(cu[b], cu[b] + L)
-        C_comp_parts.append(compress(proj["W_aKV"][sl], proj["W_bKV"][sl], proj["W_aZ"][sl],
-                                     proj["W_bZ"][sl], W["B_a"], W["B_b"], m))
-        K_icomp_parts.append(compress(proj["W_aKV_I"][sl], proj["W_bKV_I"][sl], proj["W_aZ_I"][sl],
-                                      proj["W_bZ_I"][sl], W["B_a_I"], W["B_b_I"], m))
-    C_comp = rnd(np.concatenate(C_comp_parts, axis=0)) if C_comp_parts else np.zeros((0, c))
-    K_icomp = rnd(np.concatenate(K_icomp_parts, axis=0)) if K_icomp_parts else np.zeros((0, cI))
-
+    C_comp, K_icomp, cu, cu_blocks = compressed_entries(H, W, dims, seqlens, store)
     if rows is None:
-        rows = np.arange(T)
-    rows = np.asarray(rows, dtype=np.int64)
-    seq_of = np.searchsorted(cu, rows, side="right") - 1
-
-    # Eqs. (5), (6), (7), (10) for the evaluated rows only.
-    cQ = rnd(project(H[rows], W["W_DQ"]))                    # [R, d_c]
-    wI = rnd_w(project(H[rows], W["W_w"]))                   # [R, n_h^I]
-    qI = rnd(project(cQ, W["W_IUQ"])).reshape(len(rows), nhI, cI)
-    q = rnd(project(cQ, W["W_UQ"])).reshape(len(rows), nh, c)
-
-    idx = np.full((len(rows), k), -1, dtype=np.int64)
-    O = np.zeros((len(rows), nh, c))
-    scores = []
-    for r, (tg, b) in enumerate(zip(rows, seq_of)):
-        t = int(tg - cu[b])                                  # local token index
-        avail = t // m                                       # blocks s < floor(t/m)
-        base = int(cu_blocks[b])
-        I_t = indexer_scores(qI[r], wI[r], K_icomp[base:base + avail])      # eq. (8)
-        sel = topk_select(I_t, k)                                           # eq. (9)
-        idx[r] = sel
-        chosen = sel[sel >= 0]
-        O[r] = core_attn(q[r], C_comp[base + chosen])                       # eq. (11)
-        if keep_scores:
-            scores.append(I_t)
-    out = {"C_comp": C_comp, "K_icomp": K_icomp, "cu_blocks": cu_blocks, "rows": rows,
-           "idx": idx, "O": O, "cQ": cQ, "wI": wI, "qI": qI, "q": q}
-    if keep_scores:
-        out["scores"] = scores
+        rows = np.arange(H.shape[0])
+    out = query_rows(H, W, dims, C_comp, K_icomp, cu, cu_blocks, rows, store, keep_scores)
+    out.update({"C_comp": C_comp, "K_icomp": K_icomp, "cu_blocks": cu_blocks})
     return out
 
 
@@ -390,7 +415,8 @@ def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="e
     [B, 2m, 4c + 4c^I] are updated IN PLACE (copies are the caller's choice).
     cache_len[b] must equal floor(t/m) on entry.
     Returns (O [B, n_h, c], idx [B, topk]).  If ``detail`` is a dict it
-    receives per sequence the scores I_t and the attention queries q_t.
+    receives per sequence the scores I_t, the attention queries q_t and the
+    indexer inputs q^I_t and w^I_t.
     """
     m, k = dims["m"], dims["topk"]
     nh, nhI, c, cI = dims["nh"], dims["nhI"], dims["c"], dims["cI"]
@@ -446,4 +472,6 @@ def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="e
         if detail is not None:
             detail.setdefault("scores", []).append(I_t)
             detail.setdefault("q", []).append(q)
+            detail.setdefault("qI", []).append(qI)
+            detail.setdefault("wI", []).append(wI)
     return O, idx

@@ -2,17 +2,22 @@
 and compare it with the fp64 oracle on the same seeded inputs.
 
 Comparison protocol (tolerances of the bf16 and fp32 configurations):
-* top-k sets: where the oracle's k-th / (k+1)-th score gap exceeds 1e-3
-  relative, the GPU set must equal the oracle's exactly; below that gap the
-  set must be valid (k_eff distinct visible blocks, each with an oracle score
-  within the bar of the k-th score).  Relative here means relative to
-  max(|I_(k)|, 1e-2 * max_s |I_s|), so that a k-th score that happens to sit
-  near zero does not demand more than fp32 can resolve.  Stage tests feed
-  both sides bit-identical inputs and use exactly this bar.  End-to-end bf16
-  tests widen it by the score perturbation that bf16 storage rounding itself
-  causes in the oracle (rounding_sensitivity): there both sides round their
-  own projections to bf16 and a few stored elements legitimately land on
-  neighbouring bf16 values.
+* top-k sets (eq. 9 of "Compressed Sparse Attention", cnblogs; the exactness
+  bar is a gap of 1e-3 relative to the k-th score, ties to the lower block).
+  Every candidate score I_s the oracle computes carries an admissible
+  perturbation delta_s >= 0: the worst-case error of evaluating eq. (8) in
+  fp32 from the same inputs (fp32_score_bound), plus, end to end in bf16,
+  that candidate's own bf16-storage sensitivity |I_bf16(s) - I_exact(s)|
+  (both sides round their own projections to bf16, and a stored element may
+  land on the neighbouring bf16 value).  Let top be the oracle's set and
+      lo = min_{s in top} (I_s - delta_s),  hi = max_{u not in top} (I_u + delta_u).
+  If lo - hi > 1e-3 |I_(k)| the set is stable under every admissible
+  perturbation and the GPU set must equal it exactly ("required").  With all
+  delta_s = 0 this is exactly "I_(k) - I_(k+1) > 1e-3 |I_(k)|".  Otherwise the
+  GPU set must be a correct top-k of some admissible perturbation of the
+  scores, i.e. min_{s in gpu} (I_s + delta_s) >= max_{u not in gpu}
+  (I_u - delta_u) - 1e-3 |I_(k)|, with k_eff distinct visible blocks in
+  ascending order and -1 padding.
 * outputs: the GPU output o_t is compared with eq. (11) evaluated by the
   oracle on the GPU's own index set (this isolates the attention error from
   the selection): bf16 max-abs <= 2e-2 and relative L2 <= 1e-2; fp32
@@ -86,13 +91,52 @@ def compare_dense(got, want, dtype, what=""):
     return max_abs, rel
 
 
-def check_topk_row(gpu_row, scores, k, extra_tol=0.0):
-    """Check one GPU top-k row against the oracle's fp64 scores; returns 'exact'/'valid'.
+# Rounding unit of one fp32 operation in the bound below: 2^-23, twice the
+# round-to-nearest unit, so that accumulation that truncates (as a tensor
+# core's adder may) is covered as well.
+U32 = 2.0 ** -23
 
-    extra_tol (absolute) widens the gap bar where the two sides do not see
-    bit-identical inputs (end-to-end runs, where both round their own fp32 /
-    fp64 projections to bf16 and so may store neighbouring bf16 values)."""
+
+def fp32_score_bound(qI_t, wI_t, KI_avail):
+    """Worst-case |I_fp32(t, s) - I_exact(t, s)| of eq. (8) evaluated in fp32
+    arithmetic (any summation order) from the same inputs, per visible block.
+
+    qI_t [n_h^I, c^I], wI_t [n_h^I], KI_avail [avail, c^I].  Each term
+    w_h * ReLU(q_h . K_s) is a c^I-term dot product (products of bf16 values
+    are exact in fp32; one more rounding each for fp32 inputs), a ReLU
+    (exact), a product with w_h and a sum over n_h^I heads, so the standard
+    summation bound gives gamma_n * sum_h |w_h| sum_j |q_hj K_sj| with
+    n = c^I + n_h^I + 2 and gamma_n = n u / (1 - n u)."""
+    KI_avail = np.asarray(KI_avail, dtype=np.float64)
+    if KI_avail.shape[0] == 0:
+        return np.zeros(0)
+    q, w = np.abs(np.asarray(qI_t, dtype=np.float64)), np.abs(np.asarray(wI_t, dtype=np.float64))
+    n = q.shape[1] + q.shape[0] + 2
+    gamma = n * U32 / (1.0 - n * U32)
+    return gamma * (w @ (q @ np.abs(KI_avail).T))
+
+
+def score_delta(scores_store, scores_exact, qI_t, wI_t, KI_avail):
+    """Admissible perturbation of each candidate score of one row: the fp32
+    evaluation bound plus, where given, the candidate's own bf16-storage
+    sensitivity |I_bf16(s) - I_exact(s)| from the oracle."""
+    d = fp32_score_bound(qI_t, wI_t, KI_avail)
+    if scores_exact is not None:
+        d = d + np.abs(np.asarray(scores_store, dtype=np.float64) - np.asarray(scores_exact, dtype=np.float64))
+    return d
+
+
+def check_topk_row(gpu_row, scores, k, delta=None, gap_rel=GAP_REL):
+    """Check one GPU top-k row against the oracle's fp64 scores under the
+    protocol of this module.  delta: per-candidate admissible perturbation
+    (None = 0).  gap_rel: the relative margin (the benchmark spec's 1e-3; stage
+    tests, whose two sides see bit-identical inputs, pass 0 and so demand
+    exactness wherever the set is stable under the fp32 evaluation bound
+    alone, which is stricter).  Returns "all" (k_eff = avail: every block),
+    "required" (stable set, matched exactly), "equal" (not required but
+    equal) or "valid" (a correct top-k of an admissible perturbation)."""
     gpu_row = np.asarray(gpu_row, dtype=np.int64)
+    scores = np.asarray(scores, dtype=np.float64)
     avail = len(scores)
     keff = min(k, avail)
     assert np.all(gpu_row[keff:] == -1), "padding must be -1"
@@ -101,22 +145,36 @@ def check_topk_row(gpu_row, scores, k, extra_tol=0.0):
     assert keff == 0 or (sel[0] >= 0 and sel[-1] < avail), "indices must be visible blocks"
     if keff == avail:
         assert np.array_equal(sel, np.arange(avail))
-        return "exact"
+        return "all"
+    delta = np.zeros(avail) if delta is None else np.asarray(delta, dtype=np.float64)
     want = orc.topk_select(scores, k)[:keff]
-    srt = np.sort(scores)[::-1]
-    Ik, Ik1 = srt[keff - 1], srt[keff]
-    denom = max(abs(Ik), 1e-2 * float(np.abs(scores).max()), 1e-300)
-    bar = max(GAP_REL * denom, extra_tol)
-    if Ik - Ik1 > bar:
-        assert np.array_equal(sel, want), f"set differs with gap {(Ik - Ik1) / denom:.2e} (bar {bar / denom:.2e})"
-        return "exact"
-    assert np.all(scores[sel] >= Ik - bar), "a chosen block scores below the k-th"
+    Ik = np.sort(scores)[::-1][keff - 1]
+    bar = gap_rel * abs(Ik)
+    top = np.zeros(avail, dtype=bool)
+    top[want] = True
+    lo = float((scores - delta)[top].min())
+    hi = float((scores + delta)[~top].max())
+    if lo - hi > bar:
+        assert np.array_equal(sel, want), \
+            f"stable set differs: net gap {(lo - hi) / max(abs(Ik), 1e-300):.2e} of |I_(k)|"
+        return "required"
+    if np.array_equal(sel, want):
+        return "equal"
+    mine = np.zeros(avail, dtype=bool)
+    mine[sel] = True
+    lo_g = float((scores + delta)[mine].min())
+    hi_g = float((scores - delta)[~mine].max())
+    assert lo_g >= hi_g - bar, \
+        f"not a top-k of any admissible perturbation: {lo_g:.6g} < {hi_g:.6g} - {bar:.3g}"
     return "valid"
 
 
-def rounding_sensitivity(scores_bf16, scores_exact):
-    """Score perturbation caused by bf16 storage rounding alone, from the oracle:
-    max_s |I_bf16(t, s) - I_exact(t, s)| over one row (0 for an empty row)."""
-    if len(scores_bf16) == 0:
-        return 0.0
-    return float(np.abs(np.asarray(scores_bf16) - np.asarray(scores_exact)).max())
+def new_counts():
+    return {"all": 0, "required": 0, "equal": 0, "valid": 0}
+
+
+def report(name, counts):
+    """Prints the row classification of one test (shown with pytest -s or on failure)."""
+    n = sum(counts.values())
+    print(f"[topk parity] {name}: {n} rows: {counts}")
+    return counts

@@ -100,3 +100,16 @@ def test_replica_timing_is_max_over_ranks_gloo():
         assert m == 150.0
         assert v == pytest.approx(8192 * 10 * 2 / 0.150)
     assert bench.max_over_ranks(42.0, torch.device("cpu"), 1) == 42.0
+
+
+def test_oracle_baseline_measures_rows_on_their_own():
+    """cpu_baseline times the per-query half directly (no difference of two
+    timings, no clamp): a positive per-row cost and a rate below the one the
+    token-parallel half alone would give."""
+    w = bench.synth.workloads()["tiny"]
+    tps, info = bench.oracle_baseline(w, budget_s=0.2, chunk=8)
+    assert info["rows"] >= 16 and info["per_row_s"] > 0 and info["rows_s"] > 0
+    T = sum(w.seqlens)
+    assert 0 < tps < T / info["base_s"]
+    one = bench.oracle_tiny_one_thread()
+    assert one["cores"] == 1 and one["value"] > 0

@@ -7,8 +7,8 @@ import torch
 import compressed_sparse_attention_09_b200 as csa
 from compressed_sparse_attention_09_b200 import synth
 from oracle import csa_oracle as orc
-from parity import (check_topk_row, compare_dense, f64, gpu_forward, gpu_pack, rounding_sensitivity,
-                    store_mode, weights_f64)
+from parity import (check_topk_row, compare_dense, f64, fp32_score_bound, gpu_forward, gpu_pack, new_counts,
+                    report, score_delta, store_mode, weights_f64)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -18,39 +18,42 @@ def odims(dims):
     return dict(m=dims.m, topk=dims.topk, nh=dims.nh, nhI=dims.nhI, c=dims.c, cI=dims.cI)
 
 
-def e2e(dims, seqlens, seed, rows=None):
-    """csa_forward vs the oracle: compressed entries, top-k sets, outputs."""
+def e2e(dims, seqlens, seed, rows=None, name="e2e"):
+    """csa_forward vs the oracle: compressed entries, top-k sets, outputs.
+    Returns the row classification of tests/parity.py (printed as well)."""
     W = synth.make_weights(dims, seed)
     H = synth.make_hidden(sum(seqlens), dims, seed)
     g = gpu_forward(dims, W, H, seqlens)
     o = orc.csa_forward(f64(H), weights_f64(W), odims(dims), list(seqlens), store=store_mode(dims),
                         rows=rows, keep_scores=True)
+    ox = None
     if dims.dtype == csa.CSA_BF16:
         ox = orc.csa_forward(f64(H), weights_f64(W), odims(dims), list(seqlens), store="exact",
                              rows=o["rows"], keep_scores=True)
-        sens = [rounding_sensitivity(a, b) for a, b in zip(o["scores"], ox["scores"])]
-    else:
-        sens = [0.0] * len(o["rows"])
     compare_dense(f64(g["C_comp"]), o["C_comp"], dims.dtype, "C_comp")
     compare_dense(f64(g["K_icomp"]), o["K_icomp"], dims.dtype, "K_icomp")
     cu = np.concatenate([[0], np.cumsum(seqlens)])
-    kinds = {"exact": 0, "valid": 0}
+    counts = new_counts()
     want = np.zeros((len(o["rows"]), dims.nh, dims.c))
     for r, t in enumerate(o["rows"]):
-        kinds[check_topk_row(g["idx"][t].numpy(), o["scores"][r], dims.topk, sens[r])] += 1
         b = int(np.searchsorted(cu, t, side="right") - 1)
+        base, avail = int(o["cu_blocks"][b]), int(t - cu[b]) // dims.m
+        delta = score_delta(o["scores"][r], None if ox is None else ox["scores"][r], o["qI"][r], o["wI"][r],
+                            o["K_icomp"][base:base + avail])
+        counts[check_topk_row(g["idx"][t].numpy(), o["scores"][r], dims.topk, delta)] += 1
         sel = g["idx"][t].numpy()
         sel = sel[sel >= 0]
-        want[r] = orc.core_attn(o["q"][r], o["C_comp"][o["cu_blocks"][b] + sel])
+        want[r] = orc.core_attn(o["q"][r], o["C_comp"][base + sel])
     compare_dense(f64(g["O"][torch.as_tensor(o["rows"])]), want, dims.dtype, "O")
-    return kinds
+    return report(name, counts)
 
 
 def test_tiny_fp32_full():
     """The tiny fp32 workload end to end, every row (fp32 SIMT path, 1e-5)."""
     w = synth.workloads()["tiny"]
-    kinds = e2e(w.dims, w.seqlens, w.seed)
-    assert kinds["exact"] > 0.8 * sum(kinds.values()), kinds
+    c = e2e(w.dims, w.seqlens, w.seed, name="tiny fp32")
+    assert sum(c.values()) == sum(w.seqlens)
+    assert c["required"] >= 0.85 * (c["required"] + c["equal"] + c["valid"]), c   # oracle alone: 180 of 188
 
 
 SMALL_BF16 = csa.Dims(d=512, c=128, m=4, cI=64, nhI=16, nh=8, dc=256, topk=24, dtype=csa.CSA_BF16)
@@ -59,24 +62,43 @@ SMALL_BF16 = csa.Dims(d=512, c=128, m=4, cI=64, nhI=16, nh=8, dc=256, topk=24, d
 def test_small_bf16_ragged():
     """Ragged packed bf16: tails not divisible by m, a sequence shorter than m,
     queries with fewer visible blocks than k."""
-    kinds = e2e(SMALL_BF16, (517, 3, 130, 1031), seed=21)
-    assert kinds["exact"] > 0.5 * sum(kinds.values()), kinds   # the rest passed the validity check
+    lens = (517, 3, 130, 1031)
+    c = e2e(SMALL_BF16, lens, seed=21, name="small bf16 ragged")
+    assert sum(c.values()) == sum(lens)
+    assert c["required"] >= 0.7 * (c["required"] + c["equal"] + c["valid"]), c   # oracle alone: 1081 of 1378
 
 
 def test_small_bf16_m2_fp32():
-    e2e(csa.Dims(d=256, c=64, m=2, cI=32, nhI=8, nh=4, dc=128, topk=8, dtype=csa.CSA_F32), (77, 200), 22)
-    e2e(csa.Dims(d=256, c=64, m=2, cI=32, nhI=8, nh=4, dc=128, topk=8, dtype=csa.CSA_BF16), (77, 200), 23)
+    e2e(csa.Dims(d=256, c=64, m=2, cI=32, nhI=8, nh=4, dc=128, topk=8, dtype=csa.CSA_F32), (77, 200), 22,
+        name="m=2 fp32")
+    e2e(csa.Dims(d=256, c=64, m=2, cI=32, nhI=8, nh=4, dc=128, topk=8, dtype=csa.CSA_BF16), (77, 200), 23,
+        name="m=2 bf16")
+
+
+def prefill_rows(T, m, k, n_random, seed):
+    """The first 2m rows, every row around the k clamp (t = m k - 1 .. m k + m),
+    the last row and seeded random rows."""
+    rng = np.random.default_rng(seed)
+    rows = set(range(min(T, 2 * m))) | {T - 1}
+    rows |= {t for t in range(m * k - 1, m * k + m + 1) if 0 <= t < T}
+    while len(rows) < n_random + 2 * m + m + 3:
+        rows.add(int(rng.integers(0, T)))
+    return sorted(rows)
 
 
 def test_prefill_full_size_sampled_rows():
-    """The n = 8192 prefill workload at full size; outputs checked on sampled
-    rows (the first 2m rows, the last row and seeded random rows)."""
+    """The n = 8192 prefill workload at full size; outputs and top-k sets
+    checked on 256 sampled rows (the first 2m rows, the k-clamp transition,
+    the last row and seeded random rows)."""
     w = synth.workloads()["prefill"]
     T = sum(w.seqlens)
-    rng = np.random.default_rng(5)
-    rows = sorted(set(range(2 * w.dims.m)) | {T - 1} | set(rng.integers(0, T, 24).tolist()))
-    kinds = e2e(w.dims, w.seqlens, w.seed, rows=rows)
-    assert kinds["exact"] >= 0.25 * len(rows), kinds
+    rows = prefill_rows(T, w.dims.m, w.dims.topk, 256 - 15, 5)
+    c = e2e(w.dims, w.seqlens, w.seed, rows=rows, name="prefill n=8192")
+    assert sum(c.values()) == len(rows) >= 256
+    # bf16 storage moves a candidate score by ~1.4 % of |I_(k)| (median over
+    # these rows) against a median k / (k+1) gap of 0.35 %, so only a few
+    # sets are stable here (oracle alone: 11 of 183); the rest must be valid
+    assert c["required"] >= 0.05 * (c["required"] + c["equal"] + c["valid"]), c
 
 
 # ---------------------------------------------------------------- stages
@@ -155,23 +177,30 @@ def _indexer_case(dims, lens, seed, zero_w=False):
     assert csa.csa_get_device_status() == 0
     idx = idx.cpu().numpy()
     q64, w64, K64 = f64(qI).reshape(T, dims.nhI, dims.cI), f64(wI), f64(KI)
-    kinds = {"exact": 0, "valid": 0}
+    counts = new_counts()
     for b, L in enumerate(lens):
         for t in range(L):
             row = int(cu[b]) + t
-            sc = orc.indexer_scores(q64[row], w64[row], K64[int(cb[b]):int(cb[b]) + t // dims.m])
-            kinds[check_topk_row(idx[row], sc, dims.topk)] += 1
+            Kv = K64[int(cb[b]):int(cb[b]) + t // dims.m]
+            sc = orc.indexer_scores(q64[row], w64[row], Kv)
+            counts[check_topk_row(idx[row], sc, dims.topk, fp32_score_bound(q64[row], w64[row], Kv))] += 1
             if zero_w:
                 keff = min(dims.topk, t // dims.m)
                 assert idx[row].tolist() == list(range(keff)) + [-1] * (dims.topk - keff)
-    return kinds
+    assert sum(counts.values()) == T
+    return report(f"indexer stage {lens} k={dims.topk}", counts)
+
+
+def selected(c):
+    """Rows whose set is a real selection (k_eff < visible blocks)."""
+    return c["required"] + c["equal"] + c["valid"]
 
 
 @pytest.mark.parametrize("dtype", [csa.CSA_F32, csa.CSA_BF16])
 def test_stage_indexer_topk(dtype):
     dims = csa.Dims(d=64, c=64, m=4, cI=64, nhI=8, nh=2, dc=64, topk=16, dtype=dtype)
-    kinds = _indexer_case(dims, [1000, 130, 2, 67], 41)
-    assert kinds["exact"] > 0.95 * sum(kinds.values())
+    c = _indexer_case(dims, [1000, 130, 2, 67], 41)
+    assert c["required"] >= 0.9 * selected(c), c   # oracle alone: 968 of 994
 
 
 def test_stage_indexer_ties_take_lowest_blocks():
@@ -181,8 +210,8 @@ def test_stage_indexer_ties_take_lowest_blocks():
 
 def test_stage_indexer_large_k():
     dims = csa.Dims(d=64, c=64, m=4, cI=128, nhI=16, nh=2, dc=64, topk=600, dtype=csa.CSA_BF16)
-    kinds = _indexer_case(dims, [4096, 2500], 43)
-    assert kinds["exact"] > 0.5 * sum(kinds.values())
+    c = _indexer_case(dims, [4096, 2500], 43)
+    assert c["required"] >= 0.65 * selected(c), c   # oracle alone: 1277 of 1788
 
 
 @pytest.mark.parametrize("nhI,cI", [(64, 128), (32, 64)])
@@ -191,13 +220,45 @@ def test_stage_indexer_topk_tensor_core(nhI, cI, topk):
     """The tcgen05 indexer (m = 4): ragged packed sequences with tails of 1-3
     tokens, sequences shorter than m, queries with fewer blocks than k."""
     dims = csa.Dims(d=64, c=64, m=4, cI=cI, nhI=nhI, nh=2, dc=64, topk=topk, dtype=csa.CSA_BF16)
-    kinds = _indexer_case(dims, [1000, 130, 2, 67, 515, 1], 44 + topk)
-    assert kinds["exact"] > 0.8 * sum(kinds.values()), kinds
+    c = _indexer_case(dims, [1000, 130, 2, 67, 515, 1], 44 + topk)
+    assert c["required"] >= 0.8 * selected(c), c   # oracle alone: at least 607 of 707
 
 
 def test_stage_indexer_tensor_core_ties_take_lowest_blocks():
     dims = csa.Dims(d=64, c=64, m=4, cI=128, nhI=64, nh=2, dc=64, topk=37, dtype=csa.CSA_BF16)
     _indexer_case(dims, [700, 9], 45, zero_w=True)
+
+
+def test_stage_indexer_understated_max_seqlen_stays_inside_workspace():
+    """A max_seqlen below a sequence's real length sizes the tensor-core
+    indexer's score rows too short for that sequence's later queries: their
+    items are skipped and flagged (CSA_ERR_BAD_METADATA) instead of writing
+    past the workspace, whose tail canary must survive; the sequence that
+    fits is still selected exactly as the oracle does."""
+    dims = csa.Dims(d=64, c=64, m=4, cI=128, nhI=64, nh=2, dc=64, topk=16, dtype=csa.CSA_BF16)
+    lens = [1000, 300]
+    T = sum(lens)
+    cu, cb = csa.cu_from_lengths(lens, dims.m)
+    NB = int(cb[-1])
+    qI = synth.make_normal((T, dims.nhI * dims.cI), dims, 81)
+    wI = synth.make_normal((T, dims.nhI), dims, 82).float()
+    KI = synth.make_normal((NB, dims.cI), dims, 83, std=0.5)
+    max_seqlen = 400                                  # understated: the first sequence has 1000 tokens
+    need = csa.csa_indexer_workspace_bytes(dims, T, len(lens), max_seqlen)
+    canary = 1 << 20
+    ws = torch.full((need + canary,), 0xA5, dtype=torch.uint8, device=DEV)
+    idx = torch.full((T, dims.topk), -7, dtype=torch.int32, device=DEV)
+    csa.csa_indexer_topk(dims, qI.to(DEV), dims.nhI * dims.cI, wI.to(DEV), dims.nhI, KI.to(DEV), cu.to(DEV),
+                         cb.to(DEV), len(lens), T, NB, max_seqlen, idx, ws[:need])
+    assert csa.csa_get_device_status() == 6       # CSA_ERR_BAD_METADATA
+    assert bool((ws[need:] == 0xA5).all()), "the indexer wrote past its workspace"
+    idx = idx.cpu().numpy()
+    q64, w64, K64 = f64(qI).reshape(T, dims.nhI, dims.cI), f64(wI), f64(KI)
+    for t in range(lens[1]):                          # the sequence that fits
+        row = lens[0] + t
+        Kv = K64[int(cb[1]):int(cb[1]) + t // dims.m]
+        sc = orc.indexer_scores(q64[row], w64[row], Kv)
+        check_topk_row(idx[row], sc, dims.topk, fp32_score_bound(q64[row], w64[row], Kv))
 
 
 def test_stage_indexer_topk_full_size_sampled():
@@ -220,12 +281,15 @@ def test_stage_indexer_topk_full_size_sampled():
     assert csa.csa_get_device_status() == 0
     idx = idx.cpu().numpy()
     q64, w64, K64 = f64(qI).reshape(T, dims.nhI, dims.cI), f64(wI), f64(KI)
-    rows = sorted(set(range(0, T, 61)) | {T - 1, 4 * 512, 4 * 512 + 3})
-    kinds = {"exact": 0, "valid": 0}
+    rows = sorted(set(range(0, T, 31)) | {T - 1} | set(range(4 * 512 - 1, 4 * 512 + 5)))
+    counts = new_counts()
     for t in rows:
-        sc = orc.indexer_scores(q64[t], w64[t], K64[:t // dims.m])
-        kinds[check_topk_row(idx[t], sc, dims.topk)] += 1
-    assert kinds["exact"] > 0.6 * len(rows), kinds   # the rest passed the validity check
+        Kv = K64[:t // dims.m]
+        sc = orc.indexer_scores(q64[t], w64[t], Kv)
+        counts[check_topk_row(idx[t], sc, dims.topk, fp32_score_bound(q64[t], w64[t], Kv))] += 1
+    report("indexer stage n=8192 k=512", counts)
+    assert sum(counts.values()) == len(rows)
+    assert counts["required"] >= 0.3 * selected(counts), counts   # oracle alone: 72 of 200
 
 
 def _mqa_case(dims, lens, seed, idx_fn, q_std=1.0, c_row_scale=None):
@@ -306,6 +370,7 @@ def decode_case(dims, B, pos0, cap, steps, seed, check):
     o_clen = clen[check].numpy().astype(np.int64)
     W64 = weights_f64(W)
     ws = torch.empty(csa.csa_decode_workspace_bytes(dims, B, cap), dtype=torch.uint8, device=DEV)
+    counts = new_counts()
     for step in range(steps):
         h = synth.make_normal((B, dims.d), dims, seed + 100 + step)
         O = torch.empty(B, dims.nh * c, dtype=h.dtype, device=DEV)
@@ -321,8 +386,10 @@ def decode_case(dims, B, pos0, cap, steps, seed, check):
         gidx = idx.cpu().numpy()[check]
         want = np.zeros_like(oO)
         for r in range(len(check)):
-            sens = rounding_sensitivity(detail["scores"][r], dx["scores"][r]) if dx else 0.0
-            check_topk_row(gidx[r], detail["scores"][r], dims.topk, sens)
+            avail = int(pos[check[r]]) // m
+            delta = score_delta(detail["scores"][r], dx["scores"][r] if dx else None, detail["qI"][r],
+                                detail["wI"][r], o_Kc[r][:avail])
+            counts[check_topk_row(gidx[r], detail["scores"][r], dims.topk, delta)] += 1
             sel = gidx[r][gidx[r] >= 0]
             want[r] = orc.core_attn(detail["q"][r], o_Cc[r][sel])
         compare_dense(f64(O.cpu()).reshape(B, dims.nh, c)[check], want, dims.dtype, f"decode O step {step}")
@@ -331,6 +398,8 @@ def decode_case(dims, B, pos0, cap, steps, seed, check):
     nb = int(o_clen.max())
     compare_dense(f64(d_Cc.cpu()[check][:, :nb]), o_Cc[:, :nb], dims.dtype, "C cache")
     compare_dense(f64(d_Kc.cpu()[check][:, :nb]), o_Kc[:, :nb], dims.dtype, "K cache")
+    assert sum(counts.values()) == steps * len(check)
+    return report(f"decode B={B} t0={pos0} k={dims.topk}", counts)
 
 
 def test_decode_small_across_appends():
@@ -345,10 +414,13 @@ def test_decode_small_fp32_from_start():
 
 def test_decode_full_size_sampled_sequences():
     """The decode workload at full size (64 sequences, 16384 cached entries,
-    n_h = 128, k = 2048); sampled sequences checked against the oracle."""
+    n_h = 128, k = 2048) for four steps, the last of which closes a block and
+    appends it to every cache; 8 of the 64 sequences are checked against the
+    oracle at every step, and their caches after the append."""
     w = synth.workloads()["decode"]
-    decode_case(w.dims, B=w.decode_batch, pos0=w.decode_pos, cap=w.cache_cap, steps=1, seed=w.seed,
-                check=[0, 17, 63])
+    c = decode_case(w.dims, B=w.decode_batch, pos0=w.decode_pos, cap=w.cache_cap, steps=4, seed=w.seed,
+                    check=[0, 9, 17, 26, 35, 44, 53, 63])
+    assert c["required"] >= 1, c
 
 
 def _holes(avail, k, row):

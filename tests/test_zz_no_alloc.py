@@ -53,3 +53,21 @@ def test_noalloc_indexer_rejects_sizes_beyond_its_scratch():
         csa.csa_indexer_topk_noalloc(dims, qI, dims.nhI * dims.cI, wI, dims.nhI, KI, cu, cb, 1, T, NB,
                                      4 * 4096, idx)     # max_seqlen beyond the fixed scratch
     assert e.value.status == 2   # CSA_ERR_UNSUPPORTED
+
+
+def test_noalloc_indexer_understated_max_seqlen_is_flagged():
+    """A max_seqlen below a sequence's real length would make the later
+    queries' score rows overrun the fixed scratch rows; those items are
+    skipped and flagged instead, and the next call works normally."""
+    dims = csa.Dims(d=64, c=64, m=4, cI=128, nhI=64, nh=2, dc=64, topk=100, dtype=csa.CSA_BF16)
+    T, NB, cu, cb, qI, wI, KI = _problem(dims, [6000], 304)
+    idx = torch.empty((T, dims.topk), dtype=torch.int32, device=DEV)
+    csa.csa_indexer_topk_noalloc(dims, qI, dims.nhI * dims.cI, wI, dims.nhI, KI, cu, cb, 1, T, NB, 1000, idx)
+    assert csa.csa_get_device_status() == 6   # CSA_ERR_BAD_METADATA
+    args = (dims, qI, dims.nhI * dims.cI, wI, dims.nhI, KI, cu, cb, 1, T, NB, T)
+    want = torch.empty_like(idx)
+    ws = torch.empty(csa.csa_indexer_workspace_bytes(dims, T, 1, T), dtype=torch.uint8, device=DEV)
+    csa.csa_indexer_topk(*args, want, ws)
+    csa.csa_indexer_topk_noalloc(*args, idx)
+    assert csa.csa_get_device_status() == 0
+    assert torch.equal(idx, want)
