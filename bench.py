@@ -69,6 +69,7 @@ def stage_work(dims, seqlens):
     N2 = dims.nhI * dims.cI + dims.nh * dims.c
     pairs, sel = causal_counts(seqlens, dims.m, dims.topk)
     return {
+        "A1A3_project_compress": ("tensor", 2.0 * T * dims.d * N1),
         "A1_project_hidden": ("tensor", 2.0 * T * dims.d * N1),
         "A2_project_query": ("tensor", 2.0 * T * dims.dc * N2),
         "A3_compress": ("hbm", 4.0 * T * (dims.c + dims.cI) * es + NB * (dims.c + dims.cI) * es),
@@ -197,6 +198,8 @@ class PrefillRunner:
         self.idx = torch.empty(self.T, d.topk, dtype=torch.int32, device=dev)
         self.iws = torch.empty(csa.csa_indexer_workspace_bytes(d, self.T, self.nseq, self.maxlen), dtype=torch.uint8,
                                device=dev)
+        fb = csa.csa_project_compress_workspace_bytes(d, self.T)
+        self.fws = torch.empty(fb, dtype=torch.uint8, device=dev) if fb else None
 
     def forward(self, H=None, O=None):
         d = self.dims
@@ -261,7 +264,12 @@ class PrefillRunner:
 
         def a3():   # both key sets in one launch, as csa_forward runs the stage
             csa.csa_compress_kv(d, self.packed, self.Y1, T, self.cu, self.cb, self.nseq, self.NB, self.Cc, self.KI)
-        return {
+        out = {}
+        if self.fws is not None:   # A1 with A3 in its epilogue, as csa_forward runs it
+            out["A1A3_project_compress"] = lambda: csa.csa_project_hidden_compress(
+                d, self.packed, self.H, T, self.cu, self.cb, self.nseq, self.NB, self.Y1, self.wI, self.Cc, self.KI,
+                self.fws)
+        return out | {
             "A1_project_hidden": lambda: csa.csa_project_hidden(d, self.packed, self.H, T, self.Y1, self.wI),
             "A2_project_query": lambda: csa.csa_project_query(d, self.packed, col(4 * c + 4 * cI), N1b, T, self.Y2),
             "A3_compress": a3,
@@ -495,7 +503,15 @@ def measure_stages(runner, w, args, peaks, flush, stream, reps):
             fn()
         alone[name] = stage_entry(name, statistics.mean(timed_steps(fn, reps, flush, stream)), work, peaks)
     in_step_ms = staged_step_ms(runner.forward_staged, len(STAGES), reps, flush, stream)
-    in_step = {n: stage_entry(n, ms, work, peaks, "bf16_sustained") for n, ms in zip(STAGES, in_step_ms)}
+    names = list(STAGES)
+    if runner.fws is not None:   # the compression runs inside the A1 kernel; its own interval is empty
+        names[0] = "A1A3_project_compress"
+    in_step = {}
+    for n, ms in zip(names, in_step_ms):
+        if n == "A3_compress" and runner.fws is not None:
+            in_step[n] = {"ms": ms, "note": "fused into A1A3_project_compress"}
+        else:
+            in_step[n] = stage_entry(n, ms, work, peaks, "bf16_sustained")
     st = csa.csa_get_device_status()
     if st != 0:
         raise RuntimeError(f"device status after stages: {csa.status_string(st)}")

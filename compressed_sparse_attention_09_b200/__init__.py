@@ -11,5 +11,6 @@ from .capi import (CSA_BF16, CSA_F32, CsaError, Dims, csa_cache_append, csa_comp
                    csa_hidden_row_elems, csa_query_row_elems, csa_project_hidden, csa_project_query,
                    csa_launch_count, csa_indexer_workspace_bytes,
                    csa_indexer_topk_noalloc, csa_compress_kv, csa_set_wait_limit_ns,
-                   csa_check_wait_timeout, csa_forward_staged, csa_decode_staged)
+                   csa_check_wait_timeout, csa_forward_staged, csa_decode_staged,
+                   csa_project_compress_workspace_bytes, csa_project_hidden_compress)
 from .meta import cu_from_lengths  # noqa: F401

@@ -28,6 +28,7 @@ EXPORTS = (
     "csa_status_string", "csa_hidden_row_elems", "csa_query_row_elems", "csa_project_hidden",
     "csa_project_query", "csa_launch_count", "csa_indexer_workspace_bytes", "csa_indexer_topk_noalloc",
     "csa_set_wait_limit_ns", "csa_check_wait_timeout", "csa_forward_staged", "csa_decode_staged",
+    "csa_project_compress_workspace_bytes", "csa_project_hidden_compress",
 )
 
 
@@ -100,6 +101,8 @@ def lib() -> ctypes.CDLL:
             "csa_project_query": (i, [D, vp, vp, i, i, vp, vp]),
             "csa_launch_count": (ctypes.c_uint64, []),
             "csa_set_wait_limit_ns": (i, [ctypes.c_ulonglong]),
+            "csa_project_compress_workspace_bytes": (sz, [D, i]),
+            "csa_project_hidden_compress": (i, [D, vp, vp, i, vp, vp, i, i, vp, vp, vp, vp, vp, sz, vp]),
             "csa_forward_staged": (i, [D, vp, vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp, vp]),
             "csa_decode_staged": (i, [D, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, sz, vp, vp]),
             "csa_check_wait_timeout": (i, [vp, vp]),
@@ -288,3 +291,16 @@ def csa_decode_staged(dims: Dims, packed, h, pos, ring, Ccache, KIcache, cache_l
     _check(lib().csa_decode_staged(_d(dims), _p(packed), _p(h), _p(pos), _p(ring), _p(Ccache), _p(KIcache),
                                    _p(cache_len), cap, B, _p(O), _p(idx_out), _p(ws), ws.numel() * ws.element_size(),
                                    _event_array(events), _stream(stream)), "csa_decode_staged")
+
+
+def csa_project_compress_workspace_bytes(dims: Dims, T) -> int:
+    return lib().csa_project_compress_workspace_bytes(_d(dims), T)
+
+
+def csa_project_hidden_compress(dims: Dims, packed, H, T, cu_seqlens, cu_blocks, nseq, total_blocks, Y1, wI, Ccomp,
+                                KIcomp, ws, stream=None):
+    """A1 with A3 in its epilogue (C^Comp, K^IComp, the c^Q columns of Y1, w^I)."""
+    _check(lib().csa_project_hidden_compress(_d(dims), _p(packed), _p(H), T, _p(cu_seqlens), _p(cu_blocks), nseq,
+                                             total_blocks, _p(Y1), _p(wI), _p(Ccomp), _p(KIcomp), _p(ws),
+                                             ws.numel() * ws.element_size(), _stream(stream)),
+           "csa_project_hidden_compress")

