@@ -28,7 +28,8 @@ EXPORTS = (
     "csa_status_string", "csa_hidden_row_elems", "csa_query_row_elems", "csa_project_hidden",
     "csa_project_query", "csa_launch_count", "csa_indexer_workspace_bytes", "csa_indexer_topk_noalloc",
     "csa_set_wait_limit_ns", "csa_check_wait_timeout", "csa_forward_staged", "csa_decode_staged",
-    "csa_project_compress_workspace_bytes", "csa_project_hidden_compress",
+    "csa_project_compress_workspace_bytes", "csa_project_hidden_compress", "csa_cp_workspace_bytes",
+    "csa_cp_compress", "csa_cp_queries",
 )
 
 
@@ -102,6 +103,9 @@ def lib() -> ctypes.CDLL:
             "csa_launch_count": (ctypes.c_uint64, []),
             "csa_set_wait_limit_ns": (i, [ctypes.c_ulonglong]),
             "csa_project_compress_workspace_bytes": (sz, [D, i]),
+            "csa_cp_workspace_bytes": (sz, [D, i, i]),
+            "csa_cp_compress": (i, [D, vp, vp, i, i, vp, vp, vp, vp, vp, sz, vp]),
+            "csa_cp_queries": (i, [D, vp, vp, vp, i, i, vp, vp, i, vp, vp, vp, sz, vp]),
             "csa_project_hidden_compress": (i, [D, vp, vp, i, vp, vp, i, i, vp, vp, vp, vp, vp, sz, vp]),
             "csa_forward_staged": (i, [D, vp, vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp, vp]),
             "csa_decode_staged": (i, [D, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, sz, vp, vp]),
@@ -304,3 +308,22 @@ def csa_project_hidden_compress(dims: Dims, packed, H, T, cu_seqlens, cu_blocks,
                                              total_blocks, _p(Y1), _p(wI), _p(Ccomp), _p(KIcomp), _p(ws),
                                              ws.numel() * ws.element_size(), _stream(stream)),
            "csa_project_hidden_compress")
+
+
+def csa_cp_workspace_bytes(dims: Dims, T, ctx) -> int:
+    return lib().csa_cp_workspace_bytes(_d(dims), T, ctx)
+
+
+def csa_cp_compress(dims: Dims, packed, H, T, pos0, Y1, wI, Ccomp_chunk, KIcomp_chunk, ws, stream=None):
+    """Context-parallel step 1: A1 (+A3) over a chunk of T tokens at position pos0 (H: the m rows
+    before the chunk when pos0 > 0, then the chunk)."""
+    _check(lib().csa_cp_compress(_d(dims), _p(packed), _p(H), T, pos0, _p(Y1), _p(wI), _p(Ccomp_chunk),
+                                 _p(KIcomp_chunk), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "csa_cp_compress")
+
+
+def csa_cp_queries(dims: Dims, packed, Y1, wI, T, pos0, Ccomp, KIcomp, total_blocks, O, idx_out, ws, stream=None):
+    """Context-parallel step 3: A2, A4, A5 for a chunk's queries over the whole sequence's entries."""
+    _check(lib().csa_cp_queries(_d(dims), _p(packed), _p(Y1), _p(wI), T, pos0, _p(Ccomp), _p(KIcomp), total_blocks,
+                                _p(O), _p(idx_out), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "csa_cp_queries")

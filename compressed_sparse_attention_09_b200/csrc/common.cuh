@@ -84,6 +84,8 @@ struct RowMap {
   const int* pos;         // decode: [B] token index of the new token
   int cap;                // decode: cache capacity per sequence (0 = prefill)
   int m;
+  int pos0;               // prefill: position of the first row of a sequence (0, or the
+                          // start of a context-parallel chunk of a single sequence)
 };
 
 // Visible entries of `row`: global entry index of block 0 and the count
@@ -106,7 +108,7 @@ __device__ __forceinline__ void row_entries(const RowMap& rm, int row, long long
     int mid = (lo + hi) >> 1;
     if (rm.cu_seqlens[mid] <= row) lo = mid; else hi = mid;
   }
-  int t = row - rm.cu_seqlens[lo];
+  int t = row - rm.cu_seqlens[lo] + rm.pos0;
   int a = t / rm.m;
   int b0 = rm.cu_blocks[lo], b1 = rm.cu_blocks[lo + 1];
   if (b0 < 0 || b0 + a > b1 || b1 > rm.total_blocks) {

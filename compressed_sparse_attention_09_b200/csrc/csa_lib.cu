@@ -377,10 +377,12 @@ csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int
   t.topk = d->topk; t.nhI = d->nhI; t.cI = d->cI;
   t.cu_seqlens = a.rm.cu_seqlens; t.cu_blocks = a.rm.cu_blocks; t.nseq = a.rm.nseq; t.total_blocks = NB;
   t.total_tokens = T;
+  t.pos0 = a.rm.pos0;
+  t.q_blocks = a.rm.pos0 > 0 ? T / d->m : NB;   // a chunk of one sequence: its own blocks of queries
   auto kern = d->nhI == 64 ? indexer_tc_kernel<64> : indexer_tc_kernel<32>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)idxtc::kSmem) != cudaSuccess)
     return CSA_ERR_CUDA;
-  const long long items = (long long)NB + a.rm.nseq;
+  const long long items = (long long)t.q_blocks + a.rm.nseq;
   const int grid = items < sm_count() ? (int)items : sm_count();
   kern<<<grid, idxtc::kThreads, idxtc::kSmem, st>>>(tk, tq, t);
   CSA_CHECK_LAUNCH();
@@ -963,6 +965,135 @@ csa_status csa_forward_staged(const csa_dims* d, const void* packed, const void*
     if (!events[i]) return CSA_ERR_INVALID_ARG;
   return forward_impl(d, packed, H, cu_seqlens, cu_blocks, nseq, total_tokens, total_blocks, max_seqlen, O,
                       Ccomp_out, KI_out, idx_out, ws, ws_bytes, events, stream);
+}
+
+// ------------------------------------------------------------------ context-parallel prefill
+}  // extern "C"
+
+namespace {
+// [0, a] and [0, b]: the single-sequence metadata of a context-parallel chunk
+__global__ void cp_meta_kernel(int* cu, int* cb, int a, int b) {
+  if (threadIdx.x == 0) {
+    cu[0] = 0; cu[1] = a;
+    cb[0] = 0; cb[1] = b;
+  }
+}
+
+struct CpLayout {
+  size_t meta, cc, ki, fused, y2, idx, scratch, total;
+};
+// Workspace of the two context-parallel calls for a chunk of T tokens whose
+// queries see at most ctx / m blocks (ctx = position of the chunk's end).
+CpLayout cp_layout(const csa_dims* d, int T, int ctx) {
+  const PackLayout P = pack_layout(d);
+  const size_t es = elem_size(d);
+  const int Tp = T + d->m;   // chunk plus the halo block
+  CpLayout L;
+  size_t off = 0;
+  L.meta = off; off = align_up(off + 16 * sizeof(int));
+  L.cc = off; off = align_up(off + (size_t)(Tp / d->m + 1) * d->c * es);
+  L.ki = off; off = align_up(off + (size_t)(Tp / d->m + 1) * d->cI * es);
+  L.fused = off; off = align_up(off + (fused_compress_ok(d) ? fused_layout(d, Tp).total : 0));
+  L.y2 = off; off = align_up(off + (size_t)T * P.N2 * es);
+  L.idx = off; off = align_up(off + (size_t)T * d->topk * 4);
+  L.scratch = off; off = align_up(off + indexer_scratch_bytes(ctx / d->m + 1));
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+extern "C" {
+
+size_t csa_cp_workspace_bytes(const csa_dims* d, int T, int ctx) {
+  if (check_dims(d) != CSA_OK || T <= 0 || ctx < T) return 0;
+  return cp_layout(d, T, ctx).total;
+}
+
+csa_status csa_cp_compress(const csa_dims* d, const void* packed, const void* H, int T, int pos0, void* Y1,
+                           float* wI, void* Ccomp_chunk, void* KIcomp_chunk, void* ws, size_t ws_bytes,
+                           void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!packed || !H || !Y1 || !wI || !Ccomp_chunk || !KIcomp_chunk || !ws) return CSA_ERR_INVALID_ARG;
+  if (T <= 0 || pos0 < 0 || pos0 % d->m) return CSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % kPtrAlign || reinterpret_cast<uintptr_t>(packed) % kPtrAlign)
+    return CSA_ERR_INVALID_ARG;
+  for (const void* p : {H, (const void*)Y1, (const void*)wI, (const void*)Ccomp_chunk, (const void*)KIcomp_chunk})
+    if (reinterpret_cast<uintptr_t>(p) % 16) return CSA_ERR_INVALID_ARG;
+  const CpLayout L = cp_layout(d, T, pos0 + T);
+  if (ws_bytes < L.total) return CSA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int halo = pos0 > 0 ? d->m : 0;
+  const int Tp = halo + T, nb = Tp / d->m, nb_out = T / d->m;
+  int* cu = reinterpret_cast<int*>(at(ws, L.meta));
+  int* cb = cu + 4;
+  cp_meta_kernel<<<1, 32, 0, st>>>(cu, cb, Tp, nb);
+  CSA_CHECK_LAUNCH();
+  // the halo block and the chunk as one sequence: its entry 0 (the halo
+  // block itself, which lacks its predecessor) is dropped, entries 1.. are
+  // the chunk's blocks exactly as the whole sequence would compress them
+  void* Cc = at(ws, L.cc);
+  void* KIc = at(ws, L.ki);
+  if (fused_compress_ok(d)) {
+    s = project_hidden_compress(d, packed, H, Tp, cu, cb, 1, nb, Y1, wI, Cc, KIc, at(ws, L.fused), st);
+  } else {
+    s = project_hidden(d, packed, H, Tp, Y1, wI, st);
+    if (s == CSA_OK) s = compress_kv(d, packed, Y1, Tp, cu, cb, 1, nb, Cc, KIc, st);
+  }
+  if (s != CSA_OK) return s;
+  const size_t es = elem_size(d), skip = (size_t)(halo / d->m);
+  if (nb_out > 0) {
+    if (cudaMemcpyAsync(Ccomp_chunk, static_cast<char*>(Cc) + skip * d->c * es, (size_t)nb_out * d->c * es,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(KIcomp_chunk, static_cast<char*>(KIc) + skip * d->cI * es, (size_t)nb_out * d->cI * es,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return CSA_ERR_CUDA;
+  }
+  return CSA_OK;
+}
+
+csa_status csa_cp_queries(const csa_dims* d, const void* packed, const void* Y1, const float* wI, int T, int pos0,
+                          const void* Ccomp, const void* KIcomp, int total_blocks, void* O, int* idx_out, void* ws,
+                          size_t ws_bytes, void* stream) {
+  csa_status s = check_dims(d);
+  if (s != CSA_OK) return s;
+  if (!packed || !Y1 || !wI || !Ccomp || !KIcomp || !O || !ws) return CSA_ERR_INVALID_ARG;
+  if (T <= 0 || pos0 < 0 || pos0 % d->m || total_blocks < (pos0 + T) / d->m) return CSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % kPtrAlign || reinterpret_cast<uintptr_t>(packed) % kPtrAlign)
+    return CSA_ERR_INVALID_ARG;
+  for (const void* p : {Y1, (const void*)wI, (const void*)O, Ccomp, KIcomp})
+    if (reinterpret_cast<uintptr_t>(p) % 16) return CSA_ERR_INVALID_ARG;
+  const CpLayout L = cp_layout(d, T, pos0 + T);
+  if (ws_bytes < L.total) return CSA_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  const PackLayout P = pack_layout(d);
+  const size_t es = elem_size(d);
+  const int c = d->c, cI = d->cI, NB = total_blocks;
+  int* cu = reinterpret_cast<int*>(at(ws, L.meta)) + 8;
+  int* cb = cu + 4;
+  cp_meta_kernel<<<1, 32, 0, st>>>(cu, cb, T, NB);
+  CSA_CHECK_LAUNCH();
+  char* y2 = at(ws, L.y2);
+  int* idx = idx_out ? idx_out : reinterpret_cast<int*>(at(ws, L.idx));
+  s = project_query(d, packed, static_cast<const char*>(Y1) + (size_t)(4 * c + 4 * cI) * es, P.N1b, T, y2, st);
+  if (s != CSA_OK) return s;
+  IndexerArgs ia;
+  ia.qI = y2; ia.ld_qI = P.N2; ia.wI = wI; ia.ld_wI = d->nhI; ia.KI = KIcomp; ia.idx = idx;
+  ia.topk = d->topk; ia.nhI = d->nhI; ia.sc_cap = (pos0 + T) / d->m;
+  ia.rm = RowMap{cu, cb, 1, NB, nullptr, 0, d->m, pos0};
+  if (indexer_tc_ok(d)) {
+    ia.sc_cap = (pos0 + T) / d->m + 1;
+    s = launch_indexer_tc(d, ia, T, NB, at(ws, L.scratch), L.total - L.scratch, st);
+  } else {
+    s = launch_indexer(d, ia, T, st);
+  }
+  if (s != CSA_OK) return s;
+  MqaArgs ma;
+  ma.q = y2 + (size_t)d->nhI * cI * es; ma.ld_q = P.N2; ma.C = Ccomp; ma.idx = idx;
+  ma.O = O; ma.ld_O = (long long)d->nh * c; ma.topk = d->topk; ma.nh = d->nh;
+  ma.scale_log2 = (float)(1.4426950408889634 / sqrt((double)c));
+  ma.rm = RowMap{cu, cb, 1, NB, nullptr, 0, d->m, pos0};
+  return launch_mqa(d, ma, T, st);
 }
 
 // ------------------------------------------------------------------ decode

@@ -38,6 +38,8 @@ struct IdxTcArgs {
   int topk, nhI, cI;
   const int* cu_seqlens; const int* cu_blocks;
   int nseq, total_blocks, total_tokens;
+  int q_blocks;                       // blocks of 4 queries (= total_blocks unless pos0 > 0)
+  int pos0;                           // position of the first query of sequence 0 (a chunk of one sequence)
 };
 
 namespace idxtc {
@@ -57,17 +59,21 @@ constexpr size_t kSmem = 1024 + kOffB + 256;
 constexpr int kThreads = 320;
 }  // namespace idxtc
 
-// Item `it` of the work list: compression blocks from the last one down, then
-// one tail item per sequence.  Returns false for an empty tail item and for
-// an item the metadata cannot place: its score rows would not fit the
-// scratch rows (more visible blocks than sc_cap, i.e. a max_seqlen below the
-// real length), its queries lie outside [0, total_tokens) or its blocks
-// outside [0, total_blocks).  Such an item is skipped by every role alike
-// (each evaluates the same test) and kStatusMetadata is raised.
+// Item `it` of the work list: blocks of 4 queries from the last one down,
+// then one tail item per sequence.  Normally the query blocks are the
+// compression blocks (q_blocks = total_blocks); for a context-parallel chunk
+// of one sequence whose first query sits at position pos0 (a multiple of 4),
+// query block i sees pos0/4 + i blocks of the whole sequence.  Returns false
+// for an empty tail item and for an item the metadata cannot place: its
+// score rows would not fit the scratch rows (more visible blocks than
+// sc_cap, i.e. a max_seqlen below the real length), its queries lie outside
+// [0, total_tokens) or its blocks outside [0, total_blocks).  Such an item is
+// skipped by every role alike (each evaluates the same test) and
+// kStatusMetadata is raised.
 __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, int& nq, int& avail,
                                          long long& kbase) {
-  if (it < a.total_blocks) {
-    const int g = a.total_blocks - 1 - it;
+  if (it < a.q_blocks) {
+    const int g = a.q_blocks - 1 - it;
     int lo = 0, hi = a.nseq;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -76,25 +82,28 @@ __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, 
     const int i = g - a.cu_blocks[lo];
     tok0 = a.cu_seqlens[lo] + 4 * i;
     nq = 4;
-    avail = i;
+    avail = i + (a.pos0 >> 2);
     kbase = a.cu_blocks[lo];
     if (i < 0 || tok0 < 0 || tok0 + 4 > a.cu_seqlens[lo + 1] || a.cu_seqlens[lo + 1] > a.total_tokens ||
-        avail >= a.sc_cap) {
+        avail >= a.sc_cap || kbase + avail > a.total_blocks) {
       flag_status(kStatusMetadata);
       return false;
     }
     return true;
   }
-  const int b = it - a.total_blocks;
+  const int b = it - a.q_blocks;
   const int L = a.cu_seqlens[b + 1] - a.cu_seqlens[b];
   nq = L & 3;
   tok0 = a.cu_seqlens[b + 1] - nq;
-  avail = L >> 2;
+  avail = (L >> 2) + (a.pos0 >> 2);
   kbase = a.cu_blocks[b];
   // every sequence's tail item also checks that cu_blocks gives the sequence
-  // floor(L/4) blocks, so that no block of queries goes unvisited unnoticed
+  // floor(L/4) blocks (for a chunk: at least the blocks its queries see), so
+  // that no block of queries goes unvisited unnoticed
+  const int have = a.cu_blocks[b + 1] - kbase;
   if (L < 0 || a.cu_seqlens[b] < 0 || a.cu_seqlens[b + 1] > a.total_tokens || kbase < 0 ||
-      a.cu_blocks[b + 1] - kbase != avail || kbase + avail > a.total_blocks || (nq > 0 && avail >= a.sc_cap)) {
+      (a.pos0 == 0 ? have != avail : have < avail) || kbase + avail > a.total_blocks ||
+      (nq > 0 && avail >= a.sc_cap)) {
     flag_status(kStatusMetadata);
     return false;
   }

@@ -295,6 +295,51 @@ csa_status csa_forward_staged(const csa_dims* dims, const void* packed, const vo
                               int* idx_out, void* ws, size_t ws_bytes, void* const* events, void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Context-parallel prefill of one sequence                                */
+/* ---------------------------------------------------------------------- */
+/* The forward pass of one sequence split into chunks of consecutive tokens
+ * (chunk starts on block boundaries), for processes that each own some
+ * chunks.  Entry i needs only tokens m(i-1) .. m(i+1)-1 (eqs. 3-4) and query
+ * t needs only the entries s < floor(t/m) (eq. 8), so a rank compresses its
+ * chunks alone, the caller exchanges the entries (one all-gather), and each
+ * rank then evaluates its chunks' queries alone.  Results are bit-identical
+ * to csa_forward on the whole sequence. */
+
+/* Workspace bytes for a chunk of T tokens that ends at position ctx (the
+ * same buffer may serve both calls of that chunk; 0 if invalid). */
+size_t csa_cp_workspace_bytes(const csa_dims* dims, int T, int ctx);
+
+/* Step 1: eqs. (1), (2), (5), (7), the indexer-key projections and eqs.
+ * (3)-(4) for a chunk of T tokens starting at position pos0 (a multiple of
+ * m; T a multiple of m except for the sequence's last chunk).
+ * H [dev]     : the m hidden rows before the chunk (when pos0 > 0), then the
+ *               chunk's T rows.
+ * Y1, wI [dev]: [m + T (or T when pos0 = 0), csa_hidden_row_elems] and
+ *               [same rows, nhI] fp32 outputs (the projection rows step 2
+ *               reads; the halo rows come first).
+ * Ccomp_chunk, KIcomp_chunk [dev]: the chunk's floor(T/m) entries, i.e.
+ *               global entries pos0/m .. pos0/m + floor(T/m) - 1.
+ * ws [dev]    : >= csa_cp_workspace_bytes(dims, T, pos0 + T), 256-byte
+ *               aligned. */
+csa_status csa_cp_compress(const csa_dims* dims, const void* packed, const void* H, int T, int pos0,
+                           void* Y1, float* wI, void* Ccomp_chunk, void* KIcomp_chunk, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* Step 2 (after the caller has gathered every chunk's entries): eqs. (6),
+ * (10), (8), (9), (11) for the chunk's T queries at positions pos0 ..
+ * pos0 + T - 1 over the whole sequence's entries.
+ * Y1, wI [dev]: the chunk's own rows of step 1's outputs (without the halo
+ *               rows).
+ * Ccomp, KIcomp [dev]: [total_blocks, c] / [total_blocks, cI], every entry
+ *               of the sequence; total_blocks >= (pos0 + T) / m.
+ * O [dev]     : [T, nh*c];  idx_out [dev, optional]: [T, topk] (global
+ *               block indices).
+ * ws [dev]    : as for step 1. */
+csa_status csa_cp_queries(const csa_dims* dims, const void* packed, const void* Y1, const float* wI, int T,
+                          int pos0, const void* Ccomp, const void* KIcomp, int total_blocks, void* O,
+                          int* idx_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Decode over a compressed cache                                          */
 /* ---------------------------------------------------------------------- */
 
