@@ -362,7 +362,7 @@ bool indexer_tc_ok(const csa_dims* d) {
 
 
 csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int NB, void* ws, size_t ws_bytes,
-                             cudaStream_t st) {
+                             cudaStream_t st, bool chunk = false) {
   CSA_RANGE("A4 indexer_topk");
   const int sc_cap = padded_cap(a.sc_cap > 0 ? a.sc_cap : 1);
   if (!ws || ws_bytes < indexer_scratch_bytes(sc_cap) || reinterpret_cast<uintptr_t>(ws) % 16)
@@ -378,7 +378,8 @@ csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int
   t.cu_seqlens = a.rm.cu_seqlens; t.cu_blocks = a.rm.cu_blocks; t.nseq = a.rm.nseq; t.total_blocks = NB;
   t.total_tokens = T;
   t.pos0 = a.rm.pos0;
-  t.q_blocks = a.rm.pos0 > 0 ? T / d->m : NB;   // a chunk of one sequence: its own blocks of queries
+  t.chunk = chunk ? 1 : 0;
+  t.q_blocks = chunk ? T / d->m : NB;   // a chunk of one sequence: its own blocks of queries
   auto kern = d->nhI == 64 ? indexer_tc_kernel<64> : indexer_tc_kernel<32>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)idxtc::kSmem) != cudaSuccess)
     return CSA_ERR_CUDA;
@@ -1083,7 +1084,7 @@ csa_status csa_cp_queries(const csa_dims* d, const void* packed, const void* Y1,
   ia.rm = RowMap{cu, cb, 1, NB, nullptr, 0, d->m, pos0};
   if (indexer_tc_ok(d)) {
     ia.sc_cap = (pos0 + T) / d->m + 1;
-    s = launch_indexer_tc(d, ia, T, NB, at(ws, L.scratch), L.total - L.scratch, st);
+    s = launch_indexer_tc(d, ia, T, NB, at(ws, L.scratch), L.total - L.scratch, st, true);
   } else {
     s = launch_indexer(d, ia, T, st);
   }

@@ -38,8 +38,9 @@ struct IdxTcArgs {
   int topk, nhI, cI;
   const int* cu_seqlens; const int* cu_blocks;
   int nseq, total_blocks, total_tokens;
-  int q_blocks;                       // blocks of 4 queries (= total_blocks unless pos0 > 0)
-  int pos0;                           // position of the first query of sequence 0 (a chunk of one sequence)
+  int q_blocks;                       // blocks of 4 queries (= total_blocks unless chunk)
+  int pos0;                           // chunk: position of its first query
+  int chunk;                          // 1: the queries are one chunk of one sequence (cu_blocks = [0, all blocks])
 };
 
 namespace idxtc {
@@ -102,7 +103,7 @@ __device__ __forceinline__ bool idx_item(const IdxTcArgs& a, int it, int& tok0, 
   // that no block of queries goes unvisited unnoticed
   const int have = a.cu_blocks[b + 1] - kbase;
   if (L < 0 || a.cu_seqlens[b] < 0 || a.cu_seqlens[b + 1] > a.total_tokens || kbase < 0 ||
-      (a.pos0 == 0 ? have != avail : have < avail) || kbase + avail > a.total_blocks ||
+      (a.chunk ? have < avail : have != avail) || kbase + avail > a.total_blocks ||
       (nq > 0 && avail >= a.sc_cap)) {
     flag_status(kStatusMetadata);
     return false;
