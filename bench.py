@@ -714,6 +714,39 @@ def run_stage(args):
         raise SystemExit(1)
 
 
+def run_indexer_only(args):
+    """csa_indexer_topk alone on seeded q^I, w^I and K^IComp with the sizes of
+    a workload (no projections: a few GB on the device even at n = 131072),
+    warmup + steps launches; for DRAM-traffic captures of the indexer."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.workloads()[args.workload]
+    d = w.dims
+    T, nseq, maxlen = sum(w.seqlens), len(w.seqlens), max(w.seqlens)
+    cu, cb = csa.cu_from_lengths(w.seqlens, d.m)
+    NB = int(cb[-1])
+    g = torch.Generator(device=dev).manual_seed(w.seed + 11)
+    qI = torch.randn(T, d.nhI * d.cI, device=dev, generator=g).to(torch.bfloat16)
+    wI = torch.randn(T, d.nhI, device=dev, generator=g)
+    KI = (0.5 * torch.randn(NB, d.cI, device=dev, generator=g)).to(torch.bfloat16)
+    idx = torch.empty(T, d.topk, dtype=torch.int32, device=dev)
+    ws = torch.empty(csa.csa_indexer_workspace_bytes(d, T, nseq, maxlen), dtype=torch.uint8, device=dev)
+    cu, cb = cu.to(dev), cb.to(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for i in range(args.warmup + args.steps):
+        if i == args.warmup:
+            ev[0].record()
+        csa.csa_indexer_topk(d, qI, d.nhI * d.cI, wI, d.nhI, KI, cu, cb, nseq, T, NB, maxlen, idx, ws)
+    ev[1].record()
+    torch.cuda.synchronize()
+    st = csa.csa_get_device_status()
+    ms = ev[0].elapsed_time(ev[1]) / max(args.steps, 1)
+    print(json.dumps({"stage": "A4_indexer_topk (seeded inputs)", "workload": args.workload, "ms": ms,
+                      "scratch_bytes": ws.numel(), "status": csa.status_string(st)}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
+
+
 def runner_T(w):
     return sum(w.seqlens)
 
@@ -733,7 +766,10 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--stage", choices=["A1_project_hidden", "A2_project_query", "A3_compress", "A4_indexer_topk",
-                                        "A5_sparse_mqa"], help="run only this stage (profiling)")
+                                        "A5_sparse_mqa", "A1A3_project_compress"],
+                    help="run only this stage (profiling)")
+    ap.add_argument("--indexer-only", action="store_true",
+                    help="run csa_indexer_topk alone on seeded inputs of the workload's sizes (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -742,6 +778,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.indexer_only:
+        run_indexer_only(args)
         return
     if args.stage:
         run_stage(args)

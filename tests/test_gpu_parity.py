@@ -455,11 +455,23 @@ def test_stage_sparse_mqa_tensor_core_many_blocks(fn):
 def test_stage_sparse_mqa_tensor_core_rescale():
     """Scores that grow along the row (entries s < 256 scaled by 0.025, the
     rest by 0.5, q with std 6: scaled scores of std ~4 in log2 units after
-    near-zero ones), so the running maximum of most heads rises by far more
-    than the lazy threshold and O and l are rescaled in flight.  The entry
-    scale keeps |O| near unit size, where the absolute bar applies."""
+    near-zero ones): the running maximum of most heads rises by tens of log2
+    units, far more than the kernel's lazy threshold (8), so O and l are
+    rescaled in flight.  The entry scale keeps |O| near unit size, where the
+    absolute bar applies."""
     dims = csa.Dims(d=64, c=512, m=4, cI=32, nhI=4, nh=64, dc=64, topk=640, dtype=csa.CSA_BF16)
     assert _mqa_case(dims, [2600], 59, _first_k, q_std=6.0,
+                     c_row_scale=lambda s: np.where(s < 256, 0.025, 0.5)) == 0
+
+
+def test_stage_sparse_mqa_tensor_core_rescale_in_flight():
+    """Scores whose running maximum grows by ~100 in log2 units along the row
+    (entries s < 256 scaled by 0.025, the rest by 0.5, q with std 50: scaled
+    scores of std ~36 in log2 units after near-zero ones): large jumps of the
+    maximum, rescaled in flight, and a softmax concentrated on few entries.
+    |O| stays near 0.5."""
+    dims = csa.Dims(d=64, c=512, m=4, cI=32, nhI=4, nh=64, dc=64, topk=640, dtype=csa.CSA_BF16)
+    assert _mqa_case(dims, [2600], 60, _first_k, q_std=50.0,
                      c_row_scale=lambda s: np.where(s < 256, 0.025, 0.5)) == 0
 
 
