@@ -314,6 +314,21 @@ class DecodeRunner:
         csa.csa_decode_staged(self.dims, self.packed, self.h, self.pos, self.ring, self.Cc, self.Kc, self.clen,
                               self.cap, self.B, self.O, None, self.ws, events)
 
+    def quantise_keys(self):
+        """The key cache as E4M3 codes + per-entry scales (for the q8 steps)."""
+        d = self.dims
+        self.Kq = torch.empty(self.B, self.cap, d.cI, dtype=torch.uint8, device=self.Kc.device)
+        self.Ks = torch.empty(self.B, self.cap, dtype=torch.float32, device=self.Kc.device)
+        csa.csa_quantize_keys_e4m3(self.Kc, d.cI, self.B * self.cap, d.cI, self.Kq, self.Ks)
+
+    def step_q8(self):
+        csa.csa_decode_q8(self.dims, self.packed, self.h, self.pos, self.ring, self.Cc, self.Kq, self.Ks, self.clen,
+                          self.cap, self.B, self.O, None, self.ws)
+
+    def step_q8_staged(self, events):
+        csa.csa_decode_q8_staged(self.dims, self.packed, self.h, self.pos, self.ring, self.Cc, self.Kq, self.Ks,
+                                 self.clen, self.cap, self.B, self.O, None, self.ws, events)
+
     def bytes_per_step(self):
         d = self.dims
         N1 = 4 * d.c + 4 * d.cI + d.dc + d.nhI
@@ -562,8 +577,33 @@ def run_decode(dev, args, peaks, flush, stream):
         stages[n] = {"ms": ms, "bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm"], "algorithmic_bytes": nbytes[n]}
     gbs = dr.bytes_per_step() / (dms / 1000.0) / 1e9
+    # the same step over the E4M3 key cache (codes + per-entry scales)
+    dr.quantise_keys()
+    for _ in range(3):
+        dr.step_q8()
+    qms = statistics.mean(timed_steps(dr.step_q8, args.steps, no_flush, stream))
+    q_in_step = staged_step_ms(dr.step_q8_staged, len(names), max(3, min(args.steps, 50)), no_flush, stream)
+    st = csa.csa_get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after the e4m3-key decode: {csa.status_string(st)}")
+    d = w.dims
+    avail = w.decode_pos // d.m
+    qbytes = dict(nbytes)
+    qbytes["A4_indexer_scores"] = dr.B * avail * (d.cI + 4) + dr.B * avail * 4   # codes + scales read, scores written
+    q_total = dr.bytes_per_step() - dr.B * avail * d.cI * 2 + dr.B * avail * (d.cI + 4)
+    q_stages = {}
+    for n, ms in zip(names, q_in_step):
+        gbs = qbytes[n] / (ms / 1000.0) / 1e9
+        q_stages[n] = {"ms": ms, "bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                       "frac": gbs / peaks["hbm"], "algorithmic_bytes": qbytes[n]}
+    qgbs = q_total / (qms / 1000.0) / 1e9
+    e4m3 = {"value": dr.B / (qms / 1000.0), "unit": "tokens/s", "ms_per_step": qms,
+            "cache": "K^IComp as E4M3 codes + one fp32 scale per entry; C^Comp bf16",
+            "roofline": {"bound": "hbm", "achieved": qgbs, "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": qgbs / peaks["hbm"], "algorithmic_bytes": q_total},
+            "stages_in_step": q_stages}
     out = {"value": dr.B / (dms / 1000.0), "unit": "tokens/s", "ms_per_step": dms,
-           "ms_per_step_l2_flushed": dms_flushed,
+           "ms_per_step_l2_flushed": dms_flushed, "e4m3_keys": e4m3,
            "l2": "not flushed: each step reads 1.6 GB (> 126 MB L2); ms_per_step_l2_flushed = the same with a "
                  "512 MiB write before each step",
            "workload": "64 sequences x 1 new token over 16384 cached entries (t=65536), nh=128, k=2048",

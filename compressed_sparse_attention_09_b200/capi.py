@@ -29,7 +29,7 @@ EXPORTS = (
     "csa_project_query", "csa_launch_count", "csa_indexer_workspace_bytes", "csa_indexer_topk_noalloc",
     "csa_set_wait_limit_ns", "csa_check_wait_timeout", "csa_forward_staged", "csa_decode_staged",
     "csa_project_compress_workspace_bytes", "csa_project_hidden_compress", "csa_cp_workspace_bytes",
-    "csa_cp_compress", "csa_cp_queries",
+    "csa_cp_compress", "csa_cp_queries", "csa_quantize_keys_e4m3", "csa_decode_q8", "csa_decode_q8_staged",
 )
 
 
@@ -104,6 +104,9 @@ def lib() -> ctypes.CDLL:
             "csa_set_wait_limit_ns": (i, [ctypes.c_ulonglong]),
             "csa_project_compress_workspace_bytes": (sz, [D, i]),
             "csa_cp_workspace_bytes": (sz, [D, i, i]),
+            "csa_quantize_keys_e4m3": (i, [vp, ctypes.c_longlong, i, i, vp, vp, vp]),
+            "csa_decode_q8": (i, [D, vp, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, sz, vp]),
+            "csa_decode_q8_staged": (i, [D, vp, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, sz, vp, vp]),
             "csa_cp_compress": (i, [D, vp, vp, i, i, vp, vp, vp, vp, vp, sz, vp]),
             "csa_cp_queries": (i, [D, vp, vp, vp, i, i, vp, vp, i, vp, vp, vp, sz, vp]),
             "csa_project_hidden_compress": (i, [D, vp, vp, i, vp, vp, i, i, vp, vp, vp, vp, vp, sz, vp]),
@@ -327,3 +330,25 @@ def csa_cp_queries(dims: Dims, packed, Y1, wI, T, pos0, Ccomp, KIcomp, total_blo
     _check(lib().csa_cp_queries(_d(dims), _p(packed), _p(Y1), _p(wI), T, pos0, _p(Ccomp), _p(KIcomp), total_blocks,
                                 _p(O), _p(idx_out), _p(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "csa_cp_queries")
+
+
+def csa_quantize_keys_e4m3(KI, ld, n, w, codes, scales, stream=None):
+    """bf16 rows [n, w] (row stride ld) to E4M3 codes [n, w] and fp32 scales [n]."""
+    _check(lib().csa_quantize_keys_e4m3(_p(KI), ld, n, w, _p(codes), _p(scales), _stream(stream)),
+           "csa_quantize_keys_e4m3")
+
+
+def csa_decode_q8(dims: Dims, packed, h, pos, ring, Ccache, KIcodes, KIscale, cache_len, cap, B, O, idx_out=None,
+                  ws=None, stream=None):
+    """csa_decode with the indexer-key cache as E4M3 codes + per-entry scales."""
+    _check(lib().csa_decode_q8(_d(dims), _p(packed), _p(h), _p(pos), _p(ring), _p(Ccache), _p(KIcodes), _p(KIscale),
+                               _p(cache_len), cap, B, _p(O), _p(idx_out), _p(ws), ws.numel() * ws.element_size(),
+                               _stream(stream)), "csa_decode_q8")
+
+
+def csa_decode_q8_staged(dims: Dims, packed, h, pos, ring, Ccache, KIcodes, KIscale, cache_len, cap, B, O, idx_out,
+                         ws, events, stream=None):
+    _check(lib().csa_decode_q8_staged(_d(dims), _p(packed), _p(h), _p(pos), _p(ring), _p(Ccache), _p(KIcodes),
+                                      _p(KIscale), _p(cache_len), cap, B, _p(O), _p(idx_out), _p(ws),
+                                      ws.numel() * ws.element_size(), _event_array(events), _stream(stream)),
+           "csa_decode_q8_staged")

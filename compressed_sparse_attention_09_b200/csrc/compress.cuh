@@ -15,6 +15,8 @@
 // thread takes exactly one (entry, channel group), so no thread waits on a
 // second round of loads.
 #pragma once
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 
 namespace csa {
@@ -205,12 +207,17 @@ struct AppendArgs {
   const float* Ba; const float* Bb;     // [m, c]
   const float* BaI; const float* BbI;   // [m, cI]
   int c, cI, cap, ring_w;
+  uint8_t* KIcodes;     // quantised key cache (Q8): [B, cap, cI] E4M3 codes
+  float* KIscale;       // [B, cap] scales
 };
 
 // One CTA per sequence: store the token's row in ring slot t mod 2m, then, if
-// t closes block i = (t+1)/m - 1, compress that block from the ring.
-template <typename T, int M>
+// t closes block i = (t+1)/m - 1, compress that block from the ring.  Q8:
+// the indexer-key entry goes to an E4M3 cache (its bf16 value quantised with
+// one scale, max |v| / 448) instead of a bf16 one.
+template <typename T, int M, bool Q8 = false>
 __global__ void __launch_bounds__(256) cache_append_kernel(AppendArgs a) {
+  __shared__ float ki_s[1024];
   const int b = blockIdx.x;
   const int t = a.pos[b];
   if (t < 0) {
@@ -257,9 +264,23 @@ __global__ void __launch_bounds__(256) cache_append_kernel(AppendArgs a) {
     }
     const float v = compress_channel<M>(la, lb, ca, cb, has_prev);
     if (main) static_cast<T*>(a.Ccache)[((long long)b * a.cap + i) * c + ch] = from_f32<T>(v);
+    else if (Q8) ki_s[ch] = to_f32(from_f32<T>(v));   // the entry as stored in T, then quantised below
     else static_cast<T*>(a.KIcache)[((long long)b * a.cap + i) * cI + ch] = from_f32<T>(v);
   }
   __syncthreads();
+  if constexpr (Q8) {
+    if (threadIdx.x < 32) {
+      float amax = 0.f;
+      for (int j = threadIdx.x; j < cI; j += 32) amax = fmaxf(amax, fabsf(ki_s[j]));
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      const float scale = amax > 0.f ? amax / 448.f : 1.f;
+      uint8_t* dst = a.KIcodes + ((long long)b * a.cap + i) * cI;
+      for (int j = threadIdx.x; j < cI; j += 32)
+        dst[j] = (uint8_t)__nv_cvt_float_to_fp8(ki_s[j] / scale, __NV_SATFINITE, __NV_E4M3);
+      if (threadIdx.x == 0) a.KIscale[(long long)b * a.cap + i] = scale;
+    }
+  }
   if (threadIdx.x == 0) a.cache_len[b] = i + 1;
 }
 

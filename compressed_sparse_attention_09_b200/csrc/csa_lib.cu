@@ -15,6 +15,7 @@
 #include "../../include/csa.h"
 #include "common.cuh"
 #include "compress.cuh"
+#include "decode_q8.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tcgen05.cuh"
 #include "indexer_simt.cuh"
@@ -213,6 +214,37 @@ bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d
   cuuint32_t box[3] = {b0, b1, b2};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Row-major byte matrix [outer, inner] (row stride row_bytes), boxes of
+// box_inner bytes x box_outer rows, 128-byte swizzle.
+bool make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                  uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  if (reinterpret_cast<uintptr_t>(base) % 16 || row_bytes % 16) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp16 tensor [d2, d1, d0] as make_tmap_bf16_3d.
+bool make_tmap_f16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                      uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  if (reinterpret_cast<uintptr_t>(base) % 16 || s1 % 16 || s2 % 16) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1106,9 +1138,10 @@ int csa_ring_row_elems(const csa_dims* d) {
 namespace {
 csa_status launch_append(const csa_dims* d, const void* packed, const void* rows, long long ld_rows,
                          const int* pos, void* ring, void* Ccache, void* KIcache, int* cache_len, int cap,
-                         int B, cudaStream_t st) {
+                         int B, cudaStream_t st, uint8_t* KIcodes = nullptr, float* KIscale = nullptr) {
   CSA_RANGE("A6 cache_append");
   if (B == 0) return CSA_OK;
+  const bool q8 = KIcodes != nullptr;
   const PackLayout P = pack_layout(d);
   AppendArgs a;
   a.rows = rows; a.ld_rows = ld_rows; a.pos = pos; a.ring = ring; a.Ccache = Ccache; a.KIcache = KIcache;
@@ -1118,10 +1151,12 @@ csa_status launch_append(const csa_dims* d, const void* packed, const void* rows
   a.BaI = reinterpret_cast<const float*>(at((void*)packed, P.baI));
   a.BbI = reinterpret_cast<const float*>(at((void*)packed, P.bbI));
   a.c = d->c; a.cI = d->cI; a.cap = cap; a.ring_w = 4 * d->c + 4 * d->cI;
-#define CSA_APPEND_CASE(MM)                                                     \
-  case MM:                                                                      \
-    if (d->dtype == CSA_BF16) cache_append_kernel<bf16, MM><<<B, 256, 0, st>>>(a); \
-    else cache_append_kernel<float, MM><<<B, 256, 0, st>>>(a);                  \
+  a.KIcodes = KIcodes; a.KIscale = KIscale;
+#define CSA_APPEND_CASE(MM)                                                                \
+  case MM:                                                                                 \
+    if (q8) cache_append_kernel<bf16, MM, true><<<B, 256, 0, st>>>(a);                     \
+    else if (d->dtype == CSA_BF16) cache_append_kernel<bf16, MM><<<B, 256, 0, st>>>(a);    \
+    else cache_append_kernel<float, MM><<<B, 256, 0, st>>>(a);                             \
     break;
   switch (d->m) {
     CSA_APPEND_CASE(1)
@@ -1136,7 +1171,7 @@ csa_status launch_append(const csa_dims* d, const void* packed, const void* rows
 }
 
 struct DecLayout {
-  size_t y1, wI, y2, idx, scratch, split, total;
+  size_t y1, wI, y2, idx, scratch, split, qf16, total;
 };
 DecLayout dec_layout(const csa_dims* d, int B, int cap) {
   const PackLayout P = pack_layout(d);
@@ -1149,6 +1184,7 @@ DecLayout dec_layout(const csa_dims* d, int B, int cap) {
   L.idx = off; off = align_up(off + (size_t)B * d->topk * 4);
   L.scratch = off; off = align_up(off + (size_t)B * (size_t)cap * 4);
   L.split = off; off = align_up(off + gemm_split_bytes(P.N1, B));   // K-split sums of the A1 projection
+  L.qf16 = off; off = align_up(off + (size_t)B * d->nhI * d->cI * 2);   // q^I in fp16 (quantised key cache)
   L.total = off;
   return L;
 }
@@ -1180,6 +1216,42 @@ csa_status launch_indexer_decode_tc(const csa_dims* d, const IndexerArgs& a, int
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }
+// Decode rows over an E4M3 key cache: q^I to fp16, the score rows (codes
+// widened in shared memory, entry scales in the epilogue), then the same
+// per-sequence selection as the bf16 cache.
+csa_status launch_indexer_decode_q8(const csa_dims* d, const IndexerArgs& a, const uint8_t* codes,
+                                    const float* scales, int B, int cap, float* scratch, void* qf16, cudaStream_t st,
+                                    cudaEvent_t after_scores = nullptr) {
+  CSA_RANGE("A4 indexer_topk (decode, e4m3 keys)");
+  const int w = d->nhI * d->cI;
+  bf16_to_f16_rows_kernel<<<(unsigned)(((long long)B * w + 255) / 256), 256, 0, st>>>(
+      static_cast<const bf16*>(a.qI), a.ld_qI, B, w, static_cast<__half*>(qf16));
+  CSA_CHECK_LAUNCH();
+  CUtensorMap tk, tq;
+  if (!make_tmap_u8(&tk, codes, d->cI, (uint64_t)B * cap, (uint64_t)d->cI, 128, idxq8::kM) ||
+      !make_tmap_f16_3d(&tq, qf16, d->cI, d->nhI, B, (uint64_t)d->cI * 2, (uint64_t)w * 2, 64, d->nhI, 1))
+    return CSA_ERR_UNSUPPORTED;
+  IdxDecQ8Args t;
+  t.wI = a.wI; t.ld_wI = a.ld_wI; t.pos = a.rm.pos; t.kscale = scales; t.scratch = scratch; t.B = B; t.cap = cap;
+  t.m = d->m; t.nhI = d->nhI; t.tiles_per_seq = (cap + idxq8::kM - 1) / idxq8::kM;
+  if (cudaFuncSetAttribute(indexer_decode_q8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)idxq8::kSmem) != cudaSuccess)
+    return CSA_ERR_CUDA;
+  const long long items = (long long)B * t.tiles_per_seq;
+  const int grid = items < sm_count() ? (int)items : sm_count();
+  indexer_decode_q8_kernel<<<grid, idxq8::kThreads, idxq8::kSmem, st>>>(tk, tq, t);
+  CSA_CHECK_LAUNCH();
+  if (after_scores && cudaEventRecord(after_scores, st) != cudaSuccess) return CSA_ERR_CUDA;
+  if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsel::kSmem) !=
+      cudaSuccess)
+    return CSA_ERR_CUDA;
+  decode_select_kernel<<<B, 512, dsel::kSmem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+// The quantised key cache's requirements: bf16 path, c^I = 128, n_h^I in {32, 64}.
+bool q8_ok(const csa_dims* d) { return d->dtype == CSA_BF16 && d->cI == 128 && (d->nhI == 32 || d->nhI == 64); }
 }  // namespace
 
 csa_status csa_cache_append(const csa_dims* d, const void* packed, const void* rows, const int* pos,
@@ -1203,10 +1275,17 @@ size_t csa_decode_workspace_bytes(const csa_dims* d, int B, int cap) {
 namespace {
 csa_status decode_impl(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
                        void* Ccache, void* KIcache, int* cache_len, int cap, int B, void* O, int* idx_out,
-                       void* ws, size_t ws_bytes, void* const* ev, void* stream) {
+                       void* ws, size_t ws_bytes, void* const* ev, void* stream, uint8_t* KIcodes = nullptr,
+                       float* KIscale = nullptr) {
   CSA_RANGE("csa_decode");
   csa_status s = check_dims(d);
   if (s != CSA_OK) return s;
+  const bool q8 = KIcodes != nullptr;
+  if (q8) {
+    if (!KIscale) return CSA_ERR_INVALID_ARG;
+    if (!q8_ok(d) || reinterpret_cast<uintptr_t>(KIcodes) % 16) return CSA_ERR_UNSUPPORTED;
+    KIcache = KIcodes;   // stands in for the (absent) bf16 key cache in the checks below
+  }
   if (!packed || !h || !pos || !ring || !Ccache || !KIcache || !cache_len || !O || !ws) return CSA_ERR_INVALID_ARG;
   if (cap <= 0 || B < 0) return CSA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(ws) % kPtrAlign || reinterpret_cast<uintptr_t>(packed) % kPtrAlign)
@@ -1226,7 +1305,7 @@ csa_status decode_impl(const csa_dims* d, const void* packed, const void* h, con
   s = project_hidden(d, packed, h, B, y1, wI, st, reinterpret_cast<float*>(at(ws, L.split)),
                      L.total - L.split);
   if (s != CSA_OK || (s = mark(ev, 1, st)) != CSA_OK) return s;
-  s = launch_append(d, packed, y1, P.N1b, pos, ring, Ccache, KIcache, cache_len, cap, B, st);
+  s = launch_append(d, packed, y1, P.N1b, pos, ring, Ccache, KIcache, cache_len, cap, B, st, KIcodes, KIscale);
   if (s != CSA_OK || (s = mark(ev, 2, st)) != CSA_OK) return s;
   s = project_query(d, packed, y1 + (size_t)(4 * c + 4 * cI) * es, P.N1b, B, y2, st);
   if (s != CSA_OK || (s = mark(ev, 3, st)) != CSA_OK) return s;
@@ -1234,8 +1313,11 @@ csa_status decode_impl(const csa_dims* d, const void* packed, const void* h, con
   ia.qI = y2; ia.ld_qI = P.N2; ia.wI = wI; ia.ld_wI = d->nhI; ia.KI = KIcache; ia.idx = idx;
   ia.topk = d->topk; ia.nhI = d->nhI; ia.sc_cap = cap;
   ia.rm = RowMap{nullptr, nullptr, 0, 0, pos, cap, d->m};
-  if (d->dtype == CSA_BF16 && (d->nhI == 32 || d->nhI == 64) && (d->cI == 64 || d->cI == 128) &&
-      reinterpret_cast<uintptr_t>(KIcache) % 16 == 0) {
+  if (q8) {
+    s = launch_indexer_decode_q8(d, ia, KIcodes, KIscale, B, cap, reinterpret_cast<float*>(at(ws, L.scratch)),
+                                 at(ws, L.qf16), st, ev ? (cudaEvent_t)ev[4] : nullptr);
+  } else if (d->dtype == CSA_BF16 && (d->nhI == 32 || d->nhI == 64) && (d->cI == 64 || d->cI == 128) &&
+             reinterpret_cast<uintptr_t>(KIcache) % 16 == 0) {
     s = launch_indexer_decode_tc(d, ia, B, cap, reinterpret_cast<float*>(at(ws, L.scratch)), st,
                                  ev ? (cudaEvent_t)ev[4] : nullptr);
   } else {
@@ -1271,6 +1353,36 @@ csa_status csa_decode_staged(const csa_dims* d, const void* packed, const void* 
     if (!events[i]) return CSA_ERR_INVALID_ARG;
   return decode_impl(d, packed, h, pos, ring, Ccache, KIcache, cache_len, cap, B, O, idx_out, ws, ws_bytes,
                      events, stream);
+}
+
+csa_status csa_quantize_keys_e4m3(const void* KI, long long ld, int n, int w, void* codes, float* scales,
+                                  void* stream) {
+  if (!KI || !codes || !scales || n < 0 || w <= 0 || w % 32 || ld < w) return CSA_ERR_INVALID_ARG;
+  if (n == 0) return CSA_OK;
+  const long long threads = (long long)n * 32;
+  quantize_rows_e4m3_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, (cudaStream_t)stream>>>(
+      static_cast<const bf16*>(KI), ld, n, w, static_cast<uint8_t*>(codes), scales);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+csa_status csa_decode_q8(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
+                         void* Ccache, void* KIcodes, float* KIscale, int* cache_len, int cap, int B, void* O,
+                         int* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!KIcodes) return CSA_ERR_INVALID_ARG;
+  return decode_impl(d, packed, h, pos, ring, Ccache, nullptr, cache_len, cap, B, O, idx_out, ws, ws_bytes,
+                     nullptr, stream, static_cast<uint8_t*>(KIcodes), KIscale);
+}
+
+csa_status csa_decode_q8_staged(const csa_dims* d, const void* packed, const void* h, const int* pos, void* ring,
+                                void* Ccache, void* KIcodes, float* KIscale, int* cache_len, int cap, int B,
+                                void* O, int* idx_out, void* ws, size_t ws_bytes, void* const* events,
+                                void* stream) {
+  if (!KIcodes || !events) return CSA_ERR_INVALID_ARG;
+  for (int i = 0; i < 7; ++i)
+    if (!events[i]) return CSA_ERR_INVALID_ARG;
+  return decode_impl(d, packed, h, pos, ring, Ccache, nullptr, cache_len, cap, B, O, idx_out, ws, ws_bytes, events,
+                     stream, static_cast<uint8_t*>(KIcodes), KIscale);
 }
 
 }  // extern "C"

@@ -431,7 +431,7 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
   constexpr int N = 4 * NHI;                    // MMA N: (query, head) pairs
   const int kchunks = a.cI / 64;
   constexpr uint32_t tmem_cols = N <= 128 ? 256 : 512;
-  const int items = a.total_blocks + a.nseq;
+  const int items = a.q_blocks + a.nseq;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);

@@ -388,6 +388,40 @@ csa_status csa_decode_staged(const csa_dims* dims, const void* packed, const voi
                              void* stream);
 
 /* ---------------------------------------------------------------------- */
+/* Decode over a quantised indexer-key cache (E4M3)                        */
+/* ---------------------------------------------------------------------- */
+/* A cache format of this library (the page stores C^Comp / K^IComp without
+ * fixing a precision): K^IComp entries as FP8 E4M3 codes with one fp32 scale
+ * per entry, half the bytes the indexer streams per decode step.  For an
+ * entry v (its cI values as stored in bf16): scale = max_j |v_j| / 448 in
+ * fp32 (1 for an all-zero entry), code_j = E4M3(v_j / scale) rounded to
+ * nearest even and saturated to +-448; the entry stands for code * scale.
+ * The indexer multiplies the codes (widened exactly to fp16) by q^I in fp16
+ * and applies each entry's scale to its head-weighted sum (the scale is
+ * positive, so it commutes with the ReLU).  C^Comp stays bf16. */
+
+/* Quantises n rows of w bf16 values (row stride ld elements; w a multiple
+ * of 32) into codes [n, w] (one byte each) and scales [n] (fp32), as above:
+ * e.g. a bf16 key cache [B * cap, cI] into the quantised cache. */
+csa_status csa_quantize_keys_e4m3(const void* KI, long long ld, int n, int w, void* codes, float* scales,
+                                  void* stream);
+
+/* csa_decode with the indexer-key cache quantised: KIcodes [B, cap, cI]
+ * (E4M3 codes, 16-byte aligned) and KIscale [B, cap] fp32 replace KIcache.
+ * A block closed by this step is compressed, rounded to bf16 and quantised
+ * into both.  Requires bf16 dims with cI = 128 and nhI in {32, 64}
+ * (CSA_ERR_UNSUPPORTED otherwise).  Workspace: csa_decode_workspace_bytes. */
+csa_status csa_decode_q8(const csa_dims* dims, const void* packed, const void* h, const int* pos, void* ring,
+                         void* Ccache, void* KIcodes, float* KIscale, int* cache_len, int cap, int B, void* O,
+                         int* idx_out, void* ws, size_t ws_bytes, void* stream);
+
+/* csa_decode_q8 with the stage events of csa_decode_staged. */
+csa_status csa_decode_q8_staged(const csa_dims* dims, const void* packed, const void* h, const int* pos,
+                                void* ring, void* Ccache, void* KIcodes, float* KIscale, int* cache_len,
+                                int cap, int B, void* O, int* idx_out, void* ws, size_t ws_bytes,
+                                void* const* events, void* stream);
+
+/* ---------------------------------------------------------------------- */
 /* Status                                                                  */
 /* ---------------------------------------------------------------------- */
 

@@ -34,6 +34,9 @@ import numpy as np
 __all__ = [
     "round_bf16",
     "round_f32",
+    "round_f16",
+    "round_e4m3",
+    "quantize_e4m3_rows",
     "storage_round",
     "project",
     "compress",
@@ -69,6 +72,46 @@ def round_bf16(x):
 def round_f32(x):
     """Round fp64 values to the nearest fp32 value (ties to even), returned as fp64."""
     return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+def round_f16(x):
+    """Round fp64 values to the nearest fp16 value (ties to even), returned as fp64."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+E4M3_MAX = 448.0
+
+
+def round_e4m3(x):
+    """Round fp64 values to the nearest FP8 E4M3 value (1 sign, 4 exponent bits
+    with bias 7, 3 mantissa bits; ties to even), saturating to +-448, as fp64.
+
+    Normal values (|x| >= 2^-6) have 8 steps per binade, i.e. a spacing of
+    2^(e-3) for |x| in [2^e, 2^(e+1)); below 2^-6 the subnormal spacing is
+    2^-9.  ``np.round`` rounds half to even on the scaled magnitude.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, E = np.frexp(a)                       # a = f 2^E, 0.5 <= f < 1, so the binade is 2^(E-1)
+    e = np.maximum(E - 1, -6)                # subnormals share the spacing of the lowest binade
+    step = np.ldexp(1.0, e - 3)
+    r = np.round(a / step) * step
+    return np.sign(x) * np.minimum(r, E4M3_MAX)
+
+
+def quantize_e4m3_rows(V):
+    """FP8 E4M3 codes and one fp32 scale per row, the quantised cache format.
+
+    V: [N, w] values (the entries as stored in bf16).  Per row:
+    scale = max_j |v_j| / 448 in fp32 (1 for an all-zero row), and
+    code_j = round_e4m3(v_j / scale) with the division in fp32.  The row is
+    represented as code_j * scale.  Returns (codes [N, w], scales [N]) as fp64.
+    """
+    V = np.asarray(V, dtype=np.float64)
+    amax = np.abs(V).max(axis=-1).astype(np.float32)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    x = V.astype(np.float32) / scale[..., None]
+    return round_e4m3(x.astype(np.float64)), scale.astype(np.float64)
 
 
 def storage_round(x, store):
@@ -396,7 +439,8 @@ def csa_forward_sampled(H, W, dims, seqlens, rows, store="bf16", chunk=8192):
 # One decode step over a compressed cache
 # --------------------------------------------------------------------------
 
-def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="exact", detail=None):
+def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="exact", detail=None,
+                    kcache="plain"):
     """One new token per sequence attending over a compressed cache.
 
     The same equations as ``csa_forward`` for a single query token t = pos[b]
@@ -414,6 +458,11 @@ def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="e
     C_cache [B, cap, c], K_cache [B, cap, c^I], cache_len [B] and ring
     [B, 2m, 4c + 4c^I] are updated IN PLACE (copies are the caller's choice).
     cache_len[b] must equal floor(t/m) on entry.
+    kcache="e4m3" is the quantised indexer-key cache (a format of this
+    implementation, not of the page): K_cache then holds every entry as
+    code * scale (quantize_e4m3_rows of its bf16 value), an appended entry is
+    quantised the same way, and the indexer queries enter eq. (8) rounded to
+    fp16, the precision the quantised kernels multiply them in.
     Returns (O [B, n_h, c], idx [B, topk]).  If ``detail`` is a dict it
     receives per sequence the scores I_t, the attention queries q_t and the
     indexer inputs q^I_t and w^I_t.
@@ -459,11 +508,16 @@ def csa_decode_step(h, pos, C_cache, K_cache, cache_len, ring, W, dims, store="e
                     Zb = np.concatenate([part(b_tok, j0 + 3), part(a_tok, j0 + 3)])
                     ent = compress(Ca, Cb, Za, Zb, W[bias_a], W[bias_b], m)[1]
                     cache[b, i] = rnd(ent)
+            if kcache == "e4m3":
+                codes, scale = quantize_e4m3_rows(K_cache[b, i][None, :])
+                K_cache[b, i] = codes[0] * scale[0]
             cache_len[b] = i + 1
         avail = t // m
         cQ = rnd(project(h[b:b + 1], W["W_DQ"]))
         wI = rnd_w(project(h[b:b + 1], W["W_w"]))[0]
         qI = rnd(project(cQ, W["W_IUQ"]))[0].reshape(nhI, cI)
+        if kcache == "e4m3":
+            qI = round_f16(qI)
         q = rnd(project(cQ, W["W_UQ"]))[0].reshape(nh, c)
         I_t = indexer_scores(qI, wI, K_cache[b, :avail])
         sel = topk_select(I_t, k)

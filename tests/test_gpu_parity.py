@@ -353,9 +353,17 @@ def test_stage_sparse_mqa_flags_bad_index_without_fault():
 
 # ---------------------------------------------------------------- decode
 
-def decode_case(dims, B, pos0, cap, steps, seed, check):
+def e4m3_codes_f64(codes_u8):
+    """Byte codes (uint8 tensor) as the E4M3 values they encode, fp64 numpy."""
+    return codes_u8.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def decode_case(dims, B, pos0, cap, steps, seed, check, q8=False):
     """`steps` decode steps of B sequences starting at token pos0 (GPU) vs
-    the oracle's decode step on the sequences listed in `check`."""
+    the oracle's decode step on the sequences listed in `check`.  q8: the
+    indexer-key cache is E4M3 codes + per-entry scales (csa_decode_q8),
+    quantised on the GPU from the seeded bf16 cache and, independently, by
+    the oracle from the same values."""
     m, c, cI = dims.m, dims.c, dims.cI
     W = synth.make_weights(dims, seed)
     packed = gpu_pack(dims, W)
@@ -367,6 +375,16 @@ def decode_case(dims, B, pos0, cap, steps, seed, check):
     clen = torch.full((B,), pos0 // m, dtype=torch.int32)
     d_Cc, d_Kc, d_ring, d_clen = Cc.to(DEV), Kc.to(DEV), ring.to(DEV), clen.to(DEV)
     o_Cc, o_Kc, o_ring = f64(Cc[check]), f64(Kc[check]), f64(ring[check])
+    kmode = "plain"
+    if q8:
+        kmode = "e4m3"
+        d_codes = torch.empty(B, cap, cI, dtype=torch.uint8, device=DEV)
+        d_scale = torch.empty(B, cap, dtype=torch.float32, device=DEV)
+        csa.csa_quantize_keys_e4m3(d_Kc, cI, B * cap, cI, d_codes, d_scale)
+        oc, osc = orc.quantize_e4m3_rows(o_Kc.reshape(-1, cI))
+        assert np.array_equal(e4m3_codes_f64(d_codes[check]).reshape(-1, cI), oc), "E4M3 codes differ"
+        assert np.array_equal(d_scale[check].cpu().double().numpy().reshape(-1), osc), "scales differ"
+        o_Kc = (oc * osc[:, None]).reshape(o_Kc.shape)
     o_clen = clen[check].numpy().astype(np.int64)
     W64 = weights_f64(W)
     ws = torch.empty(csa.csa_decode_workspace_bytes(dims, B, cap), dtype=torch.uint8, device=DEV)
@@ -375,14 +393,18 @@ def decode_case(dims, B, pos0, cap, steps, seed, check):
         h = synth.make_normal((B, dims.d), dims, seed + 100 + step)
         O = torch.empty(B, dims.nh * c, dtype=h.dtype, device=DEV)
         idx = torch.empty(B, dims.topk, dtype=torch.int32, device=DEV)
-        csa.csa_decode(dims, packed, h.to(DEV), pos.to(DEV), d_ring, d_Cc, d_Kc, d_clen, cap, B, O, idx, ws)
+        if q8:
+            csa.csa_decode_q8(dims, packed, h.to(DEV), pos.to(DEV), d_ring, d_Cc, d_codes, d_scale, d_clen, cap, B, O,
+                              idx, ws)
+        else:
+            csa.csa_decode(dims, packed, h.to(DEV), pos.to(DEV), d_ring, d_Cc, d_Kc, d_clen, cap, B, O, idx, ws)
         assert csa.csa_get_device_status() == 0
         detail, dx = {}, {}
         if dims.dtype == csa.CSA_BF16:   # same step with exact storage, for the rounding sensitivity
             orc.csa_decode_step(f64(h[check]), pos[check].numpy(), o_Cc.copy(), o_Kc.copy(), o_clen.copy(),
-                                o_ring.copy(), W64, odims(dims), store="exact", detail=dx)
+                                o_ring.copy(), W64, odims(dims), store="exact", detail=dx, kcache=kmode)
         oO, oidx = orc.csa_decode_step(f64(h[check]), pos[check].numpy(), o_Cc, o_Kc, o_clen, o_ring, W64,
-                                       odims(dims), store=store_mode(dims), detail=detail)
+                                       odims(dims), store=store_mode(dims), detail=detail, kcache=kmode)
         gidx = idx.cpu().numpy()[check]
         want = np.zeros_like(oO)
         for r in range(len(check)):
@@ -397,7 +419,11 @@ def decode_case(dims, B, pos0, cap, steps, seed, check):
     assert np.array_equal(d_clen.cpu().numpy()[check], o_clen)
     nb = int(o_clen.max())
     compare_dense(f64(d_Cc.cpu()[check][:, :nb]), o_Cc[:, :nb], dims.dtype, "C cache")
-    compare_dense(f64(d_Kc.cpu()[check][:, :nb]), o_Kc[:, :nb], dims.dtype, "K cache")
+    if q8:   # the entries the GPU appended, dequantised, against the oracle's quantised ones
+        gk = e4m3_codes_f64(d_codes[check][:, :nb]) * d_scale[check][:, :nb].cpu().double().numpy()[..., None]
+        compare_dense(gk, o_Kc[:, :nb], dims.dtype, "K cache (E4M3)")
+    else:
+        compare_dense(f64(d_Kc.cpu()[check][:, :nb]), o_Kc[:, :nb], dims.dtype, "K cache")
     assert sum(counts.values()) == steps * len(check)
     return report(f"decode B={B} t0={pos0} k={dims.topk}", counts)
 

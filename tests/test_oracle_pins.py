@@ -441,3 +441,42 @@ def test_forward_sampled_equals_forward(store):
     np.testing.assert_allclose(samp["O"], full["O"], atol=1e-12)
     for a, b in zip(samp["scores"], full["scores"]):
         np.testing.assert_allclose(a, b, atol=1e-12)
+
+
+# ---------------------------------------------------------------- FP8 E4M3 (quantised key cache)
+
+def test_round_e4m3_matches_torch_float8_below_saturation():
+    """round_e4m3 against torch's own float -> float8_e4m3fn conversion
+    (round to nearest even) over magnitudes from subnormal to 448."""
+    rng = np.random.default_rng(7)
+    x = np.concatenate([rng.standard_normal(4000) * s for s in (1e-3, 0.02, 1.0, 30.0, 200.0)])
+    x = x[np.abs(x) <= 448]
+    want = torch.as_tensor(x, dtype=torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(orc.round_e4m3(x.astype(np.float32).astype(np.float64)), want)
+
+
+def test_round_e4m3_hand_values():
+    # ties to even: 1.0625 lies halfway between 1.0 and 1.125, 1.1875 between 1.125 and 1.25
+    assert orc.round_e4m3(1.0625) == 1.0 and orc.round_e4m3(1.1875) == 1.25
+    # smallest normal 2^-6 and smallest subnormal 2^-9 are exact; half of 2^-9 rounds to 0 (even)
+    assert orc.round_e4m3(2.0 ** -6) == 2.0 ** -6 and orc.round_e4m3(2.0 ** -9) == 2.0 ** -9
+    assert orc.round_e4m3(2.0 ** -10) == 0.0 and orc.round_e4m3(3 * 2.0 ** -10) == 2.0 ** -8
+    # saturation: 464 would round to 480, beyond the largest finite 448
+    assert orc.round_e4m3(464.0) == 448.0 and orc.round_e4m3(-1000.0) == -448.0
+    assert orc.round_e4m3(-3.4) == -3.5 and orc.round_e4m3(0.0) == 0.0
+
+
+def test_quantize_e4m3_rows_scale_and_error():
+    rng = np.random.default_rng(8)
+    V = orc.round_bf16(rng.standard_normal((50, 128)) * rng.uniform(0.01, 10, (50, 1)))
+    V[3] = 0.0
+    codes, scale = orc.quantize_e4m3_rows(V)
+    # each row's largest magnitude maps to the largest code
+    rows = [r for r in range(50) if r != 3]
+    assert np.all(np.abs(codes[rows]).max(axis=1) == 448.0)
+    assert scale[3] == 1.0 and np.all(codes[3] == 0)
+    # every code is an E4M3 value, and the reconstruction is within half a step
+    assert np.array_equal(orc.round_e4m3(codes), codes)
+    err = np.abs(codes * scale[:, None] - V)
+    step = np.where(np.abs(codes) >= 2.0 ** -6, np.ldexp(1.0, np.frexp(np.abs(codes) + 1e-300)[1] - 4), 2.0 ** -9)
+    assert np.all(err <= 0.5 * step * scale[:, None] * (1 + 1e-6) + 1e-12)
