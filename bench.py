@@ -787,6 +787,24 @@ def run_indexer_only(args):
         raise SystemExit(1)
 
 
+def run_decode_only(args):
+    """warmup + steps decode steps of the decode workload (bf16 key cache, then
+    the E4M3 key cache); for profiling the decode kernels."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dr = DecodeRunner(synth.workloads()["decode"], dev)
+    for _ in range(args.warmup + args.steps):
+        dr.step()
+    dr.quantise_keys()
+    for _ in range(args.warmup + args.steps):
+        dr.step_q8()
+    torch.cuda.synchronize()
+    st = csa.csa_get_device_status()
+    print(json.dumps({"decode_steps": 2 * (args.warmup + args.steps), "status": csa.status_string(st)}), flush=True)
+    if st != 0:
+        raise SystemExit(1)
+
+
 def runner_T(w):
     return sum(w.seqlens)
 
@@ -808,6 +826,7 @@ def main():
     ap.add_argument("--stage", choices=["A1_project_hidden", "A2_project_query", "A3_compress", "A4_indexer_topk",
                                         "A5_sparse_mqa", "A1A3_project_compress"],
                     help="run only this stage (profiling)")
+    ap.add_argument("--decode-only", action="store_true", help="run decode steps only (profiling)")
     ap.add_argument("--indexer-only", action="store_true",
                     help="run csa_indexer_topk alone on seeded inputs of the workload's sizes (profiling)")
     args = ap.parse_args()
@@ -821,6 +840,9 @@ def main():
         return
     if args.indexer_only:
         run_indexer_only(args)
+        return
+    if args.decode_only:
+        run_decode_only(args)
         return
     if args.stage:
         run_stage(args)
