@@ -593,9 +593,9 @@ def run_decode(dev, args, peaks, flush, stream):
     q_total = dr.bytes_per_step() - dr.B * avail * d.cI * 2 + dr.B * avail * (d.cI + 4)
     q_stages = {}
     for n, ms in zip(names, q_in_step):
-        gbs = qbytes[n] / (ms / 1000.0) / 1e9
-        q_stages[n] = {"ms": ms, "bound": "hbm", "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
-                       "frac": gbs / peaks["hbm"], "algorithmic_bytes": qbytes[n]}
+        sgbs = qbytes[n] / (ms / 1000.0) / 1e9
+        q_stages[n] = {"ms": ms, "bound": "hbm", "achieved": sgbs, "peak": peaks["hbm"], "unit": "GB/s",
+                       "frac": sgbs / peaks["hbm"], "algorithmic_bytes": qbytes[n]}
     qgbs = q_total / (qms / 1000.0) / 1e9
     e4m3 = {"value": dr.B / (qms / 1000.0), "unit": "tokens/s", "ms_per_step": qms,
             "cache": "K^IComp as E4M3 codes + one fp32 scale per entry; C^Comp bf16",
