@@ -14,5 +14,5 @@ from .capi import (CSA_BF16, CSA_F32, CsaError, Dims, csa_cache_append, csa_comp
                    csa_check_wait_timeout, csa_forward_staged, csa_decode_staged,
                    csa_project_compress_workspace_bytes, csa_project_hidden_compress,
                    csa_cp_workspace_bytes, csa_cp_compress, csa_cp_queries, csa_quantize_keys_e4m3,
-                   csa_decode_q8, csa_decode_q8_staged)
+                   csa_decode_q8, csa_decode_q8_staged, csa_debug_build)
 from .meta import cu_from_lengths  # noqa: F401

@@ -1,4 +1,7 @@
-"""Builds libcsa.so in-tree with nvcc for sm_100a (no GPU needed to build).
+"""Builds libcsa.so in-tree with nvcc for sm_100a (no GPU needed to build),
+and its debug twin libcsa_debug.so (compiled with CSA_DEBUG: the kernels
+check the indices they compute before each global access and record a status
+bit instead of accessing out of range; same entry points, same results).
 
 CSA_NVTX=1 in the environment compiles in NVTX ranges named after the stages
 (host side, around each stage's launches) for profiler timelines; it takes
@@ -13,6 +16,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(os.path.dirname(PKG), "include")
 LIB = os.path.join(PKG, "libcsa.so")
+LIB_DEBUG = os.path.join(PKG, "libcsa_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -32,24 +36,29 @@ def _sources():
     return out
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    """Compile csrc/csa_lib.cu (which includes every kernel) into libcsa.so."""
-    if not force and not needs_build():
-        return LIB
-    tmp = LIB + ".tmp"
+def _compile(lib: str, defines, verbose: bool, extra) -> None:
+    tmp = lib + ".tmp"
     nvtx = ["-DCSA_NVTX"] if os.environ.get("CSA_NVTX") == "1" else []
-    cmd = [NVCC, *FLAGS, *nvtx, *extra, "-o", tmp, os.path.join(CSRC, "csa_lib.cu")]
+    cmd = [NVCC, *FLAGS, *nvtx, *defines, *extra, "-o", tmp, os.path.join(CSRC, "csa_lib.cu")]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Compile csrc/csa_lib.cu (which includes every kernel) into libcsa.so
+    and libcsa_debug.so; returns the release library's path."""
+    for lib, defines in ((LIB, []), (LIB_DEBUG, ["-DCSA_DEBUG"])):
+        if force or needs_build(lib):
+            _compile(lib, defines, verbose, extra)
     return LIB
 
 

@@ -4,7 +4,9 @@ Every function here has the name of the C entry point it calls, takes torch
 tensors (their ``data_ptr()`` is passed), plain ints or None (NULL), and
 raises ``CsaError`` when the call returns a status other than CSA_OK.  No
 step of the computation happens in Python.  Loading fails loudly if the
-library has not been built; there is no fallback.
+library has not been built; there is no fallback.  CSA_DEBUG=1 in the
+environment loads the debug build, libcsa_debug.so, instead (device-side
+index checks; see csa_debug_build in include/csa.h).
 """
 from __future__ import annotations
 
@@ -13,12 +15,12 @@ import os
 from dataclasses import dataclass
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libcsa.so")
+LIB_PATH = os.path.join(PKG, "libcsa_debug.so" if os.environ.get("CSA_DEBUG") == "1" else "libcsa.so")
 
 CSA_F32, CSA_BF16 = 0, 1
 STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "CSA_ERR_CUDA",
           4: "CSA_ERR_DEVICE_TIMEOUT", 5: "CSA_ERR_BAD_INDEX", 6: "CSA_ERR_BAD_METADATA",
-          7: "CSA_ERR_WORKSPACE"}
+          7: "CSA_ERR_WORKSPACE", 8: "CSA_ERR_DEVICE_BOUNDS"}
 
 # every symbol include/csa.h declares
 EXPORTS = (
@@ -30,6 +32,7 @@ EXPORTS = (
     "csa_set_wait_limit_ns", "csa_check_wait_timeout", "csa_forward_staged", "csa_decode_staged",
     "csa_project_compress_workspace_bytes", "csa_project_hidden_compress", "csa_cp_workspace_bytes",
     "csa_cp_compress", "csa_cp_queries", "csa_quantize_keys_e4m3", "csa_decode_q8", "csa_decode_q8_staged",
+    "csa_debug_build",
 )
 
 
@@ -75,7 +78,7 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"libcsa.so not built at {LIB_PATH}; run __graft_entry__.build()")
+            raise ImportError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; run __graft_entry__.build()")
         L = ctypes.CDLL(LIB_PATH)
         vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         D = ctypes.POINTER(csa_dims)
@@ -113,6 +116,7 @@ def lib() -> ctypes.CDLL:
             "csa_forward_staged": (i, [D, vp, vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp, vp]),
             "csa_decode_staged": (i, [D, vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, sz, vp, vp]),
             "csa_check_wait_timeout": (i, [vp, vp]),
+            "csa_debug_build": (i, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -253,6 +257,10 @@ def csa_project_hidden(dims: Dims, packed, H, T, Y1, wI, stream=None):
 def csa_project_query(dims: Dims, packed, cQ, ld_cQ, T, Y2, stream=None):
     _check(lib().csa_project_query(_d(dims), _p(packed), _p(cQ), ld_cQ, T, _p(Y2), _stream(stream)),
            "csa_project_query")
+
+
+def csa_debug_build() -> int:
+    return lib().csa_debug_build()
 
 
 def csa_launch_count() -> int:

@@ -15,11 +15,34 @@ enum : unsigned {
   kStatusTimeout = 1u,   // a bounded wait gave up
   kStatusBadIndex = 2u,  // an out-of-range block index was skipped
   kStatusMetadata = 4u,  // cu_seqlens / cu_blocks / cache_len inconsistent
+  kStatusBounds = 8u,    // a debug-build index check failed (the access was skipped)
 };
 
 __device__ unsigned g_status;
 
 __device__ __forceinline__ void flag_status(unsigned bits) { atomicOr(&g_status, bits); }
+
+// Index checks of the debug build (compiled with CSA_DEBUG): dcheck(ok)
+// records kStatusBounds when `ok` is false and returns `ok`, so that the
+// caller skips the access it guards; the release build compiles every check
+// to `true`.  They restate, next to a global access, the invariant that the
+// kernel's own logic guarantees (an entry row inside the entry array, a
+// selected index inside the visible range, k indices written per row), so
+// that a logic error shows up as a status bit instead of a stray access.
+// dguard(ok) is for a guard the release build keeps as a silent skip
+// (returns `ok` in both builds; the debug build also records the bit).
+#ifdef CSA_DEBUG
+constexpr bool kDebugBuild = true;
+__device__ __forceinline__ bool dcheck(bool ok) {
+  if (!ok) flag_status(kStatusBounds);
+  return ok;
+}
+__device__ __forceinline__ bool dguard(bool ok) { return dcheck(ok); }
+#else
+constexpr bool kDebugBuild = false;
+__device__ __forceinline__ constexpr bool dcheck(bool) { return true; }
+__device__ __forceinline__ constexpr bool dguard(bool ok) { return ok; }
+#endif
 
 // Limit of every bounded device wait, in ns of %globaltimer (set per device
 // by csa_set_wait_limit_ns; read by a wait when its first poll fails).
@@ -87,6 +110,12 @@ struct RowMap {
   int pos0;               // prefill: position of the first row of a sequence (0, or the
                           // start of a context-parallel chunk of a single sequence)
 };
+
+// Number of entries behind a RowMap: the packed entry array of a prefill
+// (total_blocks) or the rows x cap caches of a decode step.
+__device__ __forceinline__ long long rowmap_entries(const RowMap& rm, int rows) {
+  return rm.cap > 0 ? (long long)rows * rm.cap : (long long)rm.total_blocks;
+}
 
 // Visible entries of `row`: global entry index of block 0 and the count
 // floor(t/m).  Inconsistent metadata is flagged and clamped so that no access

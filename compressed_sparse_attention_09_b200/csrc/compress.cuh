@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
       res[e] = compress_channel<M>(la, lb, c_a, c_b, has_prev);
     }
   }
+  if (!dcheck(g < a.total_blocks && (!has_prev || tok - M >= a.cu_seqlens[lo]))) return;
   store_raw<T, V>(static_cast<T*>(sg.out) + (long long)g * sg.width + col, res);
 }
 

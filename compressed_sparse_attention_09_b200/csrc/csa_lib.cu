@@ -617,6 +617,7 @@ const char* csa_status_string(csa_status s) {
     case CSA_ERR_BAD_INDEX: return "out-of-range block index seen on the device";
     case CSA_ERR_BAD_METADATA: return "inconsistent cu_seqlens / cu_blocks / cache metadata";
     case CSA_ERR_WORKSPACE: return "workspace too small";
+    case CSA_ERR_DEVICE_BOUNDS: return "a debug-build index check failed on the device";
   }
   return "unknown status";
 }
@@ -629,8 +630,11 @@ csa_status csa_get_device_status(void* stream) {
   if (v & kStatusTimeout) return CSA_ERR_DEVICE_TIMEOUT;
   if (v & kStatusBadIndex) return CSA_ERR_BAD_INDEX;
   if (v & kStatusMetadata) return CSA_ERR_BAD_METADATA;
+  if (v & kStatusBounds) return CSA_ERR_DEVICE_BOUNDS;
   return CSA_OK;
 }
+
+int csa_debug_build(void) { return kDebugBuild ? 1 : 0; }
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -1212,7 +1216,7 @@ csa_status launch_indexer_decode_tc(const csa_dims* d, const IndexerArgs& a, int
   if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsel::kSmem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
-  decode_select_kernel<<<B, 512, dsel::kSmem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
+  decode_select_kernel<<<B, dsel::kThreads, dsel::kSmem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }
@@ -1245,7 +1249,7 @@ csa_status launch_indexer_decode_q8(const csa_dims* d, const IndexerArgs& a, con
   if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsel::kSmem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
-  decode_select_kernel<<<B, 512, dsel::kSmem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
+  decode_select_kernel<<<B, dsel::kThreads, dsel::kSmem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }

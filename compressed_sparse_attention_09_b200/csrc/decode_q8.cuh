@@ -58,17 +58,26 @@ struct IdxDecQ8Args {
 };
 
 namespace idxq8 {
-constexpr int kM = 128, kCI = 128, kStages = 4, kKBufs = 2;
+constexpr int kM = 128, kCI = 128, kStages = 8, kKBufs = 2, kQSlots = 2;
 constexpr int kQBytes = 64 * 128 * 2;          // q^I fp16, up to 64 heads x 128, two 64-column chunks
 constexpr int kCodeBytes = kM * kCI;           // 128 entries x 128 codes (128-byte swizzled rows)
-constexpr int kStageBytes = kQBytes + kCodeBytes;
 constexpr int kKChunk = kM * 128;              // fp16 [128 entries x 64 channels]
 constexpr int kKBytes = 2 * kKChunk;
-constexpr int kOffK = kStages * kStageBytes;
+constexpr int kOffC = kQSlots * kQBytes;       // code stages
+constexpr int kOffK = kOffC + kStages * kCodeBytes;
 constexpr int kOffW = kOffK + kKBufs * kKBytes;
 constexpr size_t kSmem = 1024 + (size_t)kOffW + 4 * 64 * 4 + 256;
-constexpr int kThreads = 320;
+constexpr int kCvtWarps = 4;                   // warps 6-9 widen the codes
+constexpr int kThreads = 32 * (6 + kCvtWarps);
 }  // namespace idxq8
+
+// Two E4M3 codes (the low and high byte of v) to an fp16 pair, low code in
+// the low half (the hardware conversion).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
+}
 
 // Instruction descriptor of kind::f16 with fp16 A/B, fp32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
@@ -77,7 +86,7 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
 
 // Score rows of the decode queries over their FP8 key caches, one work item
 // per (sequence, 128-entry tile), items of a CTA contiguous.  Warp 0: TMA
-// (q^I fp16 and the tile's codes per stage); warps 6-9: widen the codes to
+// (q^I fp16 once per sequence, the tile's codes per stage); warps 6-9: widen the codes to
 // fp16 in the MMA's swizzled K-major layout (two buffers); warp 1: MMA
 // issuer and TMEM owner (D[128 entries x n_h^I], two accumulators); warps
 // 2-5: epilogue (ReLU, head weights, entry scale).  All waits are bounded.
@@ -91,13 +100,15 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
   uint8_t* kbuf = sm + kOffK;
   float* w_s = reinterpret_cast<float*>(sm + kOffW);            // 4 epilogue warps x 64
   uint64_t* bars = reinterpret_cast<uint64_t*>(w_s + 4 * 64);
-  uint64_t* full = bars;                   // [kStages] q + codes landed
-  uint64_t* empty = full + kStages;        // [kStages] MMA done with the stage
-  uint64_t* kfull = empty + kStages;       // [kKBufs] fp16 tile written (4 converter warps)
+  uint64_t* full = bars;                   // [kStages] codes landed
+  uint64_t* empty = full + kStages;        // [kStages] codes widened (kCvtWarps arrivals)
+  uint64_t* kfull = empty + kStages;       // [kKBufs] fp16 tile written (kCvtWarps arrivals)
   uint64_t* kfree = kfull + kKBufs;        // [kKBufs] MMA done with the fp16 tile
   uint64_t* t_full = kfree + kKBufs;       // [2]
   uint64_t* t_empty = t_full + 2;          // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_empty + 2);
+  uint64_t* q_full = t_empty + 2;          // [kQSlots] q^I of a sequence landed
+  uint64_t* q_empty = q_full + kQSlots;    // [kQSlots] the sequence's last MMA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + kQSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = a.nhI;
@@ -105,9 +116,10 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
   const int qchunk = N * 128;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int s = 0; s < kKBufs; ++s) { mbar_init(&kfull[s], 4); mbar_init(&kfree[s], 1); }
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kCvtWarps); }
+    for (int s = 0; s < kKBufs; ++s) { mbar_init(&kfull[s], kCvtWarps); mbar_init(&kfree[s], 1); }
     for (int s = 0; s < 2; ++s) { mbar_init(&t_full[s], 1); mbar_init(&t_empty[s], 4); }
+    for (int s = 0; s < kQSlots; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
@@ -130,43 +142,59 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
     return j * kM < avail;
   };
 
+  // q^I (fp16) is loaded once per sequence (a CTA's items are contiguous)
+  // into one of kQSlots slots; the ring stages carry only codes, and the
+  // widening warps free a stage as soon as they have read it.
   if (warp == 0) {
     if (lane == 0) {
-      uint32_t g = 0;
+      uint32_t g = 0, nq = 0;
+      int qb = -1;
       for (int it = it0; it < it1 && !*abort_flag; ++it) {
         int b, j, avail;
         if (!item_ok(it, b, j, avail)) continue;
+        if (b != qb) {
+          const int qs = nq % kQSlots;
+          if (!mbar_wait(&q_empty[qs], ((nq / kQSlots) & 1) ^ 1)) { *abort_flag = 1; break; }
+          mbar_arrive_expect_tx(&q_full[qs], (uint32_t)(2 * qchunk));
+          for (int c = 0; c < 2; ++c) tma_load_3d(&tmQ, &q_full[qs], sm + qs * kQBytes + c * qchunk, 64 * c, 0, b);
+          qb = b;
+          ++nq;
+        }
         const int st = g % kStages;
         if (!mbar_wait(&empty[st], ((g / kStages) & 1) ^ 1)) { *abort_flag = 1; break; }
-        uint8_t* stage = sm + st * kStageBytes;
-        mbar_arrive_expect_tx(&full[st], (uint32_t)(2 * qchunk + kCodeBytes));
-        for (int c = 0; c < 2; ++c) tma_load_3d(&tmQ, &full[st], stage + c * qchunk, 64 * c, 0, b);
-        tma_load_2d(&tmK, &full[st], stage + kQBytes, 0, b * a.cap + j * kM);
+        mbar_arrive_expect_tx(&full[st], (uint32_t)kCodeBytes);
+        tma_load_2d(&tmK, &full[st], sm + kOffC + st * kCodeBytes, 0, b * a.cap + j * kM);
         ++g;
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kM, N);
-      uint32_t g = 0;
+      uint32_t g = 0, nq = 0;
+      int qb = -1;
       for (int it = it0; it < it1 && !*abort_flag; ++it) {
         int b, j, avail;
         if (!item_ok(it, b, j, avail)) continue;
-        const int st = g % kStages, kb = g % kKBufs, acc = g & 1;
-        if (!mbar_wait(&full[st], (g / kStages) & 1) || !mbar_wait(&kfull[kb], (g / kKBufs) & 1) ||
-            !mbar_wait(&t_empty[acc], ((g >> 1) & 1) ^ 1)) {
+        if (b != qb) {
+          // the previous sequence's slot is free once its MMAs complete
+          if (nq > 0) mma_commit(&q_empty[(nq - 1) % kQSlots]);
+          if (!mbar_wait(&q_full[nq % kQSlots], (nq / kQSlots) & 1)) { *abort_flag = 1; break; }
+          qb = b;
+          ++nq;
+        }
+        const int kb = g % kKBufs, acc = g & 1;
+        if (!mbar_wait(&kfull[kb], (g / kKBufs) & 1) || !mbar_wait(&t_empty[acc], ((g >> 1) & 1) ^ 1)) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
-        const uint64_t qd = sdesc_k_sw128(smem_u32(sm + st * kStageBytes));
+        const uint64_t qd = sdesc_k_sw128(smem_u32(sm + ((nq - 1) % kQSlots) * kQBytes));
         const uint64_t kd = sdesc_k_sw128(smem_u32(kbuf + kb * kKBytes));
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
             mma_bf16(tmem + (uint32_t)(acc * 64), desc_add(kd, c * kKChunk + ks * 32),
                      desc_add(qd, c * qchunk + ks * 32), idesc, (c | ks) != 0);
-        mma_commit(&empty[st]);
         mma_commit(&kfree[kb]);
         mma_commit(&t_full[acc]);
         ++g;
@@ -174,8 +202,10 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
     }
   } else if (warp >= 6) {
     // ---------------------------------------------------------------- code widening (warps 6-9)
-    // thread -> 16-byte unit u = t % 8 (16 codes) of rows t / 8 + 16 i
+    // thread -> 16-byte unit u = t % 8 (16 codes) of rows t / 8 + 16 i; all
+    // of a thread's row loads are issued before any conversion
     const int t = threadIdx.x - 192, u = t & 7, r0 = t >> 3;
+    constexpr int kRows = kM / (4 * kCvtWarps);   // rows per thread
     uint32_t g = 0;
     for (int it = it0; it < it1; ++it) {
       if (warp_aborted(abort_flag)) break;
@@ -186,29 +216,38 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
         if (lane == 0) *abort_flag = 1;
         break;
       }
-      const uint8_t* codes = sm + st * kStageBytes + kQBytes;
+      const uint8_t* codes = sm + kOffC + st * kCodeBytes;
       uint8_t* dst = kbuf + kb * kKBytes + (u >> 2) * kKChunk;   // channels 16 u .. are in chunk u / 4
-#pragma unroll 2
-      for (int i = 0; i < kM / 16; ++i) {
-        const int r = r0 + 16 * i;
-        const uint4 cw = *reinterpret_cast<const uint4*>(codes + r * 128 + ((u ^ (r & 7)) << 4));
-        const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+      uint4 cw[kRows];
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) {
+        const int r = r0 + (4 * kCvtWarps) * i;
+        cw[i] = *reinterpret_cast<const uint4*>(codes + r * 128 + ((u ^ (r & 7)) << 4));
+      }
+      // 16 fp16 channels = units uu and uu + 1 of the chunk's row; the upper
+      // four threads of each 8 store them in the other order, so that each
+      // store of 8 threads covers all 8 bank groups (the chunks are 16 KB apart)
+      const int uu = 2 * (u & 3), s0 = uu + (u >> 2), s1 = uu + 1 - (u >> 2);
+#pragma unroll
+      for (int i = 0; i < kRows; ++i) {
+        const int r = r0 + (4 * kCvtWarps) * i;
+        const uint32_t w4[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
         uint32_t h[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w4[q] & 0xFFFFu), __NV_E4M3);
-          const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w4[q] >> 16), __NV_E4M3);
-          h[2 * q] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
-          h[2 * q + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
+          h[2 * q] = e4m3x2_to_f16x2((uint16_t)(w4[q] & 0xFFFFu));
+          h[2 * q + 1] = e4m3x2_to_f16x2((uint16_t)(w4[q] >> 16));
         }
-        // 16 fp16 channels = units 2 (u % 4) and 2 (u % 4) + 1 of the chunk's row r
-        const int uu = 2 * (u & 3);
-        *reinterpret_cast<uint4*>(dst + r * 128 + ((uu ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4*>(dst + r * 128 + (((uu + 1) ^ (r & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+        const uint4 lo = make_uint4(h[0], h[1], h[2], h[3]), hi = make_uint4(h[4], h[5], h[6], h[7]);
+        *reinterpret_cast<uint4*>(dst + r * 128 + ((s0 ^ (r & 7)) << 4)) = (u >> 2) ? hi : lo;
+        *reinterpret_cast<uint4*>(dst + r * 128 + ((s1 ^ (r & 7)) << 4)) = (u >> 2) ? lo : hi;
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&kfull[kb]);
+      if (lane == 0) {
+        mbar_arrive(&kfull[kb]);
+        mbar_arrive(&empty[st]);   // every code of the stage has been read and used
+      }
       ++g;
     }
   } else {
@@ -227,21 +266,25 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
         __syncwarp();
         wb = b;
       }
+      // the entry's scale is fetched before the wait, so that its memory
+      // latency overlaps the MMA instead of following the epilogue
+      const int s = j * kM + 32 * sub + lane;
+      const float kscale = s < avail ? __ldg(a.kscale + (long long)b * a.cap + s) : 0.f;
       const int acc = g & 1;
       if (!warp_wait(&t_full[acc], (g >> 1) & 1)) { *abort_flag = 1; break; }
       tc_fence_after();
-      float sc = 0.f;
+      float sc4[4] = {0.f, 0.f, 0.f, 0.f};   // four partial sums (heads e mod 4)
       for (int hc = 0; hc < N; hc += 32) {
         float v[32];
         tmem_ld_32x32b_x32(tmem + lane_base + (uint32_t)(acc * 64 + hc), v);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sc = fmaf(w_my[hc + e], fmaxf(v[e], 0.f), sc);
+        for (int e = 0; e < 32; ++e) sc4[e & 3] = fmaf(w_my[hc + e], fmaxf(v[e], 0.f), sc4[e & 3]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[acc]);
-      const int s = j * kM + 32 * sub + lane;
-      if (s < avail) __stcg(a.scratch + (long long)b * a.cap + s, sc * __ldg(a.kscale + (long long)b * a.cap + s));
+      if (s < avail && dcheck(s < a.cap))
+        __stcg(a.scratch + (long long)b * a.cap + s, ((sc4[0] + sc4[1]) + (sc4[2] + sc4[3])) * kscale);
       ++g;
     }
   }

@@ -281,19 +281,31 @@ __device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, 
   const int lane = threadIdx.x & 31;
   const bool resident = n <= idxtc::kSelChunk;
   if (resident) warp_stage_chunk(sc, n, buf);
+  // When every key of the digit's bin is needed (in_bin == kk after the
+  // pass), the selection is already decided: exactly the keys >= the bin's
+  // lowest key value (prefix, low bits 0), and the later passes are skipped.
+  // After the second pass a bin spans 2^-13 of a binade, so at prefill sizes
+  // it usually holds the k-th key alone.
   int kk = k, above, in_bin;
   uint32_t prefix = warp_radix_pass<11, true>(sc, n, resident, buf, hist, 21, 0u, 0u, kk, &above, &in_bin) << 21;
   kk -= above;
-  prefix |= warp_radix_pass<11, false>(sc, n, resident, buf, hist, 10, 0xFFE00000u, prefix, kk, &above, &in_bin)
-            << 10;
-  kk -= above;
-  prefix |= warp_radix_pass<10, false>(sc, n, resident, buf, hist, 0, 0xFFFFFC00u, prefix, kk, &above, &in_bin);
-  kk -= above;
+  bool settled = in_bin == kk;
+  if (!settled) {
+    prefix |= warp_radix_pass<11, false>(sc, n, resident, buf, hist, 10, 0xFFE00000u, prefix, kk, &above, &in_bin)
+              << 10;
+    kk -= above;
+    settled = in_bin == kk;
+  }
+  if (!settled) {
+    prefix |= warp_radix_pass<10, false>(sc, n, resident, buf, hist, 0, 0xFFFFFC00u, prefix, kk, &above, &in_bin);
+    kk -= above;
+  }
   const uint32_t thr = prefix;
   const int need_eq = kk;
-  // in_bin = the number of keys equal to thr: when all of them are taken
-  // (the usual case) the choice is simply key >= thr
-  const bool all_eq = need_eq == in_bin;
+  // after the third pass in_bin = the number of keys equal to thr: when all
+  // of them are taken (the usual case) the choice is simply key >= thr, as it
+  // is for a selection settled early
+  const bool all_eq = settled || need_eq == in_bin;
   int out_off = 0, eq_seen = 0;
   const unsigned lt = (1u << lane) - 1u;
   if (!resident) {
@@ -340,7 +352,7 @@ __device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, 
 #pragma unroll
         for (int j = 0; j < 4; ++j)
           if (take[j]) {
-            if (p < k) out[p] = 4 * i + j;
+            if (dguard(p < k)) out[p] = 4 * i + j;
             ++p;
           }
         out_off += __shfl_sync(kFull, incl, 31);
@@ -357,7 +369,7 @@ __device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, 
       const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
       const unsigned btk = __ballot_sync(kFull, take);
       const int p = out_off + __popc(btk & lt);
-      if (take && p < k) out[p] = s;
+      if (take && dguard(p < k)) out[p] = s;
     }
     return;
   }
@@ -379,7 +391,7 @@ __device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, 
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int p = out_off + __popc(btk[u] & lt);
-          if (((btk[u] >> lane) & 1u) && p < k) out[p] = c0 + base + 32 * u + lane;
+          if (((btk[u] >> lane) & 1u) && dguard(p < k)) out[p] = c0 + base + 32 * u + lane;
           out_off += __popc(btk[u]);
         }
       } else {
@@ -392,7 +404,7 @@ __device__ __noinline__ void warp_topk_ascending(const float* sc, int n, int k, 
           const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
           const unsigned btk = __ballot_sync(kFull, take);
           const int p = out_off + __popc(btk & lt);
-          if (take && p < k) out[p] = c0 + s;
+          if (take && dguard(p < k)) out[p] = c0 + s;
           out_off += __popc(btk);
           eq_seen += __popc(beq);
         }
@@ -580,7 +592,8 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
             }
           }
           const float sc = ((p[0].x + p[0].y) + (p[1].x + p[1].y)) + ((p[2].x + p[2].y) + (p[3].x + p[3].y));
-          if (s < avail) __stcg(reinterpret_cast<unsigned*>(scr) + (size_t)q * a.sc_cap + s, ordered_key(sc));
+          if (s < avail && dcheck(s < a.sc_cap))
+            __stcg(reinterpret_cast<unsigned*>(scr) + (size_t)q * a.sc_cap + s, ordered_key(sc));
         }
         tc_fence_before();
         __syncwarp();
@@ -646,11 +659,12 @@ struct IdxDecArgs {
 };
 
 namespace idxdec {
-constexpr int kM = 128, kStages = 4;
+constexpr int kM = 128, kStages = 6, kQSlots = 2;
 constexpr int kQBytes = 64 * 128 * 2;    // up to [64 heads x 128] bf16 as two 64-column chunks
 constexpr int kKBytes = kM * 128 * 2;    // [128 blocks x 128] bf16 as two chunks
-constexpr int kStageBytes = kQBytes + kKBytes;
-constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 4 * 64 * 4 + 256;
+constexpr int kOffK = kQSlots * kQBytes;
+constexpr int kOffW = kOffK + kStages * kKBytes;
+constexpr size_t kSmem = 1024 + (size_t)kOffW + 4 * 64 * 4 + 256;
 constexpr int kThreads = 192;
 }  // namespace idxdec
 
@@ -661,13 +675,15 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
   using namespace idxdec;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* w_s = reinterpret_cast<float*>(sm + kStages * kStageBytes);     // 4 warps x 64
+  float* w_s = reinterpret_cast<float*>(sm + kOffW);     // 4 warps x 64
   uint64_t* bars = reinterpret_cast<uint64_t*>(w_s + 4 * 64);
-  uint64_t* full = bars;                   // [kStages]
+  uint64_t* full = bars;                   // [kStages] key tile landed
   uint64_t* empty = full + kStages;        // [kStages]
   uint64_t* t_full = empty + kStages;      // [2]
   uint64_t* t_empty = t_full + 2;          // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(t_empty + 2);
+  uint64_t* q_full = t_empty + 2;          // [kQSlots] q^I of a sequence landed
+  uint64_t* q_empty = q_full + kQSlots;    // [kQSlots] the sequence's last MMA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + kQSlots);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = a.nhI;
@@ -678,6 +694,7 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int s = 0; s < 2; ++s) { mbar_init(&t_full[s], 1); mbar_init(&t_empty[s], 4); }
+    for (int s = 0; s < kQSlots; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
@@ -701,38 +718,55 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
     return j * kM < avail;
   };
 
+  // q^I is loaded once per sequence (a CTA's items are contiguous, so it
+  // meets each of its sequences in one run) into one of kQSlots slots; the
+  // ring stages carry only key tiles.
   if (warp == 0) {
     if (lane == 0) {
-      uint32_t g = 0;
+      uint32_t g = 0, nq = 0;
+      int qb = -1;
       for (int it = it0; it < it1 && !*abort_flag; ++it) {
         int b, j, avail;
         if (!item_ok(it, b, j, avail)) continue;
+        if (b != qb) {
+          const int qs = nq % kQSlots;
+          if (!mbar_wait(&q_empty[qs], ((nq / kQSlots) & 1) ^ 1)) { *abort_flag = 1; break; }
+          mbar_arrive_expect_tx(&q_full[qs], (uint32_t)(kchunks * qchunk));
+          for (int c = 0; c < kchunks; ++c) tma_load_3d(&tmQ, &q_full[qs], sm + qs * kQBytes + c * qchunk, 64 * c, 0, b);
+          qb = b;
+          ++nq;
+        }
         const int st = g % kStages;
         if (!mbar_wait(&empty[st], ((g / kStages) & 1) ^ 1)) { *abort_flag = 1; break; }
-        uint8_t* stage = sm + st * kStageBytes;
-        mbar_arrive_expect_tx(&full[st], (uint32_t)(kchunks * (qchunk + kchunk)));
-        for (int c = 0; c < kchunks; ++c) {
-          tma_load_3d(&tmQ, &full[st], stage + c * qchunk, 64 * c, 0, b);
-          tma_load_2d(&tmK, &full[st], stage + kQBytes + c * kchunk, 64 * c, b * a.cap + j * kM);
-        }
+        mbar_arrive_expect_tx(&full[st], (uint32_t)(kchunks * kchunk));
+        for (int c = 0; c < kchunks; ++c)
+          tma_load_2d(&tmK, &full[st], sm + kOffK + st * kKBytes + c * kchunk, 64 * c, b * a.cap + j * kM);
         ++g;
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kM, N);
-      uint32_t g = 0;
+      uint32_t g = 0, nq = 0;
+      int qb = -1;
       for (int it = it0; it < it1 && !*abort_flag; ++it) {
         int b, j, avail;
         if (!item_ok(it, b, j, avail)) continue;
+        if (b != qb) {
+          // the previous sequence's slot is free once its MMAs complete
+          if (nq > 0) mma_commit(&q_empty[(nq - 1) % kQSlots]);
+          if (!mbar_wait(&q_full[nq % kQSlots], (nq / kQSlots) & 1)) { *abort_flag = 1; break; }
+          qb = b;
+          ++nq;
+        }
         const int st = g % kStages, acc = g & 1;
         if (!mbar_wait(&full[st], (g / kStages) & 1) || !mbar_wait(&t_empty[acc], ((g >> 1) & 1) ^ 1)) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t qa = smem_u32(sm + st * kStageBytes);
-        const uint64_t qd = sdesc_k_sw128(qa), kd = sdesc_k_sw128(qa + kQBytes);
+        const uint64_t qd = sdesc_k_sw128(smem_u32(sm + ((nq - 1) % kQSlots) * kQBytes));
+        const uint64_t kd = sdesc_k_sw128(smem_u32(sm + kOffK + st * kKBytes));
         for (int c = 0; c < kchunks; ++c)
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
@@ -761,18 +795,18 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
       const int acc = g & 1;
       if (!warp_wait(&t_full[acc], (g >> 1) & 1)) { *abort_flag = 1; break; }
       tc_fence_after();
-      float sc = 0.f;
+      float sc4[4] = {0.f, 0.f, 0.f, 0.f};   // four partial sums (heads e mod 4)
       for (int hc = 0; hc < N; hc += 32) {
         float v[32];
         tmem_ld_32x32b_x32(tmem + lane_base + (uint32_t)(acc * 64 + hc), v);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sc = fmaf(w_my[hc + e], fmaxf(v[e], 0.f), sc);
+        for (int e = 0; e < 32; ++e) sc4[e & 3] = fmaf(w_my[hc + e], fmaxf(v[e], 0.f), sc4[e & 3]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_empty[acc]);
       const int s = j * kM + 32 * sub + lane;
-      if (s < avail) __stcg(a.scratch + (long long)b * a.cap + s, sc);
+      if (s < avail && dcheck(s < a.cap)) __stcg(a.scratch + (long long)b * a.cap + s, (sc4[0] + sc4[1]) + (sc4[2] + sc4[3]));
       ++g;
     }
   }
@@ -784,19 +818,21 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
   }
 }
 
-// Exact top-k of each decode row's score row, one CTA of 16 warps per
+// Exact top-k of each decode row's score row, one CTA of 32 warps per
 // sequence, same selection rule as warp_topk_ascending (the k largest
 // scores, equal scores lowest index first, ascending indices).  Radix select
-// on the order-preserving keys in three passes of 11, 11 and 10 bits; every
-// warp builds its own histogram of its share of the row (so increments only
-// collide within a warp), the 16 are summed, and warp 0 picks the digit.
-// The ordered output splits the row into 16 contiguous segments: a counting
-// pass, a prefix over the warps, and a writing pass.  The row is read from
-// global memory (L2) on every pass; shared memory holds only histograms.
+// on the order-preserving keys in three passes of 11, 11 and 10 bits; each
+// pair of warps builds its own histogram of its share of the row (so
+// increments only collide within the pair), the 16 are summed, and warp 0
+// picks the digit.  The ordered output splits the row into 32 contiguous
+// segments: a counting pass, a prefix over the warps, and a writing pass.
+// A row of up to kResident scores is read from global memory (L2) once and
+// kept in shared memory as keys; a longer row is read on every pass.
 namespace dsel {
-constexpr int kWarps = 16, kBins = 2048;
+constexpr int kWarps = 32, kThreads = 32 * kWarps, kHists = kWarps / 2, kBins = 2048;
+constexpr int kWords = 128;        // scratch words: the pick (3) and two per-warp counts (2 x 32)
 constexpr int kResident = 16384;   // rows of up to this many scores are selected from shared memory
-constexpr size_t kSmem = (size_t)(kWarps + 1) * kBins * 4 + 64 * 4 + (size_t)kResident * 4;
+constexpr size_t kSmem = (size_t)(kHists + 1) * kBins * 4 + kWords * 4 + (size_t)kResident * 4;
 }  // namespace dsel
 
 // Warp 0: the digit of the combined histogram hist[0..NB) holding the kk-th
@@ -845,15 +881,15 @@ __device__ __forceinline__ void dsel_pick(const int* hist, int kk, int* ws) {
   }
 }
 
-__global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch, const int* pos, int cap, int m,
+__global__ void __launch_bounds__(dsel::kThreads) decode_select_kernel(const float* scratch, const int* pos, int cap, int m,
                                                             int topk, int* idx) {
   using namespace dsel;
   constexpr unsigned kFull = 0xffffffffu;
   extern __shared__ __align__(16) int dsm[];
-  int* whist = dsm;                         // [kWarps][kBins] per-warp histograms
-  int* hist = dsm + kWarps * kBins;         // [kBins] combined
-  int* ws = hist + kBins;                   // [64] scratch words
-  uint32_t* keys = reinterpret_cast<uint32_t*>(ws + 64);   // [kResident] the row's keys, when it fits
+  int* whist = dsm;                         // [kHists][kBins] histograms of the warp pairs
+  int* hist = dsm + kHists * kBins;         // [kBins] combined
+  int* ws = hist + kBins;                   // [kWords] scratch words
+  uint32_t* keys = reinterpret_cast<uint32_t*>(ws + kWords);   // [kResident] the row's keys, when it fits
   const int b = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t = pos[b];
@@ -870,22 +906,22 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
   // memory.  Longer rows are read from L2 on every pass.
   const bool resident = avail <= kResident;
   if (resident) {
-    for (int i0 = tid; i0 < avail; i0 += 512 * 8) {
+    for (int i0 = tid; i0 < avail; i0 += kThreads * 8) {
       float v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int i = i0 + 512 * u;
+        const int i = i0 + kThreads * u;
         v[u] = i < avail ? __ldcg(row + i) : 0.f;
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int i = i0 + 512 * u;
+        const int i = i0 + kThreads * u;
         if (i < avail) keys[i] = ordered_key(v[u]);
       }
     }
   }
   auto key_at = [&](int i) -> uint32_t { return resident ? keys[i] : ordered_key(__ldcg(row + i)); };
-  int* myh = whist + warp * kBins;
+  int* myh = whist + (warp >> 1) * kBins;
   uint32_t prefix = 0, mask = 0;
   int kk = topk;
 #pragma unroll 1
@@ -893,10 +929,10 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
     const int shift = pass == 0 ? 21 : pass == 1 ? 10 : 0;
     const int width = pass == 2 ? 10 : 11;
     const uint32_t dmask = (1u << width) - 1u;
-    for (int i = lane; i < kBins / 4; i += 32) reinterpret_cast<int4*>(myh)[i] = make_int4(0, 0, 0, 0);
+    for (int i = 32 * (warp & 1) + lane; i < kBins / 4; i += 64) reinterpret_cast<int4*>(myh)[i] = make_int4(0, 0, 0, 0);
     __syncthreads();
-    // this thread's scores: 4 consecutive per step, the CTA covering 2048 per step
-    for (int i0 = 4 * tid; i0 < avail; i0 += 4 * 512) {
+    // this thread's scores: 4 consecutive per step, the CTA covering 4 kThreads per step
+    for (int i0 = 4 * tid; i0 < avail; i0 += 4 * kThreads) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int i = i0 + u;
@@ -907,10 +943,10 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
       }
     }
     __syncthreads();
-    for (int bin = tid; bin < kBins; bin += 512) {
+    for (int bin = tid; bin < kBins; bin += kThreads) {
       int c = 0;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) c += whist[w * kBins + bin];
+      for (int w = 0; w < kHists; ++w) c += whist[w * kBins + bin];
       hist[bin] = c;
     }
     __syncthreads();
@@ -922,11 +958,13 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
     prefix |= (uint32_t)ws[0] << shift;
     mask |= dmask << shift;
     kk -= ws[1];
+    const bool settled = ws[2] == kk;   // every key of the bin is needed: key >= prefix decides
     __syncthreads();
+    if (settled) break;
   }
   const uint32_t thr = prefix;
   const int need_eq = kk;
-  // ordered output over 16 contiguous segments
+  // ordered output over kWarps contiguous segments
   const int seg = (((avail + kWarps - 1) / kWarps) + 31) & ~31;
   const int s0 = min(avail, warp * seg), s1 = min(avail, s0 + seg);
   int n_gt = 0, n_eq = 0;
@@ -957,7 +995,7 @@ __global__ void __launch_bounds__(512) decode_select_kernel(const float* scratch
     const bool take = gt || (eq && eq_seen + __popc(beq & lt) < need_eq);
     const unsigned btk = __ballot_sync(kFull, take);
     const int p = out_off + __popc(btk & lt);
-    if (take && p < topk) out[p] = i;
+    if (take && dguard(p < topk)) out[p] = i;
     out_off += __popc(btk);
     eq_seen += __popc(beq);
   }

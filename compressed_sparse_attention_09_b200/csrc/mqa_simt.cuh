@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(256) mqa_simt_kernel(MqaArgs a) {
         if (lane == 0 && h0 == 2 * warp && warp == 0) flag_status(kStatusBadIndex);
         continue;
       }
+      if (!dcheck(base + s < rowmap_entries(a.rm, gridDim.x))) continue;
       float cv[VEC];
       load_lane<T, VEC>(Cb + (long long)s * C + lane * VEC, cv);
 #pragma unroll

@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
       long long base;
       int avail;
       row_entries(a.rm, row, base, avail);
+      const long long n_ent = rowmap_entries(a.rm, a.rows);
       const int* ir = a.idx + (long long)row * a.topk;
       const int ntiles = mqa_ntiles(ir, a.topk, avail);
       if (ntiles == 0) continue;
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
 #pragma unroll
         for (int i = 0; i < kTile / 4; ++i) {
           const int r = r0 + 4 * i;
-          const bool v = s[i] >= 0 && s[i] < avail;
+          const bool v = s[i] >= 0 && s[i] < avail && dcheck(base + s[i] < n_ent);
           if (c16 == 0 && !v && s[i] != -1) flag_status(kStatusBadIndex);
           const __nv_bfloat16* src = v ? a.C + (base + s[i]) * kC + c16 * 8 : a.C;
           cp_async16(cst + sw128(r, c16 & 7), src, v ? 16u : 0u);

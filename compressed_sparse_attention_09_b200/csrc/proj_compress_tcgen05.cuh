@@ -132,6 +132,7 @@ __device__ __forceinline__ void pcx_compress8(const ProjCompressArgs& a, int cg,
   Vec16<__nv_bfloat16> pk;
 #pragma unroll
   for (int e = 0; e < 8; ++e) pk.e[e] = __float2bfloat16_rn(res[e]);
+  if (!dcheck(entry >= 0 && entry < a.total_blocks)) return;
   __nv_bfloat16* dst = main ? a.Ccomp + (long long)entry * a.c + chg : a.KIcomp + (long long)entry * a.cI + chg;
   *reinterpret_cast<uint4*>(dst) = pk.u;
 }

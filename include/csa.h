@@ -53,7 +53,8 @@ typedef enum {
   CSA_ERR_DEVICE_TIMEOUT = 4, /* a bounded device wait ran out           */
   CSA_ERR_BAD_INDEX = 5,      /* out-of-range block index seen on device */
   CSA_ERR_BAD_METADATA = 6,   /* cu_seqlens / cu_blocks inconsistent     */
-  CSA_ERR_WORKSPACE = 7       /* workspace smaller than required         */
+  CSA_ERR_WORKSPACE = 7,      /* workspace smaller than required         */
+  CSA_ERR_DEVICE_BOUNDS = 8   /* debug build: an index check failed      */
 } csa_status;
 
 typedef enum { CSA_F32 = 0, CSA_BF16 = 1 } csa_dtype;
@@ -432,6 +433,15 @@ csa_status csa_get_device_status(void* stream);
 
 /* Static, NUL-terminated description of a status code. */
 const char* csa_status_string(csa_status s);
+
+/* 1 in the debug build of this library (libcsa_debug.so, compiled with
+ * CSA_DEBUG), 0 in the release build (libcsa.so).  The debug build has the
+ * same entry points and results; in addition its kernels check, before each
+ * global access whose index the kernel computes (a gathered entry row, a
+ * score or index written for a query row, a compressed entry, a cache slot),
+ * that the index lies in its range, and where it does not they skip the
+ * access and record CSA_ERR_DEVICE_BOUNDS in the status word. */
+int csa_debug_build(void);
 
 /* Number of kernels this library has enqueued in this process so far (all
  * devices, all streams).  A monotone counter for accounting; never reset. */

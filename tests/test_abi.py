@@ -28,6 +28,21 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), name
 
 
+def test_debug_build_exports_every_declared_symbol():
+    """libcsa_debug.so (device-side index checks) is built beside libcsa.so
+    with the same entry points, and each reports which build it is."""
+    debug = ctypes.CDLL(os.path.join(capi.PKG, "libcsa_debug.so"))
+    for name in declared_functions():
+        assert hasattr(debug, name), name
+    debug.csa_debug_build.restype = ctypes.c_int
+    assert debug.csa_debug_build() == 1
+    release = ctypes.CDLL(os.path.join(capi.PKG, "libcsa.so"))
+    release.csa_debug_build.restype = ctypes.c_int
+    assert release.csa_debug_build() == 0
+    debug.csa_status_string.restype = ctypes.c_char_p
+    assert b"debug-build" in debug.csa_status_string(8)
+
+
 def test_no_python_fallback_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(capi, "_lib", None)
     monkeypatch.setattr(capi, "LIB_PATH", str(tmp_path / "missing.so"))
