@@ -58,7 +58,7 @@ struct IdxDecQ8Args {
 };
 
 namespace idxq8 {
-constexpr int kM = 128, kCI = 128, kStages = 8, kKBufs = 2, kQSlots = 2;
+constexpr int kM = 128, kCI = 128, kStages = 7, kKBufs = 2, kQSlots = 2;
 constexpr int kQBytes = 64 * 128 * 2;          // q^I fp16, up to 64 heads x 128, two 64-column chunks
 constexpr int kCodeBytes = kM * kCI;           // 128 entries x 128 codes (128-byte swizzled rows)
 constexpr int kKChunk = kM * 128;              // fp16 [128 entries x 64 channels]
@@ -66,9 +66,10 @@ constexpr int kKBytes = 2 * kKChunk;
 constexpr int kOffC = kQSlots * kQBytes;       // code stages
 constexpr int kOffK = kOffC + kStages * kCodeBytes;
 constexpr int kOffW = kOffK + kKBufs * kKBytes;
-constexpr size_t kSmem = 1024 + (size_t)kOffW + 4 * 64 * 4 + 256;
+constexpr int kEpiWarps = 8;                   // warps 2-5 and 10-13: even and odd items of the CTA
+constexpr size_t kSmem = 1024 + (size_t)kOffW + kEpiWarps * 64 * 4 + 256;
 constexpr int kCvtWarps = 4;                   // warps 6-9 widen the codes
-constexpr int kThreads = 32 * (6 + kCvtWarps);
+constexpr int kThreads = 32 * (2 + kEpiWarps + kCvtWarps);
 }  // namespace idxq8
 
 // Two E4M3 codes (the low and high byte of v) to an fp16 pair, low code in
@@ -89,7 +90,8 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
 // (q^I fp16 once per sequence, the tile's codes per stage); warps 6-9: widen the codes to
 // fp16 in the MMA's swizzled K-major layout (two buffers); warp 1: MMA
 // issuer and TMEM owner (D[128 entries x n_h^I], two accumulators); warps
-// 2-5: epilogue (ReLU, head weights, entry scale).  All waits are bounded.
+// 2-5 and 10-13: epilogue (ReLU, head weights, entry scale), one group per
+// accumulator.  All waits are bounded.
 __global__ void __launch_bounds__(idxq8::kThreads, 1)
     indexer_decode_q8_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                              IdxDecQ8Args a) {
@@ -99,7 +101,7 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* kbuf = sm + kOffK;
   float* w_s = reinterpret_cast<float*>(sm + kOffW);            // 4 epilogue warps x 64
-  uint64_t* bars = reinterpret_cast<uint64_t*>(w_s + 4 * 64);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(w_s + kEpiWarps * 64);
   uint64_t* full = bars;                   // [kStages] codes landed
   uint64_t* empty = full + kStages;        // [kStages] codes widened (kCvtWarps arrivals)
   uint64_t* kfull = empty + kStages;       // [kKBufs] fp16 tile written (kCvtWarps arrivals)
@@ -133,12 +135,17 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
 
   const int per = (items + gridDim.x - 1) / gridDim.x;
   const int it0 = blockIdx.x * per, it1 = min(items, it0 + per);
+  // the sequence's visible count is read once per sequence, not per item
+  int cached_b = -1, cached_avail = 0;
   auto item_ok = [&](int it, int& b, int& j, int& avail) {
     b = it / a.tiles_per_seq;
     j = it - b * a.tiles_per_seq;
-    const int t = a.pos[b];
-    avail = t >= 0 ? t / a.m : 0;
-    if (avail > a.cap) avail = a.cap;
+    if (b != cached_b) {
+      const int t = a.pos[b];
+      cached_avail = t >= 0 ? min(t / a.m, a.cap) : 0;
+      cached_b = b;
+    }
+    avail = cached_avail;
     return j * kM < avail;
   };
 
@@ -200,7 +207,7 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
         ++g;
       }
     }
-  } else if (warp >= 6) {
+  } else if (warp >= 6 && warp < 6 + kCvtWarps) {
     // ---------------------------------------------------------------- code widening (warps 6-9)
     // thread -> 16-byte unit u = t % 8 (16 codes) of rows t / 8 + 16 i; all
     // of a thread's row loads are issued before any conversion
@@ -251,9 +258,11 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
       ++g;
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 2-5)
-    const int sub = warp & 3;
-    float* w_my = w_s + (warp - 2) * 64;
+    // ---------------------------------------------------------------- epilogue (warps 2-5 and 10-13)
+    // warps 2-5 take the CTA's even items (accumulator 0), warps 10-13 the
+    // odd ones (accumulator 1), so two items are folded at a time
+    const int sub = warp & 3, grp = warp < 6 ? 0 : 1;
+    float* w_my = w_s + (warp < 6 ? warp - 2 : warp - 6 - kCvtWarps + 4) * 64;
     const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
     uint32_t g = 0;
     int wb = -1;
@@ -261,6 +270,7 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
       if (warp_aborted(abort_flag)) break;
       int b, j, avail;
       if (!item_ok(it, b, j, avail)) continue;
+      if ((int)(g & 1) != grp) { ++g; continue; }
       if (b != wb) {
         for (int hh = lane; hh < N; hh += 32) w_my[hh] = a.wI[(long long)b * a.ld_wI + hh];
         __syncwarp();

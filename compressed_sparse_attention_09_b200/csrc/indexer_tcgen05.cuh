@@ -659,13 +659,14 @@ struct IdxDecArgs {
 };
 
 namespace idxdec {
-constexpr int kM = 128, kStages = 6, kQSlots = 2;
+constexpr int kM = 128, kStages = 5, kQSlots = 2;
 constexpr int kQBytes = 64 * 128 * 2;    // up to [64 heads x 128] bf16 as two 64-column chunks
 constexpr int kKBytes = kM * 128 * 2;    // [128 blocks x 128] bf16 as two chunks
 constexpr int kOffK = kQSlots * kQBytes;
 constexpr int kOffW = kOffK + kStages * kKBytes;
-constexpr size_t kSmem = 1024 + (size_t)kOffW + 4 * 64 * 4 + 256;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;             // two groups of four: even and odd items of the CTA
+constexpr size_t kSmem = 1024 + (size_t)kOffW + kEpiWarps * 64 * 4 + 256;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
 }  // namespace idxdec
 
 __global__ void __launch_bounds__(idxdec::kThreads, 1)
@@ -675,8 +676,8 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
   using namespace idxdec;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* w_s = reinterpret_cast<float*>(sm + kOffW);     // 4 warps x 64
-  uint64_t* bars = reinterpret_cast<uint64_t*>(w_s + 4 * 64);
+  float* w_s = reinterpret_cast<float*>(sm + kOffW);     // kEpiWarps warps x 64
+  uint64_t* bars = reinterpret_cast<uint64_t*>(w_s + kEpiWarps * 64);
   uint64_t* full = bars;                   // [kStages] key tile landed
   uint64_t* empty = full + kStages;        // [kStages]
   uint64_t* t_full = empty + kStages;      // [2]
@@ -709,12 +710,17 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
   // items of this CTA: a contiguous range, so consecutive items share a sequence
   const int per = (items + gridDim.x - 1) / gridDim.x;
   const int it0 = blockIdx.x * per, it1 = min(items, it0 + per);
+  // the sequence's visible count is read once per sequence, not per item
+  int cached_b = -1, cached_avail = 0;
   auto item_ok = [&](int it, int& b, int& j, int& avail) {
     b = it / a.tiles_per_seq;
     j = it - b * a.tiles_per_seq;
-    const int t = a.pos[b];
-    avail = t >= 0 ? t / a.m : 0;
-    if (avail > a.cap) avail = a.cap;
+    if (b != cached_b) {
+      const int t = a.pos[b];
+      cached_avail = t >= 0 ? min(t / a.m, a.cap) : 0;
+      cached_b = b;
+    }
+    avail = cached_avail;
     return j * kM < avail;
   };
 
@@ -778,7 +784,9 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
       }
     }
   } else {
-    const int sub = warp & 3;
+    // epilogue: warps 2-5 take the CTA's even items (accumulator 0), warps
+    // 6-9 the odd ones (accumulator 1), so two items are folded at a time
+    const int sub = warp & 3, grp = (warp - 2) >> 2;
     float* w_my = w_s + (warp - 2) * 64;
     const uint32_t lane_base = (uint32_t)(32 * sub) << 16;
     uint32_t g = 0;
@@ -787,6 +795,7 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
       if (warp_aborted(abort_flag)) break;
       int b, j, avail;
       if (!item_ok(it, b, j, avail)) continue;
+      if ((int)(g & 1) != grp) { ++g; continue; }
       if (b != wb) {
         for (int h = lane; h < N; h += 32) w_my[h] = a.wI[(long long)b * a.ld_wI + h];
         __syncwarp();
