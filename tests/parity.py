@@ -129,7 +129,7 @@ def score_delta(scores_store, scores_exact, qI_t, wI_t, KI_avail):
 def check_topk_row(gpu_row, scores, k, delta=None, gap_rel=GAP_REL):
     """Check one GPU top-k row against the oracle's fp64 scores under the
     protocol of this module.  delta: per-candidate admissible perturbation
-    (None = 0).  gap_rel: the relative margin (the benchmark spec's 1e-3; stage
+    (None = 0).  gap_rel: the relative margin (1e-3 of the k-th score; stage
     tests, whose two sides see bit-identical inputs, pass 0 and so demand
     exactness wherever the set is stable under the fp32 evaluation bound
     alone, which is stricter).  Returns "all" (k_eff = avail: every block),
