@@ -522,6 +522,18 @@ def test_decode_tensor_core_indexer(m):
     decode_case(dims, B=5, pos0=301, cap=400, steps=6, seed=63 + m, check=[0, 3, 4])
 
 
+@pytest.mark.parametrize("q8", [False, True])
+def test_decode_indexer_many_sequences_per_cta(q8):
+    """400 sequences of one 128-entry tile each: every CTA of the decode
+    scoring kernels meets three sequences in its run of items, so the two
+    q^I slots are reused (the third sequence waits for the first one's MMAs)
+    and the epilogue groups alternate across sequence changes.  Sequences at
+    the start, middle and end of CTA runs are checked against the oracle."""
+    dims = csa.Dims(d=256, c=128, m=4, cI=128, nhI=64, nh=4, dc=128, topk=16, dtype=csa.CSA_BF16)
+    decode_case(dims, B=400, pos0=4 * 100 + 1, cap=128, steps=2, seed=73 + int(q8),
+                check=[0, 1, 2, 147, 148, 149, 296, 297, 399], q8=q8)
+
+
 def test_decode_selection_of_rows_longer_than_shared_memory():
     """Cached rows longer than the 16384 scores the selection keeps in shared
     memory are selected from L2 instead; both forms must pick the oracle's set."""
