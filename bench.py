@@ -150,6 +150,7 @@ class ClockSampler:
 # on the named workload.  A kernel change makes the figure stale: it is then
 # removed until the kernel is captured again.
 MEASURED_TRAFFIC = {
+    ("prefill", "A4_indexer_topk"): 102_978_816 + 7_641_088,
     ("prefill", "A5_sparse_mqa"): 556_276_992 + 493_239_040,
 }
 
