@@ -155,21 +155,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] . B[smem]^T, bf16 inputs, fp32 accumulation.  A is
-// K-major in TMEM with the layout of an accumulator of the same M: for
-// M = 64, row r in lane 32 (r / 16) + r % 16 (the A address must sit at a
-// lane-quarter start: a lane offset of 16 is rejected as misaligned), and
-// the bf16 pair (k = 2j, 2j + 1) packed in column j, even k in the low half.
-__device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Arrive on `bar` once every tcgen05 operation this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -283,11 +268,6 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const float* 
 }
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Instruction descriptor as idesc_bf16_f32 with the A operand MN-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32_amn(int M, int N) {
-  return idesc_bf16_f32(M, N) | (1u << 15);
-}
 
 // Instruction descriptor as idesc_bf16_f32 with the B operand MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
