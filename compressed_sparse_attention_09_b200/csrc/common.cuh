@@ -49,6 +49,19 @@ __device__ __forceinline__ constexpr bool dguard(bool ok) { return ok; }
 constexpr unsigned long long kDefaultWaitNs = 1500000000ull;   // 1.5 s
 __device__ unsigned long long g_wait_ns = kDefaultWaitNs;
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels launched with programmatic stream serialization may be scheduled
+// while the previous kernel on the stream is still finishing.  Each such
+// kernel calls pdl_prologue_done() once its prologue (barrier set-up, TMEM
+// allocation, descriptor prefetch; no global memory) is over: it lets the
+// next kernel be scheduled, then waits until the previous kernel has
+// completed and its writes are visible, before any global-memory access.
+// Without a programmatic predecessor the wait returns at once.
+__device__ __forceinline__ void pdl_prologue_done() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- conversions
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }

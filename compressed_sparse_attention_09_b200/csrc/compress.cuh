@@ -218,6 +218,7 @@ struct AppendArgs {
 // one scale, max |v| / 448) instead of a bf16 one.
 template <typename T, int M, bool Q8 = false>
 __global__ void __launch_bounds__(256) cache_append_kernel(AppendArgs a) {
+  pdl_prologue_done();
   __shared__ float ki_s[1024];
   const int b = blockIdx.x;
   const int t = a.pos[b];

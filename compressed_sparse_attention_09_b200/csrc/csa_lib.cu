@@ -45,6 +45,28 @@ std::atomic<uint64_t> g_launches{0};
     if (cudaGetLastError() != cudaSuccess) return CSA_ERR_CUDA; \
   } while (0)
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel on the stream finishes, and overlaps its
+// prologue with that kernel's tail.  Every kernel launched this way calls
+// pdl_prologue_done() (common.cuh) before its first global-memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr;
+  memset(&attr, 0, sizeof(attr));
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // NVTX ranges around each stage's launches (host side), compiled in only
 // with -DCSA_NVTX so that a profiler timeline shows the stages by name.
 #ifdef CSA_NVTX
@@ -258,12 +280,14 @@ csa_status launch_tc_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const Tc
     return CSA_ERR_CUDA;
   const int tiles = ((g.M + Cfg::BM - 1) / Cfg::BM) * ((g.N + BN - 1) / BN) * g.k_split;
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  k<<<grid, 192, Cfg::SMEM, st>>>(ta, tb, g);
+  if (launch_pdl(k, dim3(grid), dim3(192), Cfg::SMEM, st, ta, tb, g) != cudaSuccess) return CSA_ERR_CUDA;
   CSA_CHECK_LAUNCH();
   if (g.k_split > 1) {
     const int m_pad = ((g.M + Cfg::BM - 1) / Cfg::BM) * Cfg::BM;
     const long long n = (long long)g.N * g.M;
-    gemm_split_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(g.part, g.k_split, g.M, m_pad, g.N, g.out);
+    if (launch_pdl(gemm_split_reduce_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, g.part, g.k_split,
+                   g.M, m_pad, g.N, g.out) != cudaSuccess)
+      return CSA_ERR_CUDA;
     CSA_CHECK_LAUNCH();
   }
   return CSA_OK;
@@ -417,7 +441,8 @@ csa_status launch_indexer_tc(const csa_dims* d, const IndexerArgs& a, int T, int
     return CSA_ERR_CUDA;
   const long long items = (long long)t.q_blocks + a.rm.nseq;
   const int grid = items < sm_count() ? (int)items : sm_count();
-  kern<<<grid, idxtc::kThreads, idxtc::kSmem, st>>>(tk, tq, t);
+  if (launch_pdl(kern, dim3(grid), dim3(idxtc::kThreads), idxtc::kSmem, st, tk, tq, t) != cudaSuccess)
+    return CSA_ERR_CUDA;
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }
@@ -469,7 +494,8 @@ csa_status launch_mqa(const csa_dims* d, const MqaArgs& a, int rows, cudaStream_
       return CSA_ERR_CUDA;
     const long long items = (long long)rows * (d->nh / mqa::kHeads);
     const int grid = items < sm_count() ? (int)items : sm_count();
-    mqa_tc_kernel<<<grid, mqa::kThreads, mqa::kSmem, st>>>(tq, t);
+    if (launch_pdl(mqa_tc_kernel, dim3(grid), dim3(mqa::kThreads), mqa::kSmem, st, tq, t) != cudaSuccess)
+      return CSA_ERR_CUDA;
     CSA_CHECK_LAUNCH();
     return CSA_OK;
   }
@@ -1156,12 +1182,15 @@ csa_status launch_append(const csa_dims* d, const void* packed, const void* rows
   a.BbI = reinterpret_cast<const float*>(at((void*)packed, P.bbI));
   a.c = d->c; a.cI = d->cI; a.cap = cap; a.ring_w = 4 * d->c + 4 * d->cI;
   a.KIcodes = KIcodes; a.KIscale = KIscale;
-#define CSA_APPEND_CASE(MM)                                                                \
-  case MM:                                                                                 \
-    if (q8) cache_append_kernel<bf16, MM, true><<<B, 256, 0, st>>>(a);                     \
-    else if (d->dtype == CSA_BF16) cache_append_kernel<bf16, MM><<<B, 256, 0, st>>>(a);    \
-    else cache_append_kernel<float, MM><<<B, 256, 0, st>>>(a);                             \
-    break;
+#define CSA_APPEND_CASE(MM)                                                                    \
+  case MM: {                                                                                   \
+    const cudaError_t e_ = q8 ? launch_pdl(cache_append_kernel<bf16, MM, true>, dim3(B), dim3(256), 0, st, a) \
+                         : d->dtype == CSA_BF16                                                \
+                             ? launch_pdl(cache_append_kernel<bf16, MM>, dim3(B), dim3(256), 0, st, a)       \
+                             : launch_pdl(cache_append_kernel<float, MM>, dim3(B), dim3(256), 0, st, a);     \
+    if (e_ != cudaSuccess) return CSA_ERR_CUDA;                                                \
+    break;                                                                                     \
+  }
   switch (d->m) {
     CSA_APPEND_CASE(1)
     CSA_APPEND_CASE(2)
@@ -1210,13 +1239,17 @@ csa_status launch_indexer_decode_tc(const csa_dims* d, const IndexerArgs& a, int
     return CSA_ERR_CUDA;
   const long long items = (long long)B * t.tiles_per_seq;
   const int grid = items < sm_count() ? (int)items : sm_count();
-  indexer_decode_tc_kernel<<<grid, idxdec::kThreads, idxdec::kSmem, st>>>(tk, tq, t);
+  if (launch_pdl(indexer_decode_tc_kernel, dim3(grid), dim3(idxdec::kThreads), idxdec::kSmem, st, tk, tq, t) !=
+      cudaSuccess)
+    return CSA_ERR_CUDA;
   CSA_CHECK_LAUNCH();
   if (after_scores && cudaEventRecord(after_scores, st) != cudaSuccess) return CSA_ERR_CUDA;
   if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsel::kSmem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
-  decode_select_kernel<<<B, dsel::kThreads, dsel::kSmem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
+  if (launch_pdl(decode_select_kernel, dim3(B), dim3(dsel::kThreads), dsel::kSmem, st, (const float*)scratch,
+                 a.rm.pos, cap, d->m, d->topk, a.idx) != cudaSuccess)
+    return CSA_ERR_CUDA;
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }
@@ -1228,8 +1261,9 @@ csa_status launch_indexer_decode_q8(const csa_dims* d, const IndexerArgs& a, con
                                     cudaEvent_t after_scores = nullptr) {
   CSA_RANGE("A4 indexer_topk (decode, e4m3 keys)");
   const int w = d->nhI * d->cI;
-  bf16_to_f16_rows_kernel<<<(unsigned)(((long long)B * w + 255) / 256), 256, 0, st>>>(
-      static_cast<const bf16*>(a.qI), a.ld_qI, B, w, static_cast<__half*>(qf16));
+  if (launch_pdl(bf16_to_f16_rows_kernel, dim3((unsigned)(((long long)B * w + 255) / 256)), dim3(256), 0, st,
+                 static_cast<const bf16*>(a.qI), (long long)a.ld_qI, B, w, static_cast<__half*>(qf16)) != cudaSuccess)
+    return CSA_ERR_CUDA;
   CSA_CHECK_LAUNCH();
   CUtensorMap tk, tq;
   if (!make_tmap_u8(&tk, codes, d->cI, (uint64_t)B * cap, (uint64_t)d->cI, 128, idxq8::kM) ||
@@ -1243,13 +1277,17 @@ csa_status launch_indexer_decode_q8(const csa_dims* d, const IndexerArgs& a, con
     return CSA_ERR_CUDA;
   const long long items = (long long)B * t.tiles_per_seq;
   const int grid = items < sm_count() ? (int)items : sm_count();
-  indexer_decode_q8_kernel<<<grid, idxq8::kThreads, idxq8::kSmem, st>>>(tk, tq, t);
+  if (launch_pdl(indexer_decode_q8_kernel, dim3(grid), dim3(idxq8::kThreads), idxq8::kSmem, st, tk, tq, t) !=
+      cudaSuccess)
+    return CSA_ERR_CUDA;
   CSA_CHECK_LAUNCH();
   if (after_scores && cudaEventRecord(after_scores, st) != cudaSuccess) return CSA_ERR_CUDA;
   if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsel::kSmem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
-  decode_select_kernel<<<B, dsel::kThreads, dsel::kSmem, st>>>(scratch, a.rm.pos, cap, d->m, d->topk, a.idx);
+  if (launch_pdl(decode_select_kernel, dim3(B), dim3(dsel::kThreads), dsel::kSmem, st, (const float*)scratch,
+                 a.rm.pos, cap, d->m, d->topk, a.idx) != cudaSuccess)
+    return CSA_ERR_CUDA;
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }

@@ -43,6 +43,7 @@ __global__ void quantize_rows_e4m3_kernel(const __nv_bfloat16* src, long long ld
 // q^I rows (bf16, row stride ld) to fp16 [n, w]: the quantised indexer
 // multiplies the fp16 codes by fp16 queries (one operand type per MMA).
 __global__ void bf16_to_f16_rows_kernel(const __nv_bfloat16* src, long long ld, int n, int w, __half* dst) {
+  pdl_prologue_done();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)n * w) return;
   const int r = (int)(i / w), j = (int)(i % w);
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(idxq8::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_prologue_done();
   const uint32_t tmem = *tmem_slot;
 
   const int per = (items + gridDim.x - 1) / gridDim.x;

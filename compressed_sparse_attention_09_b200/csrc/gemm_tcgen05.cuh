@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_prologue_done();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
@@ -312,6 +313,7 @@ __global__ void __launch_bounds__(192, 1)
 // whatever the timing of the slices) and stored as that GEMM stores its
 // output: D[r][j] at output row j, column r, through the segments of `out`.
 __global__ void gemm_split_reduce_kernel(const float* part, int k_split, int M, int Mpad, int N, GemmOut out) {
+  pdl_prologue_done();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)N * M) return;
   const int j = (int)(i / M), r = (int)(i % M);

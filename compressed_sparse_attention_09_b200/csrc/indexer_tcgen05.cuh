@@ -469,6 +469,7 @@ __global__ void __launch_bounds__(idxtc::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_prologue_done();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
@@ -705,6 +706,7 @@ __global__ void __launch_bounds__(idxdec::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_prologue_done();
   const uint32_t tmem = *tmem_slot;
 
   // items of this CTA: a contiguous range, so consecutive items share a sequence
@@ -892,6 +894,7 @@ __device__ __forceinline__ void dsel_pick(const int* hist, int kk, int* ws) {
 
 __global__ void __launch_bounds__(dsel::kThreads) decode_select_kernel(const float* scratch, const int* pos, int cap, int m,
                                                             int topk, int* idx) {
+  pdl_prologue_done();
   using namespace dsel;
   constexpr unsigned kFull = 0xffffffffu;
   extern __shared__ __align__(16) int dsm[];

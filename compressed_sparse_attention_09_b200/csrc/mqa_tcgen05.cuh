@@ -155,6 +155,7 @@ __global__ void __launch_bounds__(mqa::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_prologue_done();
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 8) {

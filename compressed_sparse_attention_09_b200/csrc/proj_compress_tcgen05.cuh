@@ -183,6 +183,7 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_prologue_done();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
