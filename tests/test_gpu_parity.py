@@ -534,11 +534,13 @@ def test_decode_indexer_many_sequences_per_cta(q8):
                 check=[0, 1, 2, 147, 148, 149, 296, 297, 399], q8=q8)
 
 
-def test_decode_selection_of_rows_longer_than_shared_memory():
+@pytest.mark.parametrize("avail", [17000, 34000])
+def test_decode_selection_of_rows_longer_than_shared_memory(avail):
     """Cached rows longer than the 16384 scores the selection keeps in shared
-    memory are selected from L2 instead; both forms must pick the oracle's set."""
+    memory are selected from L2 instead (one and two times that length); the
+    streamed form must pick the oracle's set."""
     dims = csa.Dims(d=256, c=128, m=4, cI=128, nhI=64, nh=4, dc=128, topk=64, dtype=csa.CSA_BF16)
-    decode_case(dims, B=2, pos0=4 * 17000 + 1, cap=17100, steps=2, seed=67, check=[0, 1])
+    decode_case(dims, B=2, pos0=4 * avail + 1, cap=avail + 100, steps=2, seed=67, check=[0, 1])
 
 
 def test_decode_projection_split_over_k():
