@@ -14,7 +14,12 @@
  *    frees caller memory and never synchronises, except in
  *    csa_get_device_status().
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
- *    stream).  All work is enqueued asynchronously on it, in order.
+ *    stream).  All work is enqueued asynchronously on it, in order.  Most
+ *    kernels are launched with programmatic stream serialization: a kernel
+ *    may start its on-chip set-up while the previous kernel on the stream
+ *    finishes, but it waits for that kernel to complete before it reads or
+ *    writes any memory, so the order of all memory effects is the stream
+ *    order.
  *  - Matrices are dense row-major.  "ld" arguments are row strides in
  *    ELEMENTS.  Element type = csa_dims.dtype for activations and weights
  *    (fp32 or bf16); the indexer head weights w^I are always fp32 and block
