@@ -564,7 +564,7 @@ def run_decode(dev, args, peaks, flush, stream):
     no_flush = lambda: None   # noqa: E731
     dms = statistics.mean(timed_steps(dr.step, args.steps, no_flush, stream))
     dms_flushed = statistics.mean(timed_steps(dr.step, max(3, min(args.steps, 50)), flush, stream))
-    names = ("A1_project_hidden", "A6_cache_append", "A2_project_query", "A4_indexer_scores", "A4_topk_select",
+    names = ("A1_project_hidden", "A2_project_query", "A6_cache_append", "A4_indexer_scores", "A4_topk_select",
              "A5_sparse_mqa")
     in_step_ms = staged_step_ms(dr.step_staged, len(names), max(3, min(args.steps, 50)), no_flush, stream)
     st = csa.csa_get_device_status()

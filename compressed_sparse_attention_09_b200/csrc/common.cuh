@@ -53,13 +53,15 @@ __device__ unsigned long long g_wait_ns = kDefaultWaitNs;
 // Kernels launched with programmatic stream serialization may be scheduled
 // while the previous kernel on the stream is still finishing.  Each such
 // kernel calls pdl_prologue_done() once its prologue (barrier set-up, TMEM
-// allocation, descriptor prefetch; no global memory) is over: it lets the
-// next kernel be scheduled, then waits until the previous kernel has
-// completed and its writes are visible, before any global-memory access.
+// allocation, descriptor prefetch; no global memory) is over: it waits until
+// the previous kernel has completed and its writes are visible, then lets
+// the next kernel be scheduled.  Waiting first means that a kernel scheduled
+// early after this one may rely on everything before this one on the stream
+// being complete (only this kernel's own writes are still in flight).
 // Without a programmatic predecessor the wait returns at once.
 __device__ __forceinline__ void pdl_prologue_done() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- conversions

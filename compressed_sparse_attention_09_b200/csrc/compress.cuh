@@ -210,16 +210,18 @@ struct AppendArgs {
   int c, cI, cap, ring_w;
   uint8_t* KIcodes;     // quantised key cache (Q8): [B, cap, cI] E4M3 codes
   float* KIscale;       // [B, cap] scales
+  int wait_late;        // 1: the previous kernel on the stream reads and writes none of the above
+                        // and was scheduled after everything before it had completed (decode:
+                        // the c^Q-side projection), so the append runs beside it and waits for it
+                        // only at its end; 0: wait for the previous kernel before any access
 };
 
 // One CTA per sequence: store the token's row in ring slot t mod 2m, then, if
 // t closes block i = (t+1)/m - 1, compress that block from the ring.  Q8:
 // the indexer-key entry goes to an E4M3 cache (its bf16 value quantised with
 // one scale, max |v| / 448) instead of a bf16 one.
-template <typename T, int M, bool Q8 = false>
-__global__ void __launch_bounds__(256) cache_append_kernel(AppendArgs a) {
-  pdl_prologue_done();
-  __shared__ float ki_s[1024];
+template <typename T, int M, bool Q8>
+__device__ __forceinline__ void cache_append_cta(const AppendArgs& a, float* ki_s) {
   const int b = blockIdx.x;
   const int t = a.pos[b];
   if (t < 0) {
@@ -284,6 +286,16 @@ __global__ void __launch_bounds__(256) cache_append_kernel(AppendArgs a) {
     }
   }
   if (threadIdx.x == 0) a.cache_len[b] = i + 1;
+}
+
+// With a.wait_late the wait for the previous kernel comes after the append's
+// own work, so the kernel after it sees both complete.
+template <typename T, int M, bool Q8 = false>
+__global__ void __launch_bounds__(256) cache_append_kernel(AppendArgs a) {
+  __shared__ float ki_s[1024];
+  if (!a.wait_late) pdl_prologue_done();
+  cache_append_cta<T, M, Q8>(a, ki_s);
+  if (a.wait_late) pdl_prologue_done();
 }
 
 }  // namespace csa

@@ -1168,7 +1168,8 @@ int csa_ring_row_elems(const csa_dims* d) {
 namespace {
 csa_status launch_append(const csa_dims* d, const void* packed, const void* rows, long long ld_rows,
                          const int* pos, void* ring, void* Ccache, void* KIcache, int* cache_len, int cap,
-                         int B, cudaStream_t st, uint8_t* KIcodes = nullptr, float* KIscale = nullptr) {
+                         int B, cudaStream_t st, uint8_t* KIcodes = nullptr, float* KIscale = nullptr,
+                         bool wait_late = false) {
   CSA_RANGE("A6 cache_append");
   if (B == 0) return CSA_OK;
   const bool q8 = KIcodes != nullptr;
@@ -1182,6 +1183,7 @@ csa_status launch_append(const csa_dims* d, const void* packed, const void* rows
   a.BbI = reinterpret_cast<const float*>(at((void*)packed, P.bbI));
   a.c = d->c; a.cI = d->cI; a.cap = cap; a.ring_w = 4 * d->c + 4 * d->cI;
   a.KIcodes = KIcodes; a.KIscale = KIscale;
+  a.wait_late = wait_late ? 1 : 0;
 #define CSA_APPEND_CASE(MM)                                                                    \
   case MM: {                                                                                   \
     const cudaError_t e_ = q8 ? launch_pdl(cache_append_kernel<bf16, MM, true>, dim3(B), dim3(256), 0, st, a) \
@@ -1347,9 +1349,12 @@ csa_status decode_impl(const csa_dims* d, const void* packed, const void* h, con
   s = project_hidden(d, packed, h, B, y1, wI, st, reinterpret_cast<float*>(at(ws, L.split)),
                      L.total - L.split);
   if (s != CSA_OK || (s = mark(ev, 1, st)) != CSA_OK) return s;
-  s = launch_append(d, packed, y1, P.N1b, pos, ring, Ccache, KIcache, cache_len, cap, B, st, KIcodes, KIscale);
-  if (s != CSA_OK || (s = mark(ev, 2, st)) != CSA_OK) return s;
   s = project_query(d, packed, y1 + (size_t)(4 * c + 4 * cI) * es, P.N1b, B, y2, st);
+  if (s != CSA_OK || (s = mark(ev, 2, st)) != CSA_OK) return s;
+  // the append touches nothing the c^Q-side projection reads or writes: it runs beside it and
+  // waits for it at its end (the projection lets it start only once the H-side rows are complete)
+  s = launch_append(d, packed, y1, P.N1b, pos, ring, Ccache, KIcache, cache_len, cap, B, st, KIcodes, KIscale,
+                    /*wait_late=*/true);
   if (s != CSA_OK || (s = mark(ev, 3, st)) != CSA_OK) return s;
   IndexerArgs ia;
   ia.qI = y2; ia.ld_qI = P.N2; ia.wI = wI; ia.ld_wI = d->nhI; ia.KI = KIcache; ia.idx = idx;

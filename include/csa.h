@@ -19,7 +19,10 @@
  *    may start its on-chip set-up while the previous kernel on the stream
  *    finishes, but it waits for that kernel to complete before it reads or
  *    writes any memory, so the order of all memory effects is the stream
- *    order.
+ *    order.  The one exception is inside csa_decode / csa_decode_q8: the
+ *    cache append runs beside the c^Q-side projection of the same call,
+ *    whose buffers (workspace rows, packed weights) it does not touch; the
+ *    call as a whole keeps the stream order.
  *  - Matrices are dense row-major.  "ld" arguments are row strides in
  *    ELEMENTS.  Element type = csa_dims.dtype for activations and weights
  *    (fp32 or bf16); the indexer head weights w^I are always fp32 and block
@@ -383,8 +386,10 @@ csa_status csa_decode(const csa_dims* dims, const void* packed, const void* h, c
 /* csa_decode with stage timing: the same launches and results, plus a CUDA
  * event recorded on `stream` before the first stage (events[0]) and after
  * each stage: the H-side projection with its K-split reduction (1), the
- * cache append (2), the c^Q-side projection (3), the indexer scores (4),
- * the top-k selection (5) and the MQA (6).
+ * c^Q-side projection (2), the cache append (3), the indexer scores (4),
+ * the top-k selection (5) and the MQA (6).  (csa_decode runs the append
+ * beside the c^Q-side projection, which touches none of its buffers; the
+ * event between them serialises the two here.)
  * events [host] : 7 cudaEvent_t handles (passed as void*), created by the
  *                 caller; a NULL array or handle returns CSA_ERR_INVALID_ARG
  *                 before any launch.  Recording adds no kernel. */
