@@ -310,7 +310,7 @@ csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const vo
     g.out = out;
     g.k_split = 1;
     g.part = nullptr;
-    if (M >= 128) {  // activations as the M operand, 128 x BN tiles
+    if (M > 64) {  // activations as the M operand, 128 x BN tiles (rows past M read as zero, not stored)
       // BN = 192 where it fills the last wave and the padded columns better
       // (the packed weights are padded to 256 rows, so both widths stay in range)
       auto wave_eff = [&](int bn) {
@@ -354,8 +354,7 @@ csa_status launch_gemm(const csa_dims* d, const void* A, long long lda, const vo
         break;
       }
     }
-    if (M <= 64) return launch_tc_gemm<64, 8>(ta, tb, g, st);
-    return CSA_ERR_UNSUPPORTED;
+    return launch_tc_gemm<64, 8>(ta, tb, g, st);
   }
   SimtGemmArgs g{A, lda, B, ldb, M, N, K, out};
   dim3 grid((N + 127) / 128, (M + 127) / 128);

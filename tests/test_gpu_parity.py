@@ -68,6 +68,15 @@ def test_small_bf16_ragged():
     assert c["required"] >= 0.7 * (c["required"] + c["equal"] + c["valid"]), c   # oracle alone: 1067 of 1378
 
 
+def test_small_bf16_between_one_and_two_row_tiles():
+    """A packed batch of 100 tokens: more rows than the swapped decode GEMM
+    takes (64) and fewer than one 128-row tile of the prefill GEMM, whose rows
+    past the end read as zero and are not stored."""
+    lens = (37, 63)
+    c = e2e(SMALL_BF16, lens, seed=24, name="small bf16 T=100")
+    assert sum(c.values()) == sum(lens)
+
+
 def test_small_bf16_m2_fp32():
     e2e(csa.Dims(d=256, c=64, m=2, cI=32, nhI=8, nh=4, dc=128, topk=8, dtype=csa.CSA_F32), (77, 200), 22,
         name="m=2 fp32")
@@ -541,6 +550,13 @@ def test_decode_selection_of_rows_longer_than_shared_memory(avail):
     streamed form must pick the oracle's set."""
     dims = csa.Dims(d=256, c=128, m=4, cI=128, nhI=64, nh=4, dc=128, topk=64, dtype=csa.CSA_BF16)
     decode_case(dims, B=2, pos0=4 * avail + 1, cap=avail + 100, steps=2, seed=67, check=[0, 1])
+
+
+def test_decode_between_64_and_128_sequences():
+    """100 sequences: the decode projections run as 128-row prefill tiles
+    (the swapped form takes at most 64 rows) with the last 28 rows empty."""
+    dims = csa.Dims(d=256, c=128, m=4, cI=128, nhI=64, nh=4, dc=128, topk=16, dtype=csa.CSA_BF16)
+    decode_case(dims, B=100, pos0=301, cap=400, steps=4, seed=75, check=[0, 1, 50, 98, 99])
 
 
 def test_decode_projection_split_over_k():

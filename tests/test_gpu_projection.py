@@ -34,7 +34,7 @@ def check(got, want, dtype, what):
 
 
 @pytest.mark.parametrize("dtype", [csa.CSA_BF16, csa.CSA_F32])
-@pytest.mark.parametrize("T", [1, 37, 64, 129, 300])
+@pytest.mark.parametrize("T", [1, 37, 64, 65, 100, 127, 128, 129, 300])
 def test_projections(dtype, T):
     dims = csa.Dims(d=200 if dtype == csa.CSA_BF16 else 196, c=64, m=4, cI=32, nhI=16, nh=4, dc=192, topk=8,
                     dtype=dtype)
