@@ -960,6 +960,10 @@ csa_status forward_impl(const csa_dims* d, const void* packed, const void* H, co
   const FwdLayout L = fwd_layout(d, T);
   if (ws_bytes < L.total) return CSA_ERR_WORKSPACE;
   if (T == 0) return CSA_OK;
+  if (max_seqlen > T) max_seqlen = T;   // no sequence is longer than the batch
+  // the CUDA-core indexer holds a query's candidate scores in shared memory: a
+  // bound it cannot hold is refused here, before the first launch
+  if (!indexer_tc_ok(d) && indexer_smem(d, max_seqlen / d->m) > kMaxSmem) return CSA_ERR_UNSUPPORTED;
   const PackLayout P = pack_layout(d);
   cudaStream_t st = (cudaStream_t)stream;
   const size_t es = elem_size(d);
@@ -989,8 +993,7 @@ csa_status forward_impl(const csa_dims* d, const void* packed, const void* H, co
   ia.topk = d->topk; ia.nhI = d->nhI; ia.sc_cap = max_seqlen / d->m;
   ia.rm = RowMap{cu_seqlens, cu_blocks, nseq, NB, nullptr, 0, d->m};
   if (indexer_tc_ok(d)) {
-    if (max_seqlen > T) max_seqlen = T;   // scratch rows are sized for T / m blocks
-    ia.sc_cap = max_seqlen / d->m + 1;
+    ia.sc_cap = max_seqlen / d->m + 1;   // scratch rows are sized for T / m blocks
     s = launch_indexer_tc(d, ia, T, NB, at(ws, L.scratch), L.total - L.scratch, st);
   } else {
     s = launch_indexer(d, ia, T, st);
@@ -1127,6 +1130,7 @@ csa_status csa_cp_queries(const csa_dims* d, const void* packed, const void* Y1,
     if (reinterpret_cast<uintptr_t>(p) % 16) return CSA_ERR_INVALID_ARG;
   const CpLayout L = cp_layout(d, T, pos0 + T);
   if (ws_bytes < L.total) return CSA_ERR_WORKSPACE;
+  if (!indexer_tc_ok(d) && indexer_smem(d, (pos0 + T) / d->m) > kMaxSmem) return CSA_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
   const PackLayout P = pack_layout(d);
   const size_t es = elem_size(d);
@@ -1336,6 +1340,11 @@ csa_status decode_impl(const csa_dims* d, const void* packed, const void* h, con
   const DecLayout L = dec_layout(d, B, cap);
   if (ws_bytes < L.total) return CSA_ERR_WORKSPACE;
   if (B == 0) return CSA_OK;
+  const bool idx_tc = !q8 && d->dtype == CSA_BF16 && (d->nhI == 32 || d->nhI == 64) &&
+                      (d->cI == 64 || d->cI == 128) && reinterpret_cast<uintptr_t>(KIcache) % 16 == 0;
+  // the CUDA-core indexer holds a row of cap scores in shared memory: refused
+  // here, before the append changes any cache
+  if (!q8 && !idx_tc && indexer_smem(d, cap) > kMaxSmem) return CSA_ERR_UNSUPPORTED;
   const PackLayout P = pack_layout(d);
   cudaStream_t st = (cudaStream_t)stream;
   const size_t es = elem_size(d);
@@ -1362,8 +1371,7 @@ csa_status decode_impl(const csa_dims* d, const void* packed, const void* h, con
   if (q8) {
     s = launch_indexer_decode_q8(d, ia, KIcodes, KIscale, B, cap, reinterpret_cast<float*>(at(ws, L.scratch)),
                                  at(ws, L.qf16), st, ev ? (cudaEvent_t)ev[4] : nullptr);
-  } else if (d->dtype == CSA_BF16 && (d->nhI == 32 || d->nhI == 64) && (d->cI == 64 || d->cI == 128) &&
-             reinterpret_cast<uintptr_t>(KIcache) % 16 == 0) {
+  } else if (idx_tc) {
     s = launch_indexer_decode_tc(d, ia, B, cap, reinterpret_cast<float*>(at(ws, L.scratch)), st,
                                  ev ? (cudaEvent_t)ev[4] : nullptr);
   } else {

@@ -216,7 +216,11 @@ csa_status csa_project_hidden_compress(const csa_dims* dims, const void* packed,
  *             place a query or block outside total_tokens / total_blocks.
  * ws [dev]  : workspace of ws_bytes >= csa_indexer_workspace_bytes(), 256-byte
  *             aligned, no initialisation needed.
- * The score matrix is never written to memory. */
+ * The score matrix is never written to memory.  The tensor-core indexer runs
+ * for bf16 dims with m = 4, nhI in {32, 64} and cI in {64, 128}; otherwise
+ * the CUDA-core indexer holds each query's candidate scores in shared memory
+ * and requires 4 * (nhI*cI + nhI + 296 + floor(max_seqlen/m)) <= 227 KB
+ * (CSA_ERR_UNSUPPORTED before any launch otherwise). */
 csa_status csa_indexer_topk(const csa_dims* dims, const void* qI, int ld_qI, const float* wI,
                             int ld_wI, const void* KI, const int* cu_seqlens, const int* cu_blocks,
                             int nseq, int total_tokens, int total_blocks, int max_seqlen, int* idx,
@@ -275,7 +279,10 @@ size_t csa_forward_workspace_bytes(const csa_dims* dims, int total_tokens, int n
  * packed [dev]     : output of csa_pack_weights.
  * H [dev]          : [total_tokens, d] hidden states.
  * max_seqlen [host]: upper bound of every sequence length (as for
- *                    csa_indexer_topk).
+ *                    csa_indexer_topk); a bound above total_tokens is
+ *                    taken as total_tokens.  Where the CUDA-core indexer
+ *                    runs, its limit on floor(max_seqlen/m) (see
+ *                    csa_indexer_topk) is checked before any launch.
  * O [dev]          : [total_tokens, nh*c] attention outputs o_{t,i}.
  * Ccomp_out, KI_out, idx_out [dev, optional, may be NULL]: copies of
  *                    C^Comp [total_blocks, c], K^IComp [total_blocks, cI]
@@ -343,7 +350,9 @@ csa_status csa_cp_compress(const csa_dims* dims, const void* packed, const void*
  *               of the sequence; total_blocks >= (pos0 + T) / m.
  * O [dev]     : [T, nh*c];  idx_out [dev, optional]: [T, topk] (global
  *               block indices).
- * ws [dev]    : as for step 1. */
+ * ws [dev]    : as for step 1.
+ * Where the CUDA-core indexer runs, its limit (csa_indexer_topk) applies to
+ * (pos0 + T) / m and is checked before any launch. */
 csa_status csa_cp_queries(const csa_dims* dims, const void* packed, const void* Y1, const float* wI, int T,
                           int pos0, const void* Ccomp, const void* KIcomp, int total_blocks, void* O,
                           int* idx_out, void* ws, size_t ws_bytes, void* stream);
@@ -378,7 +387,11 @@ size_t csa_decode_workspace_bytes(const csa_dims* dims, int B, int cap);
 /* One decode step: each of B independent sequences gets one new token h_b
  * at position pos[b] and attends over its cached entries s < floor(t/m).
  * h [dev] : [B, d].  O [dev] : [B, nh*c].  idx_out [dev, optional] : [B, topk].
- * The caches, cache_len and ring are updated as by csa_cache_append. */
+ * The caches, cache_len and ring are updated as by csa_cache_append.
+ * Unless the tensor-core decode indexer runs (bf16, nhI in {32, 64}, cI in
+ * {64, 128}, KIcache 16-byte aligned), a row of cap scores must fit in one
+ * block's shared memory: 4 * (nhI*cI + nhI + 296 + cap) <= 227 KB, else
+ * CSA_ERR_UNSUPPORTED before any launch (no cache is changed). */
 csa_status csa_decode(const csa_dims* dims, const void* packed, const void* h, const int* pos,
                       void* ring, void* Ccache, void* KIcache, int* cache_len, int cap, int B,
                       void* O, int* idx_out, void* ws, size_t ws_bytes, void* stream);

@@ -129,6 +129,29 @@ def test_decode_workspace_too_small_rejected():
     assert csa.csa_launch_count() == n0
 
 
+def test_indexer_row_limit_refused_before_any_launch():
+    """The CUDA-core indexer (fp32 here) keeps a query's candidate scores in
+    shared memory.  A forward whose longest sequence, a decode step whose cache
+    capacity, or a context-parallel chunk whose prefix needs more than one
+    block's shared memory is refused with CSA_ERR_UNSUPPORTED before anything
+    is launched: in particular before the decode append changes a cache.
+    (Only refusals are exercised: the addresses are fake.)"""
+    L = csa.lib()
+    d = ctypes.byref(TINY.c_struct())
+    p = ctypes.c_void_p(1 << 20)
+    n0 = csa.csa_launch_count()
+    T = 300_000            # 75000 blocks of fp32 scores: more than 227 KB
+    ws = csa.csa_forward_workspace_bytes(TINY, T, 1)
+    assert L.csa_forward(d, p, p, p, p, 1, T, T // 4, T, p, None, None, None, p, ws, None) == 2
+    cap = 100_000
+    ws = csa.csa_decode_workspace_bytes(TINY, 3, cap)
+    assert L.csa_decode(d, p, p, p, p, p, p, p, cap, 3, p, None, p, ws, None) == 2
+    ws = csa.csa_cp_workspace_bytes(TINY, 4096, T)
+    assert ws > 0
+    assert L.csa_cp_queries(d, p, p, p, 4096, T - 4096, p, p, T // 4, p, None, p, ws, None) == 2
+    assert csa.csa_launch_count() == n0
+
+
 def test_decode_workspace_holds_scores_and_split_sums():
     """The decode workspace covers the [B, cap] fp32 scores and the four fp32
     K-slices of the hidden-side projection ([slice][token][feature], features
